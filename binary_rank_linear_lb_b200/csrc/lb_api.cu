@@ -1,0 +1,542 @@
+// Host side of liblb.so: argument validation, workspace layout, plan building
+// and launches for every entry point declared in include/lb.h.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lb_internal.cuh"
+
+namespace lb {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+int g_sm_count[kMaxDevices];
+int g_cc_major[kMaxDevices];
+cudaError_t g_cfg_err[kMaxDevices];
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+void init_device(int d) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, d) != cudaSuccess) {
+        g_cfg_err[d] = cudaErrorInvalidDevice;
+        return;
+    }
+    g_sm_count[d] = prop.multiProcessorCount;
+    g_cc_major[d] = prop.major;
+    g_cfg_err[d] = prop.major == 10 ? decode_configure() : cudaErrorInvalidDeviceFunction;
+}
+
+// Returns LB_OK when the current device is an sm_100 part and the kernels are configured.
+lb_status ensure_device() {
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return LB_ERR_CUDA;
+    std::call_once(g_dev_once[d], init_device, d);
+    if (g_cc_major[d] != 10) return LB_ERR_UNSUPPORTED;
+    return g_cfg_err[d] == cudaSuccess ? LB_OK : LB_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int vec_kind_for(lb_dtype t) {
+    switch (t) {
+        case LB_F16: return VK_X_F16;
+        case LB_BF16: return VK_X_BF16;
+        default: return VK_X_F32;
+    }
+}
+
+// Fill the size fields of a job whose matrix has `rows` packed rows of `cols` signs.
+void set_job_shape(LbJob& J, int64_t rows, int64_t cols) {
+    J.rows = (int)rows;
+    J.cols = (int)cols;
+    J.ldw = (int)cdiv(cols, 32);
+    J.n_slices = (int)cdiv(cols, kSliceElems);
+    J.n_rowblocks = (int)cdiv(rows, kRowBlock);
+}
+
+// Append `J` to phase `ph`, assigning its unit range.
+void add_job(LbPhase& ph, std::vector<LbJob>& jobs, LbJob J) {
+    J.unit_begin = ph.n_units;
+    ph.n_units += J.n_slices * J.n_rowblocks;
+    ph.n_jobs += 1;
+    jobs.push_back(J);
+}
+
+bool branch_ok(const lb_branch& b) {
+    return b.Vp && b.Up && b.h && b.g && b.l;
+}
+bool branch_aligned(const lb_branch& b) {
+    return aligned(b.Vp, 16) && aligned(b.Up, 16) && aligned(b.h, 2) && aligned(b.g, 2) &&
+           aligned(b.l, 2);
+}
+
+// ------------------------------------------------------------ stack layout
+struct StackLayout {
+    size_t sumsq;                 // [n_layers][2] floats
+    size_t t;                     // first t accumulator
+    std::vector<size_t> t_off;    // [layer][proj][branch]
+    std::vector<size_t> o_off;    // [layer][proj] output accumulators (q,k,v,gate,up), else 0
+    size_t acc_end;               // end of the region zeroed per call
+    size_t x_dev, y_dev;          // staging for lb_stack_forward_host
+    size_t phases, jobs;          // plan
+    int n_phases, n_jobs;
+    size_t total;
+};
+
+bool stack_desc_ok(const lb_stack_desc* d) {
+    if (!d || !d->lin || !d->ranks) return false;
+    if (d->n_layers <= 0 || d->hidden <= 0 || d->inter <= 0) return false;
+    if (d->n_branches < 1 || d->n_branches > 2) return false;
+    const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
+    if (d->flags & ~LB_STACK_MLP_ONLY) return false;
+    if (mlp_only) {
+        if (d->n_layers != 1) return false;
+    } else {
+        if (d->n_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0) return false;
+        if ((int64_t)d->n_heads * d->head_dim != d->hidden) return false;
+        if (d->n_heads % d->n_kv_heads != 0) return false;
+    }
+    for (int L = 0; L < d->n_layers; ++L)
+        for (int p = 0; p < LB_N_PROJ; ++p) {
+            const bool used = !mlp_only || p >= LB_GATE;
+            if (!used) continue;
+            if (d->ranks[L * LB_N_PROJ + p] <= 0 || d->ranks[L * LB_N_PROJ + p] > (1 << 24))
+                return false;
+            for (int b = 0; b < d->n_branches; ++b)
+                if (!branch_ok(d->lin[(L * LB_N_PROJ + p) * d->n_branches + b])) return false;
+        }
+    return true;
+}
+
+// in / out features of projection p.
+void proj_shape(const lb_stack_desc* d, int p, int64_t& in, int64_t& out) {
+    const int64_t kv = (int64_t)d->n_kv_heads * d->head_dim;
+    switch (p) {
+        case LB_Q: in = d->hidden; out = d->hidden; break;
+        case LB_K: case LB_V: in = d->hidden; out = kv; break;
+        case LB_O: in = d->hidden; out = d->hidden; break;
+        case LB_GATE: case LB_UP: in = d->hidden; out = d->inter; break;
+        default: in = d->inter; out = d->hidden; break;
+    }
+}
+
+bool proj_used(const lb_stack_desc* d, int p) {
+    return !(d->flags & LB_STACK_MLP_ONLY) || p >= LB_GATE;
+}
+
+StackLayout stack_layout(const lb_stack_desc* d) {
+    StackLayout L;
+    const int nl = d->n_layers, nb = d->n_branches;
+    size_t off = sizeof(WsHeader);
+    L.sumsq = off;
+    off = round_up(off + sizeof(float) * 2 * nl, 256);
+    L.t = off;
+    L.t_off.assign((size_t)nl * LB_N_PROJ * nb, 0);
+    L.o_off.assign((size_t)nl * LB_N_PROJ, 0);
+    for (int l = 0; l < nl; ++l)
+        for (int p = 0; p < LB_N_PROJ; ++p) {
+            if (!proj_used(d, p)) continue;
+            const int64_t r = d->ranks[l * LB_N_PROJ + p];
+            for (int b = 0; b < nb; ++b) {
+                L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b] = off;
+                off = round_up(off + sizeof(float) * (size_t)r, 256);
+            }
+        }
+    for (int l = 0; l < nl; ++l)
+        for (int p = 0; p < LB_N_PROJ; ++p) {
+            if (!proj_used(d, p) || p == LB_O || p == LB_DOWN) continue;
+            int64_t in, out;
+            proj_shape(d, p, in, out);
+            L.o_off[(size_t)l * LB_N_PROJ + p] = off;
+            off = round_up(off + sizeof(float) * (size_t)out, 256);
+        }
+    L.acc_end = off;
+    L.x_dev = off;
+    off = round_up(off + 2 * (size_t)d->hidden, 256);
+    L.y_dev = off;
+    off = round_up(off + 4 * (size_t)d->hidden, 256);
+    const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
+    L.n_phases = mlp_only ? 4 : 8 * nl;
+    // jobs: per layer 2*(3+1+2+1)*nb = 14 nb (decoder); 2*(2+1)*nb = 6 nb (MLP only)
+    L.n_jobs = mlp_only ? 6 * nb : 14 * nb * nl;
+    L.phases = off;
+    off = round_up(off + sizeof(LbPhase) * (size_t)L.n_phases, 256);
+    L.jobs = off;
+    off = round_up(off + sizeof(LbJob) * (size_t)L.n_jobs, 256);
+    L.total = off;
+    return L;
+}
+
+// Build the phase program of a stack (host copies; pointers into `ws`).
+void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
+                      std::vector<LbPhase>& phases, std::vector<LbJob>& jobs) {
+    const int nb = d->n_branches;
+    const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
+    auto br = [&](int l, int p, int b) -> const lb_branch& {
+        return d->lin[((size_t)l * LB_N_PROJ + p) * nb + b];
+    };
+    auto tptr = [&](int l, int p, int b) {
+        return reinterpret_cast<float*>(ws + L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b]);
+    };
+    auto optr = [&](int l, int p) {
+        return reinterpret_cast<float*>(ws + L.o_off[(size_t)l * LB_N_PROJ + p]);
+    };
+    float* sumsq = reinterpret_cast<float*>(ws + L.sumsq);
+    float* yres = const_cast<float*>(reinterpret_cast<const float*>(LB_TAG_Y));
+
+    auto new_phase = [&]() {
+        LbPhase ph = {};
+        ph.job_begin = (int)jobs.size();
+        return ph;
+    };
+    // First contraction of projection p of layer l over vector source (kind, src...).
+    auto stage1 = [&](LbPhase& ph, int l, int p, int kind, const void* src, const float* src2,
+                      float* acc_sumsq, float* resid_init, int b) {
+        int64_t in, out;
+        proj_shape(d, p, in, out);
+        const int64_t r = d->ranks[l * LB_N_PROJ + p];
+        LbJob J = {};
+        J.P = br(l, p, b).Vp;
+        set_job_shape(J, r, in);
+        J.kind = kind;
+        J.src = src;
+        J.src2 = src2;
+        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).g);
+        J.out = tptr(l, p, b);
+        J.acc_sumsq = acc_sumsq;
+        J.resid_init = resid_init;
+        J.gqa_hd = d->head_dim;
+        J.gqa_ghd = d->n_kv_heads > 0 ? d->head_dim * (d->n_heads / d->n_kv_heads) : 1;
+        add_job(ph, jobs, J);
+    };
+    auto stage2 = [&](LbPhase& ph, int l, int p, float* out_ptr, const float* norm, int b) {
+        int64_t in, out;
+        proj_shape(d, p, in, out);
+        const int64_t r = d->ranks[l * LB_N_PROJ + p];
+        LbJob J = {};
+        J.P = br(l, p, b).Up;
+        set_job_shape(J, out, r);
+        J.kind = VK_T;
+        J.src = tptr(l, p, b);
+        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).l);
+        J.oscale = reinterpret_cast<const __half*>(br(l, p, b).h);
+        J.out = out_ptr;
+        J.norm_sumsq = norm;
+        J.norm_n = d->hidden;
+        add_job(ph, jobs, J);
+    };
+
+    if (mlp_only) {
+        LbPhase p0 = new_phase();
+        for (int p : {LB_GATE, LB_UP})
+            for (int b = 0; b < nb; ++b)
+                stage1(p0, 0, p, VK_X_BF16, LB_TAG_X, nullptr, nullptr, nullptr, b);
+        p0.zero_ptr = yres;
+        p0.zero_n = d->hidden;
+        phases.push_back(p0);
+        LbPhase p1 = new_phase();
+        for (int p : {LB_GATE, LB_UP})
+            for (int b = 0; b < nb; ++b) stage2(p1, 0, p, optr(0, p), nullptr, b);
+        phases.push_back(p1);
+        LbPhase p2 = new_phase();
+        for (int b = 0; b < nb; ++b)
+            stage1(p2, 0, LB_DOWN, VK_SILU_MUL, optr(0, LB_GATE), optr(0, LB_UP), nullptr,
+                   nullptr, b);
+        phases.push_back(p2);
+        LbPhase p3 = new_phase();
+        for (int b = 0; b < nb; ++b) stage2(p3, 0, LB_DOWN, yres, nullptr, b);
+        phases.push_back(p3);
+        return;
+    }
+
+    for (int l = 0; l < d->n_layers; ++l) {
+        float* ss_attn = sumsq + 2 * l;
+        float* ss_mlp = sumsq + 2 * l + 1;
+        // q, k, v first contractions: input rmsnorm(h); layer 0 reads x and seeds h.
+        LbPhase a = new_phase();
+        bool first = true;
+        for (int p : {LB_Q, LB_K, LB_V})
+            for (int b = 0; b < nb; ++b) {
+                if (l == 0)
+                    stage1(a, l, p, VK_X_BF16, LB_TAG_X, nullptr, first ? ss_attn : nullptr,
+                           first ? yres : nullptr, b);
+                else
+                    stage1(a, l, p, VK_X_F32, LB_TAG_Y, nullptr, first ? ss_attn : nullptr,
+                           nullptr, b);
+                first = false;
+            }
+        phases.push_back(a);
+        LbPhase bq = new_phase();
+        for (int p : {LB_Q, LB_K, LB_V})
+            for (int b = 0; b < nb; ++b) stage2(bq, l, p, optr(l, p), ss_attn, b);
+        phases.push_back(bq);
+        LbPhase c = new_phase();
+        for (int b = 0; b < nb; ++b)
+            stage1(c, l, LB_O, VK_GQA, optr(l, LB_V), nullptr, nullptr, nullptr, b);
+        phases.push_back(c);
+        LbPhase e = new_phase();
+        for (int b = 0; b < nb; ++b) stage2(e, l, LB_O, yres, nullptr, b);
+        phases.push_back(e);
+        LbPhase f = new_phase();
+        first = true;
+        for (int p : {LB_GATE, LB_UP})
+            for (int b = 0; b < nb; ++b) {
+                stage1(f, l, p, VK_X_F32, LB_TAG_Y, nullptr, first ? ss_mlp : nullptr, nullptr,
+                       b);
+                first = false;
+            }
+        phases.push_back(f);
+        LbPhase g = new_phase();
+        for (int p : {LB_GATE, LB_UP})
+            for (int b = 0; b < nb; ++b) stage2(g, l, p, optr(l, p), ss_mlp, b);
+        phases.push_back(g);
+        LbPhase h = new_phase();
+        for (int b = 0; b < nb; ++b)
+            stage1(h, l, LB_DOWN, VK_SILU_MUL, optr(l, LB_GATE), optr(l, LB_UP), nullptr,
+                   nullptr, b);
+        phases.push_back(h);
+        LbPhase k = new_phase();
+        for (int b = 0; b < nb; ++b) stage2(k, l, LB_DOWN, yres, nullptr, b);
+        phases.push_back(k);
+    }
+}
+
+}  // namespace
+
+int device_sm_count() {
+    const int d = current_device();
+    return (d >= 0 && d < kMaxDevices) ? g_sm_count[d] : 0;
+}
+
+bool device_is_sm100() {
+    const int d = current_device();
+    return d >= 0 && d < kMaxDevices && g_cc_major[d] == 10;
+}
+
+}  // namespace lb
+
+using namespace lb;
+
+extern "C" {
+
+const char* lb_status_string(lb_status s) {
+    switch (s) {
+        case LB_OK: return "LB_OK";
+        case LB_ERR_INVALID_ARG: return "LB_ERR_INVALID_ARG";
+        case LB_ERR_ALIGNMENT: return "LB_ERR_ALIGNMENT";
+        case LB_ERR_UNSUPPORTED: return "LB_ERR_UNSUPPORTED";
+        case LB_ERR_CUDA: return "LB_ERR_CUDA";
+        case LB_ERR_TIMEOUT: return "LB_ERR_TIMEOUT";
+        case LB_ERR_WORKSPACE: return "LB_ERR_WORKSPACE";
+        default: return "LB_ERR_UNKNOWN";
+    }
+}
+
+int lb_version(void) { return 100; }
+
+lb_status lb_pack_signs(const float* latent, int64_t rows, int64_t cols, int64_t ld, int axis,
+                        uint32_t* packed, int64_t ld_words, void* stream) {
+    if (!latent || !packed || rows <= 0 || cols <= 0 || ld < cols) return LB_ERR_INVALID_ARG;
+    if (axis != 0 && axis != 1) return LB_ERR_INVALID_ARG;
+    const int64_t k = axis == 1 ? cols : rows;
+    if (ld_words < cdiv(k, 32)) return LB_ERR_INVALID_ARG;
+    if (!aligned(latent, 4) || !aligned(packed, 4)) return LB_ERR_ALIGNMENT;
+    const lb_status st = ensure_device();
+    if (st != LB_OK) return st;
+    return launch_pack(latent, rows, cols, ld, axis, packed, ld_words,
+                       static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? LB_OK
+               : LB_ERR_CUDA;
+}
+
+size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r, int n_branches) {
+    (void)in;
+    (void)out;
+    if (M <= 0 || r <= 0 || n_branches < 1 || n_branches > 2) return 0;
+    const int64_t mc = std::min<int64_t>(M, kMaxDecodeM);
+    return sizeof(WsHeader) + round_up(sizeof(float) * (size_t)(mc * n_branches * r), 256);
+}
+
+int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r) {
+    (void)M;
+    (void)in;
+    (void)out;
+    (void)r;
+    return 0;
+}
+
+lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t in, int64_t out,
+                            int64_t r, const lb_branch* br, int n_branches, float* y,
+                            void* workspace, size_t ws_bytes, void* stream) {
+    if (!x || !y || !br || !workspace) return LB_ERR_INVALID_ARG;
+    if (M <= 0 || in <= 0 || out <= 0 || r <= 0) return LB_ERR_INVALID_ARG;
+    if (in > (1 << 28) || out > (1 << 28) || r > (1 << 24)) return LB_ERR_INVALID_ARG;
+    if (n_branches < 1 || n_branches > 2) return LB_ERR_INVALID_ARG;
+    if (x_dtype != LB_F16 && x_dtype != LB_BF16 && x_dtype != LB_F32) return LB_ERR_INVALID_ARG;
+    for (int b = 0; b < n_branches; ++b)
+        if (!branch_ok(br[b])) return LB_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(workspace, 16)) return LB_ERR_ALIGNMENT;
+    for (int b = 0; b < n_branches; ++b)
+        if (!branch_aligned(br[b])) return LB_ERR_ALIGNMENT;
+    if (ws_bytes < lb_linear_workspace_size(M, in, out, r, n_branches)) return LB_ERR_WORKSPACE;
+    lb_status st = ensure_device();
+    if (st != LB_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xsz = x_dtype == LB_F32 ? 4 : 2;
+    WsHeader* hdr = static_cast<WsHeader*>(workspace);
+    float* t = reinterpret_cast<float*>(static_cast<char*>(workspace) + sizeof(WsHeader));
+    for (int64_t m0 = 0; m0 < M; m0 += kMaxDecodeM) {
+        const int mc = (int)std::min<int64_t>(kMaxDecodeM, M - m0);
+        LinearPlan plan;
+        std::memset(&plan, 0, sizeof(plan));
+        std::vector<LbJob> jobs;
+        jobs.reserve(2 * kMaxLinearJobs);
+        LbPhase p0 = {};
+        p0.job_begin = 0;
+        for (int m = 0; m < mc; ++m)
+            for (int b = 0; b < n_branches; ++b) {
+                LbJob J = {};
+                J.P = br[b].Vp;
+                set_job_shape(J, r, in);
+                J.kind = vec_kind_for(x_dtype);
+                J.src = static_cast<const char*>(x) + (size_t)(m0 + m) * (size_t)in * xsz;
+                J.vscale = reinterpret_cast<const __half*>(br[b].g);
+                J.out = t + ((size_t)m * n_branches + b) * (size_t)r;
+                add_job(p0, jobs, J);
+            }
+        p0.zero_ptr = y + (size_t)m0 * (size_t)out;
+        p0.zero_n = (int)(mc * out);
+        LbPhase p1 = {};
+        p1.job_begin = (int)jobs.size();
+        for (int m = 0; m < mc; ++m)
+            for (int b = 0; b < n_branches; ++b) {
+                LbJob J = {};
+                J.P = br[b].Up;
+                set_job_shape(J, out, r);
+                J.kind = VK_T;
+                J.src = t + ((size_t)m * n_branches + b) * (size_t)r;
+                J.vscale = reinterpret_cast<const __half*>(br[b].l);
+                J.oscale = reinterpret_cast<const __half*>(br[b].h);
+                J.out = y + (size_t)(m0 + m) * (size_t)out;
+                add_job(p1, jobs, J);
+            }
+        if ((int64_t)mc * out > 0x7fffffff) return LB_ERR_INVALID_ARG;
+        plan.phases[0] = p0;
+        plan.phases[1] = p1;
+        std::copy(jobs.begin(), jobs.end(), plan.jobs);
+        const size_t zero_bytes = sizeof(WsHeader) + sizeof(float) * (size_t)mc * n_branches * r;
+        if (cudaMemsetAsync(workspace, 0, zero_bytes, s) != cudaSuccess) return LB_ERR_CUDA;
+        if (launch_linear_plan(plan, hdr, 2, s) != cudaSuccess) return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+size_t lb_stack_workspace_size(const lb_stack_desc* d) {
+    if (!stack_desc_ok(d)) return 0;
+    return stack_layout(d).total;
+}
+
+lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    if (!stack_desc_ok(d) || !workspace) return LB_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return LB_ERR_ALIGNMENT;
+    const int nb = d->n_branches;
+    for (int l = 0; l < d->n_layers; ++l)
+        for (int p = 0; p < LB_N_PROJ; ++p) {
+            if (!proj_used(d, p)) continue;
+            for (int b = 0; b < nb; ++b)
+                if (!branch_aligned(d->lin[((size_t)l * LB_N_PROJ + p) * nb + b]))
+                    return LB_ERR_ALIGNMENT;
+        }
+    const StackLayout L = stack_layout(d);
+    if (ws_bytes < L.total) return LB_ERR_WORKSPACE;
+    lb_status st = ensure_device();
+    if (st != LB_OK) return st;
+    std::vector<LbPhase> phases;
+    std::vector<LbJob> jobs;
+    build_stack_plan(d, L, static_cast<char*>(workspace), phases, jobs);
+    if ((int)phases.size() != L.n_phases || (int)jobs.size() != L.n_jobs) return LB_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    if (cudaMemcpyAsync(ws + L.phases, phases.data(), sizeof(LbPhase) * phases.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return LB_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + L.jobs, jobs.data(), sizeof(LbJob) * jobs.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return LB_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
+    return LB_OK;
+}
+
+lb_status lb_stack_forward(const lb_stack_desc* d, void* workspace, size_t ws_bytes,
+                           const void* x, float* y, void* stream) {
+    if (!stack_desc_ok(d) || !workspace || !x || !y) return LB_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(x, 16) || !aligned(y, 16)) return LB_ERR_ALIGNMENT;
+    const StackLayout L = stack_layout(d);
+    if (ws_bytes < L.total) return LB_ERR_WORKSPACE;
+    lb_status st = ensure_device();
+    if (st != LB_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
+    if (launch_stack_plan(reinterpret_cast<const LbPhase*>(ws + L.phases),
+                          reinterpret_cast<const LbJob*>(ws + L.jobs), L.n_phases,
+                          reinterpret_cast<WsHeader*>(ws), x, y, s) != cudaSuccess)
+        return LB_ERR_CUDA;
+    return LB_OK;
+}
+
+lb_status lb_stack_forward_host(const lb_stack_desc* d, void* workspace, size_t ws_bytes,
+                                const void* x_host, float* y_host, void* stream) {
+    if (!stack_desc_ok(d) || !workspace || !x_host || !y_host) return LB_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return LB_ERR_ALIGNMENT;
+    const StackLayout L = stack_layout(d);
+    if (ws_bytes < L.total) return LB_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    void* xd = ws + L.x_dev;
+    float* yd = reinterpret_cast<float*>(ws + L.y_dev);
+    if (cudaMemcpyAsync(xd, x_host, 2 * (size_t)d->hidden, cudaMemcpyHostToDevice, s) !=
+        cudaSuccess)
+        return LB_ERR_CUDA;
+    lb_status st = lb_stack_forward(d, workspace, ws_bytes, xd, yd, stream);
+    if (st != LB_OK) return st;
+    if (cudaMemcpyAsync(y_host, yd, 4 * (size_t)d->hidden, cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return LB_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
+    return LB_OK;
+}
+
+lb_status lb_workspace_status(const void* workspace, void* stream) {
+    if (!workspace) return LB_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
+    int err = 0;
+    if (cudaMemcpy(&err, &static_cast<const WsHeader*>(workspace)->error, sizeof(int),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LB_ERR_CUDA;
+    return err == 0 ? LB_OK : LB_ERR_TIMEOUT;
+}
+
+const float* lb_stack_output(const lb_stack_desc* d, const void* workspace, int layer, int proj) {
+    if (!stack_desc_ok(d) || !workspace) return nullptr;
+    if (layer < 0 || layer >= d->n_layers || proj < 0 || proj >= LB_N_PROJ) return nullptr;
+    if (!proj_used(d, proj) || proj == LB_O || proj == LB_DOWN) return nullptr;
+    const StackLayout L = stack_layout(d);
+    return reinterpret_cast<const float*>(static_cast<const char*>(workspace) +
+                                          L.o_off[(size_t)layer * LB_N_PROJ + proj]);
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+// Internal declarations shared by the CUDA sources of liblb.so.
+//
+// The decode path is a persistent "phase program": a list of phases, each a
+// set of GEMV jobs out[row] (+)= oscale[row] * sum_col sign(P[row][col]) * v[col]
+// over packed sign matrices P, separated by grid-wide waits.  One linear is two
+// phases (the V contraction, then the U contraction); a decoder layer is eight.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/lb.h"
+
+namespace lb {
+
+// ---------------------------------------------------------------- constants
+constexpr int kDecodeThreads = 512;          // 16 warps per CTA, one CTA per SM
+constexpr int kDecodeWarps = kDecodeThreads / 32;
+constexpr int kSliceElems = 1024;            // columns covered by one lookup table
+constexpr int kSliceWords = kSliceElems / 32;
+constexpr int kRowBlock = 32;                // rows per warp work item (8 steps x 4 rows)
+constexpr int kLutBytes = 128 * 1024;        // 128 chunks x 256 entries x fp32
+constexpr int kStageBytes = 8 * 1024;        // staged vector slice + scratch
+constexpr int kDecodeSmem = 64 * 1024 + kLutBytes + kStageBytes;  // worst-case alignment
+constexpr int kMaxLinearJobs = 16;           // per phase in a single-linear call
+constexpr int kMaxDecodeM = 8;               // rows of x the decode path takes at once
+constexpr float kRmsEps = 1e-5f;
+
+// Workspace header (first 256 bytes of every workspace).
+struct WsHeader {
+    unsigned int barrier;     // grid barrier arrival counter (zeroed per call)
+    int error;                // 0 or LB_ERR_TIMEOUT (zeroed per call)
+    unsigned int exit_count;
+    int pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header must be 256 bytes");
+
+// Where a job's vector v[col] comes from.
+enum VecKind : int {
+    VK_X_F16 = 0,      // v = g[j] * x[j], x fp16
+    VK_X_BF16 = 1,     // v = g[j] * x[j], x bf16
+    VK_X_F32 = 2,      // v = g[j] * x[j], x fp32
+    VK_T = 3,          // v = l[k] * t[k] * rs, rs = rsqrt(sumsq/n + eps) or 1
+    VK_GQA = 4,        // v = g[j] * src[(j / (group*hd)) * hd + j % hd]
+    VK_SILU_MUL = 5,   // v = g[j] * silu(src[j]) * src2[j]
+};
+
+struct LbJob {
+    const uint32_t* P;        // packed rows [rows][ldw]
+    const void* src;          // vector source
+    const float* src2;        // second source (VK_SILU_MUL)
+    const __half* vscale;     // g (first contraction) or l (second)
+    const __half* oscale;     // h (second contraction) or nullptr
+    float* out;               // fp32 accumulation target [rows], zeroed beforehand
+    const float* norm_sumsq;  // VK_T: sum of squares of the normed input, or nullptr
+    float* acc_sumsq;         // owner of a slice adds sum(src^2) of the slice here
+    float* resid_init;        // owner of a slice writes float(src) of the slice here
+    int rows, cols, ldw, kind;
+    int n_slices, n_rowblocks, unit_begin, norm_n;
+    int gqa_ghd, gqa_hd, pad0, pad1;
+};
+
+struct LbPhase {
+    int job_begin, n_jobs, n_units, zero_n;
+    float* zero_ptr;          // if set, the CTAs zero zero_n floats here during the phase
+    long long pad;
+};
+
+// Stack plans are prepared once and reused with different x / y buffers, so
+// job pointers that mean "the call's x" or "the call's y" are stored as tags.
+#define LB_TAG_X ((const void*)1)
+#define LB_TAG_Y ((const void*)2)
+
+// Plan of a single linear call, passed by value as a kernel parameter.
+struct LinearPlan {
+    LbPhase phases[2];
+    LbJob jobs[2 * kMaxLinearJobs];
+};
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint4 ld_stream_v4(const uint32_t* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" :: "l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ float lds_f32(uint32_t saddr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr));
+    return v;
+}
+
+// ------------------------------------------------------------ host helpers
+int device_sm_count();               // SMs of the current device (cached per device)
+bool device_is_sm100();
+cudaError_t decode_configure();      // one-time kernel attribute setup per device
+
+// Decode phase program launches (lb_decode.cu).
+cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,
+                               cudaStream_t s);
+cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, int n_phases,
+                              WsHeader* hdr, const void* x, float* y, cudaStream_t s);
+
+// Packer (lb_pack.cu).
+cudaError_t launch_pack(const float* latent, int64_t rows, int64_t cols, int64_t ld, int axis,
+                        uint32_t* packed, int64_t ld_words, cudaStream_t s);
+
+}  // namespace lb

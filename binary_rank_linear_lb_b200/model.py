@@ -1,0 +1,83 @@
+"""Device-resident factorised linears and decoder stacks built from seeded inputs.
+
+Each branch is generated from its own seeds (``synth``) and binarised on the GPU
+with ``lb_pack_signs``; the fp32 latents are dropped right after packing.
+
+``signs="bits"`` instead draws the packed words directly from a uniform bit
+source.  The signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so the
+packed matrices have the same distribution; this only shortens the set-up of
+the largest stacks (whose latents would be hundreds of GB of fp32) and is never
+used where a result is compared with the oracle.
+"""
+from __future__ import annotations
+
+from typing import List, Optional
+
+import torch
+
+from . import Branch, Stack, pack_signs, synth
+from .configs import Model, proj_shape
+
+
+def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int, branch: int,
+                 device="cuda", signs: str = "latent") -> Branch:
+    s = lambda k: synth.tensor_seed(base, layer, proj, branch, k)
+    h = synth.scale(out_f, s(synth.KIND_H), device)
+    g = synth.scale(in_f, s(synth.KIND_G), device)
+    l = synth.scale(r, s(synth.KIND_L), device)
+    if signs == "latent":
+        V = synth.latent(in_f, r, s(synth.KIND_V), device)
+        Vp = pack_signs(V, axis=0)
+        del V
+        U = synth.latent(out_f, r, s(synth.KIND_U), device)
+        Up = pack_signs(U, axis=1)
+        del U
+    elif signs == "bits":
+        def words(n_rows, k, seed):
+            gen = torch.Generator(device=device)
+            gen.manual_seed(seed)
+            ldw = (k + 31) // 32
+            w = torch.randint(-2 ** 31, 2 ** 31, (n_rows, ldw), generator=gen, device=device,
+                              dtype=torch.int64).to(torch.int32)
+            if k % 32:
+                w[:, -1] &= (1 << (k % 32)) - 1
+            return w
+        Vp = words(r, in_f, s(synth.KIND_V))
+        Up = words(out_f, r, s(synth.KIND_U))
+    else:
+        raise ValueError(signs)
+    return Branch(Vp, Up, h, g, l)
+
+
+def build_linear(in_f: int, out_f: int, r: int, base: int = 0, layer: int = 0, proj: int = 0,
+                 n_branches: int = 2, device="cuda", signs: str = "latent") -> List[Branch]:
+    return [build_branch(in_f, out_f, r, base, layer, proj, b, device, signs)
+            for b in range(n_branches)]
+
+
+def build_stack(model: Model, bpw: float, base: int = 0, n_layers: Optional[int] = None,
+                n_branches: int = 2, device="cuda", signs: str = "latent",
+                ranks: Optional[List[int]] = None) -> Stack:
+    nl = n_layers or model.n_layers
+    rk = ranks or model.ranks(bpw)
+    linears, all_ranks = [], []
+    for li in range(nl):
+        L = []
+        for p in range(7):
+            i, o = proj_shape(p, model.hidden, model.inter, model.kv_dim)
+            L.append(build_linear(i, o, rk[p], base, li, p, n_branches, device, signs))
+        linears.append(L)
+        all_ranks.append(list(rk))
+    return Stack(linears, all_ranks, model.hidden, model.inter, model.n_heads, model.n_kv_heads,
+                 model.head_dim, device=device)
+
+
+def build_mlp_block(model: Model, bpw: float, base: int = 0, n_branches: int = 2,
+                    device="cuda", signs: str = "latent",
+                    ranks: Optional[List[int]] = None) -> Stack:
+    rk = ranks or model.ranks(bpw)
+    L: list = [None] * 7
+    for p in (4, 5, 6):
+        i, o = proj_shape(p, model.hidden, model.inter, model.kv_dim)
+        L[p] = build_linear(i, o, rk[p], base, 0, p, n_branches, device, signs)
+    return Stack([L], [list(rk)], model.hidden, model.inter, mlp_only=True, device=device)

@@ -1,0 +1,195 @@
+/*
+ * lb.h — C ABI of liblb.so, a B200 (sm_100a) implementation of the inference
+ * forward of the LittleBit factorised binary linear layer.
+ *
+ * The layer ("Samsung LittleBit: A 13B LLM Under 1 GB, and What the Paper
+ * Really Shows", section "How it works", items 1-3):
+ *
+ *   y = sum_{b in {primary, residual}} h_b o ( sign(U_b) . ( l_b o ( sign(V_b)^T . ( g_b o x ) ) ) )
+ *
+ *   U_b : out x r and V_b : in x r are latent factors of which only the signs
+ *         are kept at inference (item 1: "uses only their signs, +1 or -1");
+ *   h_b (out), g_b (in), l_b (r) are FP16 scale vectors along the rows, the
+ *         columns and the latent dimension of W (item 2);
+ *   b runs over a primary and a residual branch whose outputs are summed
+ *         (item 3, and the figure of the two-branch layer beside it).
+ *   sign(v) = -1 for v < 0 and +1 otherwise, so sign(0) = sign(-0.0) = +1 and a
+ *   NaN latent packs as +1.
+ *
+ * Packed sign format.  A packed row of K signs is ceil(K/32) (or ld_words >=
+ * that) little-endian uint32 words; bit (e % 32) of word (e / 32) is 1 exactly
+ * when element e is negative (sign -1).  Bits past K are written as 0 by
+ * lb_pack_signs and ignored by every forward.  V_b is stored packed along the
+ * input dimension (Vp_b[r][ld_v], ld_v >= ceil(in/32)) and U_b packed along the
+ * latent dimension (Up_b[out][ld_u], ld_u >= ceil(r/32)).
+ *
+ * Conventions for every entry point.
+ *   - The caller owns all memory.  Device pointers are CUDA device (or managed)
+ *     addresses on the current device; host pointers are ordinary host memory.
+ *     No forward call allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are stream-ordered and asynchronous unless stated otherwise.
+ *   - Argument errors are reported synchronously by the return value, before
+ *     anything is launched.  Launch failures return LB_ERR_CUDA.  Faults that
+ *     happen later on the device surface at the caller's next synchronisation.
+ *   - Matrices are row-major.  x is M x in, y is M x out.
+ *   - The library keeps no state between calls and is thread-safe.
+ */
+#ifndef LB_H
+#define LB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LB_OK = 0,
+    LB_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad enum      */
+    LB_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned                */
+    LB_ERR_UNSUPPORTED = 3,   /* valid but not supported (e.g. no sm_100 device) */
+    LB_ERR_CUDA = 4,          /* a CUDA runtime call failed                      */
+    LB_ERR_TIMEOUT = 5,       /* a device-side wait gave up (see lb_stack_status)*/
+    LB_ERR_WORKSPACE = 6      /* workspace missing or smaller than required      */
+} lb_status;
+
+typedef enum { LB_F16 = 0, LB_BF16 = 1, LB_F32 = 2 } lb_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *lb_status_string(lb_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int lb_version(void);
+
+/*
+ * lb_pack_signs — binarise an fp32 latent factor into packed sign words.
+ * Defines the "signs only at inference" step (item 1 of "How it works").
+ *
+ *   latent   : device, rows x cols fp32, row stride ld elements (ld >= cols)
+ *   axis = 1 : every row is packed along its columns
+ *              -> packed[rows][ld_words], ld_words >= ceil(cols/32)   (U: out x r)
+ *   axis = 0 : every column is packed along the rows
+ *              -> packed[cols][ld_words], ld_words >= ceil(rows/32)   (V: in x r)
+ *   packed   : device, written in full (padding bits and padding words are 0)
+ *   bit = 1 exactly when the latent element is < 0.0f (so -0.0 and NaN give 0).
+ * Errors: LB_ERR_INVALID_ARG for null pointers, rows/cols <= 0, ld < cols,
+ * ld_words too small or axis not in {0, 1}; LB_ERR_ALIGNMENT if latent or
+ * packed is not 4-byte aligned.
+ */
+lb_status lb_pack_signs(const float *latent, int64_t rows, int64_t cols, int64_t ld,
+                        int axis, uint32_t *packed, int64_t ld_words, void *stream);
+
+/* One branch of a factorised layer (all device pointers). */
+typedef struct {
+    const uint32_t *Vp;   /* [r][ld_v] signs of V_b packed along in          */
+    const uint32_t *Up;   /* [out][ld_u] signs of U_b packed along r         */
+    const uint16_t *h;    /* [out] FP16 row scale (IEEE binary16 bits)       */
+    const uint16_t *g;    /* [in]  FP16 column scale                         */
+    const uint16_t *l;    /* [r]   FP16 latent scale                         */
+} lb_branch;
+
+/*
+ * lb_linear_forward — y = the layer applied to the M rows of x (formula above).
+ *
+ *   x         : device, M x in, dtype x_dtype (LB_F16, LB_BF16 or LB_F32)
+ *   br        : host array of n_branches (1 or 2) lb_branch; every branch shares
+ *               in, out, r, ld_v = ceil(in/32) and ld_u = ceil(r/32)
+ *   y         : device, M x out fp32, overwritten
+ *   workspace : device scratch of at least lb_linear_workspace_size(...) bytes,
+ *               16-byte aligned; contents need not be initialised and are
+ *               clobbered.  Concurrent calls need distinct workspaces.
+ * Small M runs the lookup-table decode kernels; large M runs the tcgen05
+ * tensor-core kernels.  Both accumulate in fp32.
+ * Errors: LB_ERR_INVALID_ARG (null pointer, M/in/out/r <= 0, n_branches not 1
+ * or 2, bad dtype), LB_ERR_ALIGNMENT (x, y, workspace or a packed pointer not
+ * 16-byte aligned), LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED (no sm_100 device),
+ * LB_ERR_CUDA.
+ */
+lb_status lb_linear_forward(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
+                            int64_t out, int64_t r, const lb_branch *br, int n_branches,
+                            float *y, void *workspace, size_t ws_bytes, void *stream);
+
+size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
+                                int n_branches);
+
+/* Which kernels lb_linear_forward uses for M rows: 0 = decode, 1 = tensor core. */
+int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r);
+
+/*
+ * Decoder stacks.  A stack runs, for one token (batch 1), the linears of
+ * n_layers Llama-2-shaped decoder layers and the glue between them:
+ *
+ *   a = rmsnorm(h) (weightless, eps 1e-5); q,k,v = L_q(a), L_k(a), L_v(a);
+ *   attn = v broadcast over the query heads of its key/value group (attention
+ *   over one position); h += L_o(attn); a = rmsnorm(h);
+ *   h += L_down(silu(L_gate(a)) * L_up(a)).
+ *
+ * With LB_STACK_MLP_ONLY each layer is y = L_down(silu(L_gate(x)) * L_up(x))
+ * (no attention, norm or residual; n_layers must be 1).
+ * Activations between linears are fp32; the input is bf16 and the output fp32.
+ * The pages describe the layer only: this glue is the plainest decoder around it.
+ */
+enum { LB_Q = 0, LB_K = 1, LB_V = 2, LB_O = 3, LB_GATE = 4, LB_UP = 5, LB_DOWN = 6,
+       LB_N_PROJ = 7 };
+enum { LB_STACK_MLP_ONLY = 1 };
+
+typedef struct {
+    int n_layers, hidden, inter, n_heads, n_kv_heads, head_dim, n_branches, flags;
+    const lb_branch *lin;   /* host array [n_layers][LB_N_PROJ][n_branches]       */
+    const int64_t *ranks;   /* host array [n_layers][LB_N_PROJ] latent rank r     */
+} lb_stack_desc;
+
+/* Bytes of device workspace a stack needs (header, accumulators, plan). */
+size_t lb_stack_workspace_size(const lb_stack_desc *d);
+
+/*
+ * lb_stack_prepare — validate the descriptor and write the stack's execution
+ * plan into `workspace` (device, 256-byte aligned, >= lb_stack_workspace_size).
+ * Synchronous: returns after the plan is on the device.  The plan stays valid
+ * while the weights stay where they are; pass the same descriptor and
+ * workspace to every lb_stack_forward of that stack.
+ * Errors: LB_ERR_INVALID_ARG (null pointer, non-positive or inconsistent
+ * sizes: n_heads*head_dim must equal hidden, n_heads a multiple of n_kv_heads,
+ * every rank > 0, MLP_ONLY with n_layers != 1), LB_ERR_ALIGNMENT,
+ * LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED, LB_ERR_CUDA.
+ */
+lb_status lb_stack_prepare(const lb_stack_desc *d, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/*
+ * lb_stack_forward — one token through a prepared stack.
+ *   x : device bf16 [hidden];  y : device fp32 [hidden], overwritten.
+ * One memset and one cooperative persistent kernel on `stream`.  Grid-wide
+ * waits inside the kernel are bounded; if one gives up the kernel returns
+ * early and lb_workspace_status reports LB_ERR_TIMEOUT.
+ */
+lb_status lb_stack_forward(const lb_stack_desc *d, void *workspace, size_t ws_bytes,
+                           const void *x, float *y, void *stream);
+
+/*
+ * lb_stack_forward_host — the same through host buffers: copies x (host bf16)
+ * to the device, runs the stack, copies y (host fp32) back and synchronises
+ * `stream`.  The device-side x and y live in the workspace.  Pinned host
+ * memory gives asynchronous copies; pageable memory also works.
+ */
+lb_status lb_stack_forward_host(const lb_stack_desc *d, void *workspace, size_t ws_bytes,
+                                const void *x_host, float *y_host, void *stream);
+
+/* Synchronises `stream`, then reports whether the last stack or linear call
+ * that used `workspace` finished its device-side waits: LB_OK or LB_ERR_TIMEOUT. */
+lb_status lb_workspace_status(const void *workspace, void *stream);
+
+/* Device fp32 output of linear `proj` (LB_Q ... LB_DOWN) of layer `layer` from
+ * the last lb_stack_forward on this workspace (read it after the stream is
+ * synchronised), or NULL for LB_O and LB_DOWN (those add straight into the
+ * residual stream) and for bad arguments.  Lets callers check the q and k
+ * projections, which feed nothing else in the stack. */
+const float *lb_stack_output(const lb_stack_desc *d, const void *workspace, int layer,
+                             int proj);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LB_H */

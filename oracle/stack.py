@@ -49,7 +49,8 @@ def rmsnorm(v: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
 
 
 def silu(v: np.ndarray) -> np.ndarray:
-    return v / (1.0 + np.exp(-v))
+    with np.errstate(over="ignore"):     # exp(-v) -> inf for very negative v gives -0.0
+        return v / (1.0 + np.exp(-v))
 
 
 def gqa_broadcast(v: np.ndarray, n_heads: int, n_kv_heads: int, head_dim: int) -> np.ndarray:

@@ -1,0 +1,87 @@
+"""lb_linear_forward against the oracle (GPU).
+
+Bar: max|y - y_ref| <= 2e-3 * max|y_ref| per output tensor (fp32 outputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import binary_rank_linear_lb_b200 as lb
+from binary_rank_linear_lb_b200 import synth
+from binary_rank_linear_lb_b200.configs import SINGLE, rank_for
+from binary_rank_linear_lb_b200.model import build_linear
+
+from helpers import assert_close, oracle_linear, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(in_f, out_f, r, M, dtype, nb=2, base=0, rows=None):
+    brs = build_linear(in_f, out_f, r, base=base, n_branches=nb)
+    x = synth.activation((M, in_f), synth.tensor_seed(base, 0, 0, 0, synth.KIND_X), dtype, "cuda")
+    y = lb.linear_forward(x, brs, in_f, out_f, r)
+    torch.cuda.synchronize()
+    ob = oracle_linear(in_f, out_f, r, base, 0, 0, nb)
+    y_ref = oracle.forward(to_f64(x), ob, in_f, out_f, r, rows=rows)
+    got = y.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got = got[:, rows]
+    return got, y_ref
+
+
+def test_single_linear_config():
+    """in 512, out 256, r 32, two branches, M = 1, fp16 x."""
+    got, ref = run_case(SINGLE["in_f"], SINGLE["out_f"], SINGLE["r"], 1, torch.float16)
+    assert_close(got, ref, what="single")
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (32, 32, 32), (100, 33, 7), (1000, 300, 70),
+                                   (1024, 1024, 1024), (1100, 2100, 1088), (300, 5000, 2100)])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+def test_ragged_shapes(shape, dtype):
+    got, ref = run_case(*shape, M=1, dtype=dtype)
+    assert_close(got, ref, what=str(shape))
+
+
+@pytest.mark.parametrize("M", [2, 3, 8, 11])
+def test_small_batches(M):
+    got, ref = run_case(777, 513, 96, M, torch.bfloat16)
+    for m in range(M):
+        assert_close(got[m], ref[m], what=f"row {m}")
+
+
+def test_one_branch():
+    got, ref = run_case(640, 320, 64, 1, torch.bfloat16, nb=1)
+    assert_close(got, ref, what="one branch")
+
+
+@pytest.mark.parametrize("bpw", [1.0, 0.55, 0.3, 0.1])
+@pytest.mark.parametrize("shape", [(4096, 11008), (11008, 4096)])
+def test_7b_mlp_shapes(shape, bpw):
+    r = rank_for(bpw, *shape)
+    got, ref = run_case(shape[0], shape[1], r, 1, torch.bfloat16, base=1)
+    assert_close(got, ref, what=f"{shape} @ {bpw}")
+
+
+@pytest.mark.parametrize("shape", [(8192, 28672, 3136), (28672, 8192, 3136), (8192, 1024, 448)])
+def test_70b_shapes_sampled_rows(shape):
+    """Full-size 70B linears; the oracle evaluates 96 sampled output rows."""
+    rng = np.random.default_rng(shape[1])
+    rows = np.sort(rng.choice(shape[1], size=96, replace=False)).tolist()
+    rows[-1] = shape[1] - 1
+    got, ref = run_case(*shape, M=1, dtype=torch.bfloat16, base=2, rows=rows)
+    # the tolerance is relative to max|y_ref| over the sampled rows
+    assert_close(got, ref, what=f"70B {shape}")
+
+
+def test_workspace_reports_ok_and_repeat_calls_agree():
+    in_f, out_f, r = 2048, 1536, 256
+    brs = build_linear(in_f, out_f, r)
+    x = synth.activation((1, in_f), 7, torch.bfloat16, "cuda")
+    ws = torch.empty(lb.linear_workspace_size(1, in_f, out_f, r, 2), dtype=torch.uint8,
+                     device="cuda")
+    y1 = lb.linear_forward(x, brs, in_f, out_f, r, workspace=ws).clone()
+    y2 = lb.linear_forward(x, brs, in_f, out_f, r, workspace=ws)
+    assert lb.workspace_status(ws) == lb.LB_OK
+    torch.testing.assert_close(y1, y2, rtol=1e-5, atol=1e-4 * y1.abs().max().item())

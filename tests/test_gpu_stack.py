@@ -1,0 +1,102 @@
+"""lb_stack_forward (decoder stacks and the 7B MLP block) against the oracle (GPU).
+
+The oracle runs the whole stack itself from the same seeded inputs; no GPU
+intermediate ever enters it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import stack as ostack
+import binary_rank_linear_lb_b200 as lb
+from binary_rank_linear_lb_b200 import synth
+from binary_rank_linear_lb_b200.configs import LLAMA2_13B, LLAMA2_7B, LLAMA2_70B, Model
+from binary_rank_linear_lb_b200.model import build_mlp_block, build_stack
+
+from helpers import assert_close, oracle_linear, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_layers(model: Model, ranks, n_layers, base):
+    layers = []
+    for li in range(n_layers):
+        L = {}
+        for p, name in enumerate(ostack_names()):
+            i, o = model.shapes()[p]
+            L[name] = ostack.Linear(oracle_linear(i, o, ranks[p], base, li, p), i, o, ranks[p])
+        layers.append(L)
+    return layers
+
+
+def ostack_names():
+    return ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def run_stack(model, bpw, n_layers, base, ranks=None):
+    rk = ranks or model.ranks(bpw)
+    st = build_stack(model, bpw, base=base, n_layers=n_layers, ranks=rk)
+    x = synth.activation(model.hidden, synth.tensor_seed(base, 0, 0, 0, synth.KIND_X),
+                         torch.bfloat16, "cuda")
+    y = st.forward(x)
+    torch.cuda.synchronize()
+    assert st.status() == lb.LB_OK
+    layers = oracle_layers(model, rk, n_layers, base)
+    h_ref, outs = ostack.decoder_stack(to_f64(x), layers, model.n_heads, model.n_kv_heads,
+                                       model.head_dim, keep=True)
+    return st, x, y, h_ref, outs
+
+
+SMALL = Model("small", hidden=256, inter=512, n_layers=3, n_heads=4, n_kv_heads=2, head_dim=64)
+
+
+def test_small_decoder_stack_and_intermediates():
+    st, x, y, h_ref, outs = run_stack(SMALL, 1.0, 3, base=3, ranks=[64, 32, 32, 64, 96, 96, 96])
+    assert_close(y.cpu().numpy(), h_ref, what="small stack")
+    for li in range(3):
+        for p, name in ((0, "q"), (1, "k"), (2, "v"), (4, "gate"), (5, "up")):
+            got = st.output(li, p).cpu().numpy()
+            assert_close(got, outs[li][name], what=f"layer {li} {name}")
+
+
+def test_forward_host_matches_device():
+    st = build_stack(SMALL, 1.0, base=4, n_layers=2, ranks=[64, 32, 32, 64, 96, 96, 96])
+    x = synth.activation(SMALL.hidden, 11, torch.bfloat16, "cuda")
+    y = st.forward(x).cpu()
+    xh = x.cpu().pin_memory()
+    yh = torch.empty(SMALL.hidden, dtype=torch.float32).pin_memory()
+    st.forward_host(xh, yh)
+    torch.testing.assert_close(yh, y, rtol=1e-4, atol=1e-4 * y.abs().max().item())
+
+
+@pytest.mark.parametrize("bpw", [0.55, 0.1])
+def test_13b_stack_two_layers_full_width(bpw):
+    _, _, y, h_ref, _ = run_stack(LLAMA2_13B, bpw, 2, base=5)
+    assert_close(y.cpu().numpy(), h_ref, what=f"13B x2 @ {bpw}")
+
+
+@pytest.mark.slow
+def test_13b_stack_full_depth_0p1():
+    _, _, y, h_ref, _ = run_stack(LLAMA2_13B, 0.1, LLAMA2_13B.n_layers, base=6)
+    assert_close(y.cpu().numpy(), h_ref, what="13B x40 @ 0.1")
+
+
+@pytest.mark.slow
+def test_70b_stack_two_layers_full_width():
+    _, _, y, h_ref, _ = run_stack(LLAMA2_70B, 0.55, 2, base=7)
+    assert_close(y.cpu().numpy(), h_ref, what="70B x2 @ 0.55")
+
+
+@pytest.mark.parametrize("bpw", [1.0, 0.55, 0.3, 0.1])
+def test_7b_mlp_block(bpw):
+    base = 8
+    st = build_mlp_block(LLAMA2_7B, bpw, base=base)
+    x = synth.activation(LLAMA2_7B.hidden, 13, torch.bfloat16, "cuda")
+    y = st.forward(x)
+    torch.cuda.synchronize()
+    rk = LLAMA2_7B.ranks(bpw)
+    mk = lambda p: ostack.Linear(oracle_linear(*LLAMA2_7B.shapes()[p], rk[p], base, 0, p),
+                                 *LLAMA2_7B.shapes()[p], rk[p])
+    ref = ostack.mlp_block(to_f64(x), mk(4), mk(5), mk(6))
+    assert_close(y.cpu().numpy(), ref, what=f"7B MLP @ {bpw}")
