@@ -53,7 +53,8 @@ class lb_stack_desc(ctypes.Structure):
 EXPORTS = ("lb_status_string", "lb_version", "lb_pack_signs", "lb_linear_forward",
            "lb_linear_workspace_size", "lb_linear_path", "lb_stack_workspace_size",
            "lb_stack_prepare", "lb_stack_forward", "lb_stack_forward_host",
-           "lb_workspace_status", "lb_stack_output")
+           "lb_workspace_status", "lb_stack_output", "lb_linear_forward_noalloc",
+           "lb_noalloc_scratch_bytes")
 
 _lib = None
 
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.lb_workspace_status.restype = st
         L.lb_stack_output.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int]
         L.lb_stack_output.restype = vp
+        L.lb_linear_forward_noalloc.argtypes = [vp, st, i64, i64, i64, i64, vp, ctypes.c_int, vp,
+                                                vp]
+        L.lb_linear_forward_noalloc.restype = st
+        L.lb_noalloc_scratch_bytes.restype = sz
         _lib = L
     return _lib
 
@@ -178,6 +183,24 @@ def linear_forward(x: torch.Tensor, branches: Sequence[Branch], in_f: int, out_f
     _check(lib().lb_linear_forward(_ptr(x2), dt, M, in_f, out_f, r, ctypes.addressof(arr), nb,
                                    _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
            "lb_linear_forward")
+    return y
+
+
+def linear_forward_noalloc(x: torch.Tensor, branches: Sequence[Branch], in_f: int, out_f: int,
+                           r: int, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """lb_linear_forward_noalloc: like linear_forward, with the library's own fixed scratch.
+
+    For callers that cannot allocate device memory; `y` (M x out, fp32) must be given.
+    """
+    x2 = x if x.dim() == 2 else x.reshape(1, -1)
+    nb = len(branches)
+    arr = (lb_branch * nb)(*[b.c_struct() for b in branches])
+    dt = _DTYPES.get(x2.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported x dtype {x2.dtype}")
+    _check(lib().lb_linear_forward_noalloc(_ptr(x2), dt, x2.shape[0], in_f, out_f, r,
+                                           ctypes.addressof(arr), nb, _ptr(y), _stream(stream)),
+           "lb_linear_forward_noalloc")
     return y
 
 

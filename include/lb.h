@@ -114,6 +114,32 @@ lb_status lb_linear_forward(const void *x, lb_dtype x_dtype, int64_t M, int64_t 
 size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
                                 int n_branches);
 
+/*
+ * lb_linear_forward_noalloc — lb_linear_forward for callers that cannot
+ * allocate device memory (code running under another framework's allocator,
+ * plugins in a process whose device pool is already taken, real-time paths
+ * where an allocation may block or fail).  The pages have no counterpart to
+ * this entry point; it only moves the scratch.
+ *
+ * Same arguments and results as lb_linear_forward, without `workspace`: the
+ * scratch lives in a fixed __device__ array of lb_noalloc_scratch_bytes()
+ * bytes (256 KiB) inside liblb.so, which every GPU that loads the library holds
+ * until the process exits.  Calls whose lb_linear_workspace_size(M, in, out, r,
+ * n_branches) exceeds it return LB_ERR_WORKSPACE (with two branches: r up to 32736 for
+ * M = 1, up to 4092 for M >= 8).  The first call on a device looks up the
+ * array's device address; make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents; each call
+ * clears what must start at zero, and calls that overlap on the GPU (streams
+ * not ordered with each other) race on it.  It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ */
+lb_status lb_linear_forward_noalloc(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
+                                    int64_t out, int64_t r, const lb_branch *br,
+                                    int n_branches, float *y, void *stream);
+
+/* Size in bytes of the fixed scratch array used by lb_linear_forward_noalloc. */
+size_t lb_noalloc_scratch_bytes(void);
+
 /* Which kernels lb_linear_forward uses for M rows: 0 = decode, 1 = tensor core. */
 int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r);
 
