@@ -21,7 +21,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -39,16 +38,25 @@ WORKLOADS = {
     "mlp7b-0.55": ("llama2-7b", 0.55, "mlp"),
     "mlp7b-0.3": ("llama2-7b", 0.3, "mlp"),
     "mlp7b-0.1": ("llama2-7b", 0.1, "mlp"),
+    # single linears through lb_linear_forward: (in, out), bits/weight, M rows of x
+    "prefill-gate7b-1.0-M4096": ((4096, 11008), 1.0, "linear", 4096),
+    "prefill-gate7b-0.1-M4096": ((4096, 11008), 0.1, "linear", 4096),
+    "prefill-gate7b-1.0-M512": ((4096, 11008), 1.0, "linear", 512),
+    "decode-gate70b-1.0-M1": ((8192, 28672), 1.0, "linear", 1),
 }
 METRIC = "batch-1 layer-stack tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 
 
-def describe(name: str) -> str:
-    model, bpw, kind = WORKLOADS[name]
+def describe(name: str, n_layers: int = 0) -> str:
+    model, bpw, kind = WORKLOADS[name][:3]
+    if kind == "linear":
+        (i, o), M = model, WORKLOADS[name][3]
+        return f"one factorised linear {i}->{o}, {bpw} bits/weight, 2 branches, M={M} rows of x"
     if kind == "mlp":
         return f"{model} MLP block (gate, up 4096->11008, down 11008->4096), {bpw} bits/weight, batch 1"
-    return f"{model} decoder linear stack, all layers, {bpw} bits/weight, 2 branches, batch 1"
+    layers = f"{n_layers} layers" if n_layers else "all layers"
+    return f"{model} decoder linear stack, {layers}, {bpw} bits/weight, 2 branches, batch 1"
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -81,85 +89,134 @@ def barrier(world: int, device=None):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons through NVML while the timed loop runs."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
-        self.proc = None
-        self.lines = []
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.index = device_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _handle(self, nv):
+        import torch
+        props = torch.cuda.get_device_properties(self.index)
+        uuid = str(getattr(props, "uuid", ""))
+        for cand in (uuid, "GPU-" + uuid):
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(cand)
+            except Exception:
+                pass
+        bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                    props.pci_device_id)
+        return nv.nvmlDeviceGetHandleByPciBusId(bus)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, rs))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.thread.join(timeout=5)
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
 
 
 # ---------------------------------------------------------------- workloads
-def build_workload(name: str, device, seed: int):
-    from binary_rank_linear_lb_b200.configs import MODELS, linear_bytes
+class LinearStep:
+    """One lb_linear_forward call on M rows, shaped like a stack for the timing loop."""
+
+    def __init__(self, in_f, out_f, r, M, device, seed):
+        import torch
+        import binary_rank_linear_lb_b200 as lb
+        from binary_rank_linear_lb_b200 import synth
+        from binary_rank_linear_lb_b200.model import build_linear
+        self.lb, self.in_f, self.out_f, self.r, self.M = lb, in_f, out_f, r, M
+        self.brs = build_linear(in_f, out_f, r, base=seed, device=device, signs="bits")
+        self.x = synth.activation((M, in_f), seed + 1, torch.bfloat16, device)
+        self.y = torch.empty((M, out_f), dtype=torch.float32, device=device)
+        self.ws = torch.empty(lb.linear_workspace_size(M, in_f, out_f, r, 2), dtype=torch.uint8,
+                              device=device)
+        self.hidden = in_f
+
+    def forward(self, x=None, y=None):
+        return self.lb.linear_forward(self.x, self.brs, self.in_f, self.out_f, self.r, y=self.y,
+                                      workspace=self.ws)
+
+    def forward_host(self, xh, yh):
+        import torch
+        self.x.copy_(xh.view(self.M, self.in_f), non_blocking=True)
+        self.forward()
+        yh.view(self.M, self.out_f).copy_(self.y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    def status(self):
+        return self.lb.workspace_status(self.ws)
+
+
+def build_workload(name: str, device, seed: int, n_layers: int = 0):
+    from binary_rank_linear_lb_b200.configs import MODELS, linear_bytes, linear_flops, rank_for
     from binary_rank_linear_lb_b200.model import build_mlp_block, build_stack
-    model_name, bpw, kind = WORKLOADS[name]
+    model_name, bpw, kind = WORKLOADS[name][:3]
+    if kind == "linear":
+        (i, o), M = model_name, WORKLOADS[name][3]
+        r = rank_for(bpw, i, o)
+        st = LinearStep(i, o, r, M, device, seed)
+        nbytes = linear_bytes(i, o, r) + M * i * 2 + M * o * 4
+        st.flops = linear_flops(M, i, o, r)
+        return st, st, bpw, kind, nbytes
     model = MODELS[model_name]
     if kind == "mlp":
         st = build_mlp_block(model, bpw, base=seed, device=device, signs="bits")
         nbytes = sum(linear_bytes(*model.shapes()[p], model.ranks(bpw)[p]) for p in (4, 5, 6))
     else:
-        st = build_stack(model, bpw, base=seed, device=device, signs="bits")
-        nbytes = model.bytes_per_token(bpw)
+        nl = n_layers or model.n_layers
+        st = build_stack(model, bpw, base=seed, n_layers=nl, device=device, signs="bits")
+        nbytes = model.bytes_per_token(bpw, nl)
     return st, model, bpw, kind, nbytes
 
 
 def peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s, source) from the measured peaks file."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         d = json.load(open(path))
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except (OSError, KeyError, ValueError):
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0, "fallback"
 
 
 def cpu_oracle_rate(name: str, budget_s: float = 12.0):
@@ -168,10 +225,30 @@ def cpu_oracle_rate(name: str, budget_s: float = 12.0):
     import oracle
     from oracle import stack as ostack
     from binary_rank_linear_lb_b200.configs import MODELS
-    model_name, bpw, kind = WORKLOADS[name]
+    model_name, bpw, kind = WORKLOADS[name][:3]
+    rng = np.random.default_rng(0)
+    if kind == "linear":
+        from binary_rank_linear_lb_b200.configs import rank_for
+        (i, o), M = model_name, WORKLOADS[name][3]
+        r = rank_for(bpw, i, o)
+        brs = []
+        for _ in range(2):
+            Vp = rng.integers(0, 2 ** 32, size=(r, (i + 31) // 32), dtype=np.uint64).astype(np.uint32)
+            Up = rng.integers(0, 2 ** 32, size=(o, (r + 31) // 32), dtype=np.uint64).astype(np.uint32)
+            sc = lambda n: np.abs(1 + 0.1 * rng.standard_normal(n))
+            brs.append(oracle.Branch(Vp, Up, sc(o), sc(i), sc(r)))
+        xs = rng.standard_normal((1, i))
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < 1000:
+            oracle.forward(xs, brs, i, o, r)
+            reps += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = (time.perf_counter() - t0) / reps
+        return 1.0 / dt, oracle.threads(), f"{reps} rows of x through the full layer (rows/s)"
     model = MODELS[model_name]
     rk = model.ranks(bpw)
-    rng = np.random.default_rng(0)
 
     def lin(p):
         i, o = model.shapes()[p]
@@ -210,6 +287,80 @@ def cpu_oracle_rate(name: str, budget_s: float = 12.0):
         f"{layers_done} of {model.n_layers} decoder layers of one token, time scaled to all layers")
 
 
+# ---------------------------------------------------------------- sweeps
+def _time_events(fn, iters, flush=None):
+    """Median device time (ms) of fn() over iters runs, L2 flushed before each."""
+    import torch
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def sweep_prefill(device, flush, tflops_peak):
+    """The 7B gate projection (4096 -> 11008) over the token batch M, both paths."""
+    import torch
+    import binary_rank_linear_lb_b200 as lb
+    from binary_rank_linear_lb_b200 import synth
+    from binary_rank_linear_lb_b200.configs import linear_bytes, linear_flops, rank_for
+    from binary_rank_linear_lb_b200.model import build_linear
+    in_f, out_f = 4096, 11008
+    out = []
+    for bpw in (1.0, 0.1):
+        r = rank_for(bpw, in_f, out_f)
+        brs = build_linear(in_f, out_f, r, base=77, device=device, signs="bits")
+        for M in (1, 8, 64, 512, 4096):
+            x = synth.activation((M, in_f), 5, torch.bfloat16, device)
+            y = torch.empty((M, out_f), dtype=torch.float32, device=device)
+            ws = torch.empty(lb.linear_workspace_size(M, in_f, out_f, r, 2), dtype=torch.uint8,
+                             device=device)
+            fn = lambda: lb.linear_forward(x, brs, in_f, out_f, r, y=y, workspace=ws)
+            for _ in range(3):
+                fn()
+            ms = _time_events(fn, 10, flush)
+            fl = linear_flops(M, in_f, out_f, r)
+            by = linear_bytes(in_f, out_f, r) + M * in_f * 2 + M * out_f * 4
+            out.append({"bits_per_weight": bpw, "r": r, "M": M,
+                        "path": "tcgen05" if lb.linear_path(M, in_f, out_f, r) else "lut-decode",
+                        "ms": ms, "tflops": fl / ms / 1e9, "gbs": by / ms / 1e6,
+                        "tensor_frac_fp16": fl / ms / 1e9 / tflops_peak,
+                        "tensor_frac_fp8": fl / ms / 1e9 / (2 * tflops_peak)})
+            del x, y, ws
+    return out
+
+
+def sweep_stacks(device, skip: str, hbm_peak):
+    """tokens/s of the other stack workloads (fewer steps; same timing rules)."""
+    import torch
+    from binary_rank_linear_lb_b200 import synth
+    out = {}
+    for name in ("stack70b-1.0", "stack70b-0.55", "stack13b-0.55", "stack13b-0.1", "mlp7b-1.0",
+                 "mlp7b-0.55", "mlp7b-0.3", "mlp7b-0.1"):
+        if name == skip:
+            continue
+        st, model, bpw, kind, nbytes = build_workload(name, device, 99)
+        x = synth.activation(model.hidden, 3, torch.bfloat16, device)
+        y = torch.empty(model.hidden, dtype=torch.float32, device=device)
+        flush = None
+        if nbytes < 2 * L2_BYTES:
+            flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+        for _ in range(3):
+            st.forward(x, y)
+        ms = _time_events(lambda: st.forward(x, y), 10, flush)
+        out[name] = {"tokens_per_s": 1e3 / ms, "ms_per_token": ms, "bytes_per_token": nbytes,
+                     "gbs": nbytes / ms / 1e6, "hbm_frac": nbytes / ms / 1e6 / hbm_peak}
+        del st, flush
+        torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -219,7 +370,11 @@ def main():
     ap.add_argument("--workload", default="stack70b-1.0", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="decoder layers (default: all); fewer only for profiling captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the extra sweeps (prefill M sweep, other stacks) on rank 0")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.warmup < 3:
@@ -255,9 +410,14 @@ def main():
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
 
-    st, model, bpw, kind, nbytes = build_workload(args.workload, device, args.seed + rank)
-    x = synth.activation(model.hidden, 1234 + rank, torch.bfloat16, device)
-    y = torch.empty(model.hidden, dtype=torch.float32, device=device)
+    st, model, bpw, kind, nbytes = build_workload(args.workload, device, args.seed + rank,
+                                                  args.layers)
+    if kind == "linear":
+        x, y, tokens = st.x, st.y, st.M
+    else:
+        x = synth.activation(model.hidden, 1234 + rank, torch.bfloat16, device)
+        y = torch.empty(model.hidden, dtype=torch.float32, device=device)
+        tokens = 1
     stream = torch.cuda.current_stream(device)
     flush = None
     if nbytes < 2 * L2_BYTES:
@@ -269,13 +429,11 @@ def main():
     if st.status() != lb.LB_OK:
         raise RuntimeError("device-side wait timed out during warm-up")
 
-    uuid = str(torch.cuda.get_device_properties(device).uuid)
-    gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world, device)
     torch.cuda.synchronize(device)
-    with ClockSampler(gpu_id) as clocks:
+    with ClockSampler(device.index) as clocks:
         t_wall = time.perf_counter()
         for i in range(args.steps):
             if flush is not None:
@@ -291,11 +449,11 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
     total_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = total_ms / args.steps
-    value = world * args.steps / (total_ms / 1e3)
+    value = world * args.steps * tokens / (total_ms / 1e3)
 
     # End to end through the public host-buffer entry point (copies inside the timing).
     xh = x.cpu().pin_memory()
-    yh = torch.empty(model.hidden, dtype=torch.float32).pin_memory()
+    yh = torch.empty(tuple(y.shape), dtype=torch.float32).pin_memory()
     for _ in range(3):
         st.forward_host(xh, yh)
     barrier(world, device)
@@ -304,25 +462,38 @@ def main():
     for i in range(e2e_steps):
         st.forward_host(xh, yh)
     e2e_s = max_over_ranks(time.perf_counter() - t0, world, device)
-    e2e_value = world * e2e_steps / e2e_s
+    e2e_value = world * e2e_steps * tokens / e2e_s
 
-    hbm_peak, peak_kind = peaks()
+    hbm_peak, tflops_peak, peak_kind = peaks()
     achieved = nbytes / (ms_per_step / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_kind,
+            "kernel": "stack_program_kernel"}
+    launches = args.steps
+    if kind == "linear":
+        if lb.linear_path(st.M, st.in_f, st.out_f, st.r):
+            tf = st.flops / (ms_per_step / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": tf, "peak": tflops_peak, "unit": "TFLOP/s",
+                    "frac": tf / tflops_peak, "traffic": None,
+                    "peak_source": peak_kind + " (bf16 dense; fp16 runs at the same rate)",
+                    "kernel": "prefill_gemm_kernel", "fp8_frac": tf / (2 * tflops_peak)}
+            launches = 4 * args.steps
+        else:
+            roof["kernel"] = "linear_program_kernel"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": describe(args.workload), "bits_per_weight": bpw,
+        "config": {"workload": describe(args.workload, args.layers), "bits_per_weight": bpw,
                    "bytes_per_token": nbytes, "parallelism": f"replicas{world}",
                    "l2": "flushed between steps" if flush is not None
                    else "working set larger than L2", "signs": "uniform random bits"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
-                     "peak_source": peak_kind, "kernel": "stack_program_kernel"},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 2 * model.hidden,
-                "d2h_bytes_per_step": 4 * model.hidden},
-        "gpu_launches": args.steps,
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                "d2h_bytes_per_step": yh.numel() * yh.element_size()},
+        "gpu_launches": launches,
         "clocks": clocks.summary(),
         "wall_s": t_wall,
     }
@@ -330,6 +501,16 @@ def main():
         rate, cores, sample = cpu_oracle_rate(args.workload)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}
+    if rank == 0 and world == 1 and not args.no_sweep:
+        del st
+        torch.cuda.empty_cache()
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+        line["sweeps"] = {
+            "prefill_gate7b": sweep_prefill(device, flush, tflops_peak),
+            "stacks": sweep_stacks(device, args.workload, hbm_peak),
+            "peaks": {"hbm_gbs": hbm_peak, "fp16_tflops": tflops_peak,
+                      "fp8_tflops_nominal_ratio": 2 * tflops_peak, "source": peak_kind},
+        }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

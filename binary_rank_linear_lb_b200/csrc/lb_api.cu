@@ -32,6 +32,7 @@ void init_device(int d) {
     g_sm_count[d] = prop.multiProcessorCount;
     g_cc_major[d] = prop.major;
     g_cfg_err[d] = prop.major == 10 ? decode_configure() : cudaErrorInvalidDeviceFunction;
+    if (g_cfg_err[d] == cudaSuccess) g_cfg_err[d] = prefill_configure();
 }
 
 // Returns LB_OK when the current device is an sm_100 part and the kernels are configured.
@@ -81,14 +82,20 @@ bool branch_aligned(const lb_branch& b) {
 }
 
 // ------------------------------------------------------------ stack layout
+// Accumulators are laid out phase by phase: region p holds everything phase p
+// accumulates into (t of its first contractions, outputs of its second
+// contractions, the RMSNorm sum of squares).  The kernel zeroes region p+1
+// during phase p and region 0 during the last phase, so a call leaves the
+// workspace ready for the next one; lb_stack_prepare zeroes it once.
 struct StackLayout {
-    size_t sumsq;                 // [n_layers][2] floats
-    size_t t;                     // first t accumulator
-    std::vector<size_t> t_off;    // [layer][proj][branch]
-    std::vector<size_t> o_off;    // [layer][proj] output accumulators (q,k,v,gate,up), else 0
-    size_t acc_end;               // end of the region zeroed per call
-    size_t x_dev, y_dev;          // staging for lb_stack_forward_host
-    size_t phases, jobs;          // plan
+    std::vector<size_t> sumsq_off;   // [layer][2] (attention norm, MLP norm)
+    std::vector<size_t> t_off;       // [layer][proj][branch]
+    std::vector<size_t> o_off;       // [layer][proj] outputs of q,k,v,gate,up (else 0)
+    std::vector<size_t> region_off;  // [phase] first byte of the phase's region
+    std::vector<size_t> region_len;  // [phase] bytes (0: nothing, or y for MLP-only)
+    size_t acc_end;                  // end of the accumulator area
+    size_t x_dev, y_dev;             // staging for lb_stack_forward_host
+    size_t phases, jobs;             // plan
     int n_phases, n_jobs;
     size_t total;
 };
@@ -96,6 +103,7 @@ struct StackLayout {
 bool stack_desc_ok(const lb_stack_desc* d) {
     if (!d || !d->lin || !d->ranks) return false;
     if (d->n_layers <= 0 || d->hidden <= 0 || d->inter <= 0) return false;
+    if (d->n_layers > 4096 || d->hidden > (1 << 24) || d->inter > (1 << 24)) return false;
     if (d->n_branches < 1 || d->n_branches > 2) return false;
     const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
     if (d->flags & ~LB_STACK_MLP_ONLY) return false;
@@ -134,41 +142,69 @@ bool proj_used(const lb_stack_desc* d, int p) {
     return !(d->flags & LB_STACK_MLP_ONLY) || p >= LB_GATE;
 }
 
+// The phases of one decoder layer (or of the MLP-only block): which
+// projections each phase covers and whether it is the first contraction.
+struct PhaseSpec {
+    int projs[3];
+    int n_projs;
+    bool first;      // first contraction (writes t) or second (writes outputs)
+    int norm;        // -1, or which RMSNorm sum of squares (0 attention, 1 MLP)
+};
+
+std::vector<PhaseSpec> layer_phases(bool mlp_only) {
+    if (mlp_only)
+        return {{{LB_GATE, LB_UP, 0}, 2, true, -1}, {{LB_GATE, LB_UP, 0}, 2, false, -1},
+                {{LB_DOWN, 0, 0}, 1, true, -1}, {{LB_DOWN, 0, 0}, 1, false, -1}};
+    return {{{LB_Q, LB_K, LB_V}, 3, true, 0}, {{LB_Q, LB_K, LB_V}, 3, false, 0},
+            {{LB_O, 0, 0}, 1, true, -1},      {{LB_O, 0, 0}, 1, false, -1},
+            {{LB_GATE, LB_UP, 0}, 2, true, 1}, {{LB_GATE, LB_UP, 0}, 2, false, 1},
+            {{LB_DOWN, 0, 0}, 1, true, -1},   {{LB_DOWN, 0, 0}, 1, false, -1}};
+}
+
 StackLayout stack_layout(const lb_stack_desc* d) {
     StackLayout L;
     const int nl = d->n_layers, nb = d->n_branches;
-    size_t off = sizeof(WsHeader);
-    L.sumsq = off;
-    off = round_up(off + sizeof(float) * 2 * nl, 256);
-    L.t = off;
+    const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
+    const std::vector<PhaseSpec> spec = layer_phases(mlp_only);
+    L.sumsq_off.assign((size_t)nl * 2, 0);
     L.t_off.assign((size_t)nl * LB_N_PROJ * nb, 0);
     L.o_off.assign((size_t)nl * LB_N_PROJ, 0);
+    size_t off = sizeof(WsHeader);
     for (int l = 0; l < nl; ++l)
-        for (int p = 0; p < LB_N_PROJ; ++p) {
-            if (!proj_used(d, p)) continue;
-            const int64_t r = d->ranks[l * LB_N_PROJ + p];
-            for (int b = 0; b < nb; ++b) {
-                L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b] = off;
-                off = round_up(off + sizeof(float) * (size_t)r, 256);
+        for (const PhaseSpec& ps : spec) {
+            const size_t begin = off;
+            if (ps.first && ps.norm >= 0) {
+                L.sumsq_off[(size_t)l * 2 + ps.norm] = off;
+                off += 256;
             }
-        }
-    for (int l = 0; l < nl; ++l)
-        for (int p = 0; p < LB_N_PROJ; ++p) {
-            if (!proj_used(d, p) || p == LB_O || p == LB_DOWN) continue;
-            int64_t in, out;
-            proj_shape(d, p, in, out);
-            L.o_off[(size_t)l * LB_N_PROJ + p] = off;
-            off = round_up(off + sizeof(float) * (size_t)out, 256);
+            for (int i = 0; i < ps.n_projs; ++i) {
+                const int p = ps.projs[i];
+                if (ps.first) {
+                    const int64_t r = d->ranks[l * LB_N_PROJ + p];
+                    for (int b = 0; b < nb; ++b) {
+                        L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b] = off;
+                        off = round_up(off + sizeof(float) * (size_t)r, 256);
+                    }
+                } else if (p != LB_O && p != LB_DOWN) {
+                    int64_t in, out;
+                    proj_shape(d, p, in, out);
+                    L.o_off[(size_t)l * LB_N_PROJ + p] = off;
+                    off = round_up(off + sizeof(float) * (size_t)out, 256);
+                }
+            }
+            L.region_off.push_back(begin);
+            L.region_len.push_back(off - begin);
         }
     L.acc_end = off;
     L.x_dev = off;
     off = round_up(off + 2 * (size_t)d->hidden, 256);
     L.y_dev = off;
     off = round_up(off + 4 * (size_t)d->hidden, 256);
-    const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
-    L.n_phases = mlp_only ? 4 : 8 * nl;
-    // jobs: per layer 2*(3+1+2+1)*nb = 14 nb (decoder); 2*(2+1)*nb = 6 nb (MLP only)
-    L.n_jobs = mlp_only ? 6 * nb : 14 * nb * nl;
+    L.n_phases = (int)spec.size() * nl;
+    // jobs: one per projection and branch in each of the two contractions
+    int per_layer = 0;
+    for (const PhaseSpec& ps : spec) per_layer += ps.n_projs * nb;
+    L.n_jobs = per_layer * nl;
     L.phases = off;
     off = round_up(off + sizeof(LbPhase) * (size_t)L.n_phases, 256);
     L.jobs = off;
@@ -182,132 +218,85 @@ void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
                       std::vector<LbPhase>& phases, std::vector<LbJob>& jobs) {
     const int nb = d->n_branches;
     const bool mlp_only = (d->flags & LB_STACK_MLP_ONLY) != 0;
+    const std::vector<PhaseSpec> spec = layer_phases(mlp_only);
     auto br = [&](int l, int p, int b) -> const lb_branch& {
         return d->lin[((size_t)l * LB_N_PROJ + p) * nb + b];
     };
+    auto at = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
     auto tptr = [&](int l, int p, int b) {
-        return reinterpret_cast<float*>(ws + L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b]);
+        return at(L.t_off[((size_t)l * LB_N_PROJ + p) * nb + b]);
     };
-    auto optr = [&](int l, int p) {
-        return reinterpret_cast<float*>(ws + L.o_off[(size_t)l * LB_N_PROJ + p]);
-    };
-    float* sumsq = reinterpret_cast<float*>(ws + L.sumsq);
+    auto optr = [&](int l, int p) { return at(L.o_off[(size_t)l * LB_N_PROJ + p]); };
     float* yres = const_cast<float*>(reinterpret_cast<const float*>(LB_TAG_Y));
-
-    auto new_phase = [&]() {
-        LbPhase ph = {};
-        ph.job_begin = (int)jobs.size();
-        return ph;
-    };
-    // First contraction of projection p of layer l over vector source (kind, src...).
-    auto stage1 = [&](LbPhase& ph, int l, int p, int kind, const void* src, const float* src2,
-                      float* acc_sumsq, float* resid_init, int b) {
-        int64_t in, out;
-        proj_shape(d, p, in, out);
-        const int64_t r = d->ranks[l * LB_N_PROJ + p];
-        LbJob J = {};
-        J.P = br(l, p, b).Vp;
-        set_job_shape(J, r, in);
-        J.kind = kind;
-        J.src = src;
-        J.src2 = src2;
-        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).g);
-        J.out = tptr(l, p, b);
-        J.acc_sumsq = acc_sumsq;
-        J.resid_init = resid_init;
-        J.gqa_hd = d->head_dim;
-        J.gqa_ghd = d->n_kv_heads > 0 ? d->head_dim * (d->n_heads / d->n_kv_heads) : 1;
-        add_job(ph, jobs, J);
-    };
-    auto stage2 = [&](LbPhase& ph, int l, int p, float* out_ptr, const float* norm, int b) {
-        int64_t in, out;
-        proj_shape(d, p, in, out);
-        const int64_t r = d->ranks[l * LB_N_PROJ + p];
-        LbJob J = {};
-        J.P = br(l, p, b).Up;
-        set_job_shape(J, out, r);
-        J.kind = VK_T;
-        J.src = tptr(l, p, b);
-        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).l);
-        J.oscale = reinterpret_cast<const __half*>(br(l, p, b).h);
-        J.out = out_ptr;
-        J.norm_sumsq = norm;
-        J.norm_n = d->hidden;
-        add_job(ph, jobs, J);
-    };
-
-    if (mlp_only) {
-        LbPhase p0 = new_phase();
-        for (int p : {LB_GATE, LB_UP})
-            for (int b = 0; b < nb; ++b)
-                stage1(p0, 0, p, VK_X_BF16, LB_TAG_X, nullptr, nullptr, nullptr, b);
-        p0.zero_ptr = yres;
-        p0.zero_n = d->hidden;
-        phases.push_back(p0);
-        LbPhase p1 = new_phase();
-        for (int p : {LB_GATE, LB_UP})
-            for (int b = 0; b < nb; ++b) stage2(p1, 0, p, optr(0, p), nullptr, b);
-        phases.push_back(p1);
-        LbPhase p2 = new_phase();
-        for (int b = 0; b < nb; ++b)
-            stage1(p2, 0, LB_DOWN, VK_SILU_MUL, optr(0, LB_GATE), optr(0, LB_UP), nullptr,
-                   nullptr, b);
-        phases.push_back(p2);
-        LbPhase p3 = new_phase();
-        for (int b = 0; b < nb; ++b) stage2(p3, 0, LB_DOWN, yres, nullptr, b);
-        phases.push_back(p3);
-        return;
-    }
+    const int gqa_group = (!mlp_only && d->n_kv_heads > 0) ? d->n_heads / d->n_kv_heads : 1;
 
     for (int l = 0; l < d->n_layers; ++l) {
-        float* ss_attn = sumsq + 2 * l;
-        float* ss_mlp = sumsq + 2 * l + 1;
-        // q, k, v first contractions: input rmsnorm(h); layer 0 reads x and seeds h.
-        LbPhase a = new_phase();
-        bool first = true;
-        for (int p : {LB_Q, LB_K, LB_V})
-            for (int b = 0; b < nb; ++b) {
-                if (l == 0)
-                    stage1(a, l, p, VK_X_BF16, LB_TAG_X, nullptr, first ? ss_attn : nullptr,
-                           first ? yres : nullptr, b);
-                else
-                    stage1(a, l, p, VK_X_F32, LB_TAG_Y, nullptr, first ? ss_attn : nullptr,
-                           nullptr, b);
-                first = false;
+        for (const PhaseSpec& ps : spec) {
+            LbPhase ph = {};
+            ph.job_begin = (int)jobs.size();
+            float* norm = ps.norm >= 0 ? at(L.sumsq_off[(size_t)l * 2 + ps.norm]) : nullptr;
+            bool first_job = true;
+            for (int i = 0; i < ps.n_projs; ++i) {
+                const int p = ps.projs[i];
+                int64_t in, out;
+                proj_shape(d, p, in, out);
+                const int64_t r = d->ranks[l * LB_N_PROJ + p];
+                for (int b = 0; b < nb; ++b) {
+                    LbJob J = {};
+                    if (ps.first) {
+                        J.P = br(l, p, b).Vp;
+                        set_job_shape(J, r, in);
+                        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).g);
+                        J.out = tptr(l, p, b);
+                        if (p == LB_O) {
+                            J.kind = VK_GQA;
+                            J.src = optr(l, LB_V);
+                            J.gqa_hd = d->head_dim;
+                            J.gqa_ghd = d->head_dim * gqa_group;
+                        } else if (p == LB_DOWN) {
+                            J.kind = VK_SILU_MUL;
+                            J.src = optr(l, LB_GATE);
+                            J.src2 = optr(l, LB_UP);
+                        } else if (mlp_only || (l == 0 && p <= LB_V)) {
+                            // the call's bf16 input; layer 0's q/k/v also seed the residual
+                            J.kind = VK_X_BF16;
+                            J.src = LB_TAG_X;
+                            if (!mlp_only && first_job && p == LB_Q) J.resid_init = yres;
+                        } else {
+                            J.kind = VK_X_F32;
+                            J.src = LB_TAG_Y;
+                        }
+                        if (first_job && norm) J.acc_sumsq = norm;
+                    } else {
+                        J.P = br(l, p, b).Up;
+                        set_job_shape(J, out, r);
+                        J.kind = VK_T;
+                        J.src = tptr(l, p, b);
+                        J.vscale = reinterpret_cast<const __half*>(br(l, p, b).l);
+                        J.oscale = reinterpret_cast<const __half*>(br(l, p, b).h);
+                        J.out = (p == LB_O || p == LB_DOWN) ? yres : optr(l, p);
+                        J.norm_sumsq = norm;
+                        J.norm_n = d->hidden;
+                    }
+                    first_job = false;
+                    add_job(ph, jobs, J);
+                }
             }
-        phases.push_back(a);
-        LbPhase bq = new_phase();
-        for (int p : {LB_Q, LB_K, LB_V})
-            for (int b = 0; b < nb; ++b) stage2(bq, l, p, optr(l, p), ss_attn, b);
-        phases.push_back(bq);
-        LbPhase c = new_phase();
-        for (int b = 0; b < nb; ++b)
-            stage1(c, l, LB_O, VK_GQA, optr(l, LB_V), nullptr, nullptr, nullptr, b);
-        phases.push_back(c);
-        LbPhase e = new_phase();
-        for (int b = 0; b < nb; ++b) stage2(e, l, LB_O, yres, nullptr, b);
-        phases.push_back(e);
-        LbPhase f = new_phase();
-        first = true;
-        for (int p : {LB_GATE, LB_UP})
-            for (int b = 0; b < nb; ++b) {
-                stage1(f, l, p, VK_X_F32, LB_TAG_Y, nullptr, first ? ss_mlp : nullptr, nullptr,
-                       b);
-                first = false;
-            }
-        phases.push_back(f);
-        LbPhase g = new_phase();
-        for (int p : {LB_GATE, LB_UP})
-            for (int b = 0; b < nb; ++b) stage2(g, l, p, optr(l, p), ss_mlp, b);
-        phases.push_back(g);
-        LbPhase h = new_phase();
-        for (int b = 0; b < nb; ++b)
-            stage1(h, l, LB_DOWN, VK_SILU_MUL, optr(l, LB_GATE), optr(l, LB_UP), nullptr,
-                   nullptr, b);
-        phases.push_back(h);
-        LbPhase k = new_phase();
-        for (int b = 0; b < nb; ++b) stage2(k, l, LB_DOWN, yres, nullptr, b);
-        phases.push_back(k);
+            phases.push_back(ph);
+        }
+    }
+    // Phase p zeroes the region of phase p+1; the last phase zeroes region 0
+    // for the next call.  The MLP-only block's final phase accumulates into y.
+    const int n = (int)phases.size();
+    for (int p = 0; p < n; ++p) {
+        const int q = (p + 1) % n;
+        if (mlp_only && q == n - 1) {
+            phases[p].zero_ptr = yres;
+            phases[p].zero_n = d->hidden;
+        } else if (L.region_len[q] > 0) {
+            phases[p].zero_ptr = at(L.region_off[q]);
+            phases[p].zero_n = (int)(L.region_len[q] / sizeof(float));
+        }
     }
 }
 
@@ -359,20 +348,21 @@ lb_status lb_pack_signs(const float* latent, int64_t rows, int64_t cols, int64_t
                : LB_ERR_CUDA;
 }
 
+// The tensor-core path runs for at least kPrefillMinM rows when the shapes
+// allow its 64-wide K blocks.
+static bool use_prefill(int64_t M, int64_t in, int64_t out, int64_t r) {
+    return M >= kPrefillMinM && prefill_shape_ok(M, in, out, r);
+}
+
 size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r, int n_branches) {
-    (void)in;
-    (void)out;
-    if (M <= 0 || r <= 0 || n_branches < 1 || n_branches > 2) return 0;
+    if (M <= 0 || in <= 0 || out <= 0 || r <= 0 || n_branches < 1 || n_branches > 2) return 0;
+    if (use_prefill(M, in, out, r)) return prefill_workspace_bytes(M, in, r);
     const int64_t mc = std::min<int64_t>(M, kMaxDecodeM);
     return sizeof(WsHeader) + round_up(sizeof(float) * (size_t)(mc * n_branches * r), 256);
 }
 
 int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r) {
-    (void)M;
-    (void)in;
-    (void)out;
-    (void)r;
-    return 0;
+    return use_prefill(M, in, out, r) ? 1 : 0;
 }
 
 lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t in, int64_t out,
@@ -393,6 +383,15 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
     if (st != LB_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_prefill(M, in, out, r)) {
+        bool scales16 = true;   // the tensor-core path reads g in 16-byte vectors
+        for (int b = 0; b < n_branches; ++b) scales16 = scales16 && aligned(br[b].g, 16);
+        if (scales16)
+            return launch_prefill(x, vec_kind_for(x_dtype), M, in, out, r, br, n_branches, y,
+                                  workspace, s) == cudaSuccess
+                       ? LB_OK
+                       : LB_ERR_CUDA;
+    }
     const size_t xsz = x_dtype == LB_F32 ? 4 : 2;
     WsHeader* hdr = static_cast<WsHeader*>(workspace);
     float* t = reinterpret_cast<float*>(static_cast<char*>(workspace) + sizeof(WsHeader));
@@ -469,6 +468,7 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
     if ((int)phases.size() != L.n_phases || (int)jobs.size() != L.n_jobs) return LB_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
+    if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
     if (cudaMemcpyAsync(ws + L.phases, phases.data(), sizeof(LbPhase) * phases.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
@@ -489,7 +489,6 @@ lb_status lb_stack_forward(const lb_stack_desc* d, void* workspace, size_t ws_by
     if (st != LB_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
-    if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
     if (launch_stack_plan(reinterpret_cast<const LbPhase*>(ws + L.phases),
                           reinterpret_cast<const LbJob*>(ws + L.jobs), L.n_phases,
                           reinterpret_cast<WsHeader*>(ws), x, y, s) != cudaSuccess)

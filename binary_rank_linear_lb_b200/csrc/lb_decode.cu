@@ -7,67 +7,115 @@
 // Each contraction is a GEMV whose matrix is a packed sign matrix P[rows][cols]
 // and whose vector v is built on the fly (g o x, l o t, ...).
 //
-// Lookup tables.  For a slice of 1024 columns the CTA tabulates, for every
+// Lookup tables.  For a slice of 512 columns the CTA tabulates, for every
 // chunk of 8 consecutive columns, all 256 signed sums  T_c[e] = sum_q (bit q of
 // e ? -v_q : +v_q).  One byte of a packed row then costs one shared-memory load
-// and one add instead of eight sign-selects and adds.  Table layout (bytes):
-//   lut + (qb>>1)*64K + e*256 + (qb&1)*128 + w*4    chunk c = 4w + qb
-// so the 32 lanes of a warp, which always look up 32 different words w, hit 32
-// different banks.  A single PRMT assembles the address from the sign byte and
-// a per-lane constant, so a lookup is PRMT + LDS + FADD.
+// and one add.  With chunk c = 4w + qb (word w = 4*gam + reg of the slice, byte
+// qb of the word) the table entry lives at byte
+//     e*256 + (reg&1)*128 + 4*(8*gam + 4*(reg>>1) + qb)
+// of the 64 KB table, i.e. in bank 8*gam + 4*(reg>>1) + qb.
+//
+// Lane mapping of the lookups.  Lane l = 4*rho + gam (rho = 0..7 picks one of 8
+// rows of a step, gam = 0..3 one of four 16-byte word groups of the row).  At
+// step (r, jj) the lane reads register r of its group (with the two halves of
+// the group swapped when rho >= 4) and byte (jj + rho) % 4 of that word, so
+// the 32 lanes touch 32 chunks in 32 different banks.  A single PRMT merges the
+// sign byte (the entry index) with a per-lane constant into the address, so a
+// lookup is PRMT + LDS + FADD.
 //
 // Work split.  A job (one matrix) is cut into units of 32 rows x one slice.
 // The units of a phase are dealt to the CTAs in contiguous, equal ranges; a CTA
 // rebuilds its table whenever its range enters a new (job, slice).  Partial
-// row sums over a slice are added to the fp32 output with red.global.add, so the
-// V-contraction result t never leaves L2 between the two phases.
+// row sums over a slice go to the fp32 output with red.global.add, so the
+// V-contraction result t stays in L2 between the two phases.
 //
 // Phases are separated by a grid-wide wait (bounded spin); the kernel is
-// launched cooperatively so that every CTA is resident.  While waiting, HBM is
-// kept busy by L2 prefetches of the next phase's first sign rows.
+// launched cooperatively so that every CTA is resident.  At the start of each
+// phase a CTA issues L2 prefetches for the sign rows it will read in the next
+// phase, so HBM keeps streaming through the waits.
 #include "lb_internal.cuh"
 
 namespace lb {
 namespace {
 
 constexpr long long kSpinLimitCycles = 4000000000LL;   // ~2 s at 2 GHz
-constexpr int kPrefetchUnits = 8;                       // units prefetched per CTA ahead
+constexpr int kPrefetchSegments = 2048;                 // next-phase 64-byte segments per CTA
 constexpr int kPrefetchAhead = 2 * kDecodeWarps;        // rowblocks ahead within a tile
-constexpr int kVecPad = kSliceElems + kSliceElems / 32; // padded staged vector
 
 struct Smem {
-    uint32_t lut;     // shared-window address of the table, a multiple of 64 KB
+    uint32_t lut;     // shared-window address of the 64 KB table
     float* vec;       // staged vector slice, index e + e/32
     float* red;       // 32 floats of reduction scratch
     int* flag;        // one int
+    LbPhase* phase;   // the current phase, copied from the plan
+    LbJob* jobs;      // its jobs (at most kMaxPhaseJobs), copied from the plan
 };
 
 __device__ __forceinline__ Smem smem_layout() {
     extern __shared__ __align__(16) unsigned char dsmem[];
     Smem s;
-    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsmem);
-    s.lut = (sbase + 65535u) & ~65535u;
-    unsigned char* after = dsmem + (s.lut - sbase) + kLutBytes;
-    s.vec = reinterpret_cast<float*>(after);
+    s.lut = (uint32_t)__cvta_generic_to_shared(dsmem);
+    s.vec = reinterpret_cast<float*>(dsmem + kLutBytes);
     s.red = s.vec + kVecPad;
     s.flag = reinterpret_cast<int*>(s.red + 32);
+    s.phase = reinterpret_cast<LbPhase*>(dsmem + kLutBytes + 4 * kVecPad + 4 * 32 + 64);
+    s.jobs = reinterpret_cast<LbJob*>(s.phase + 1);
     return s;
+}
+
+// Copy phase ph and its jobs into shared memory (plan data never changes
+// during a call, so this can run before the grid-wide wait).
+__device__ void cache_phase(const LbPhase* phases, int p, const LbJob* jobs, const Smem& sm) {
+    const LbPhase ph = phases[p];
+    if (threadIdx.x == 0) *sm.phase = ph;
+    const int n_words = ph.n_jobs * (int)(sizeof(LbJob) / 4);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(jobs + ph.job_begin);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(sm.jobs);
+    for (int i = threadIdx.x; i < n_words; i += kDecodeThreads) dst[i] = src[i];
 }
 
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
 
-// Grid-wide wait: every CTA adds one arrival, then waits until `target`
-// arrivals are counted.  Gives up after kSpinLimitCycles and records
-// LB_ERR_TIMEOUT; returns false if this CTA must stop.
-__device__ bool grid_sync(WsHeader* hdr, unsigned target, int* flag) {
+struct CallArgs {
+    const void* x;
+    float* y;
+};
+
+template <typename T>
+__device__ __forceinline__ T* resolve(T* p, const CallArgs& a) {
+    if ((const void*)p == LB_TAG_X) return (T*)a.x;
+    if ((const void*)p == LB_TAG_Y) return (T*)a.y;
+    return p;
+}
+
+// Local copy of a job with the call's x / y substituted for their tags.
+__device__ __forceinline__ LbJob fetch_job(const LbJob* jobs, int j, const CallArgs& a) {
+    LbJob J = jobs[j];
+    J.src = resolve(J.src, a);
+    J.out = resolve(J.out, a);
+    J.resid_init = resolve(J.resid_init, a);
+    return J;
+}
+
+// Grid-wide wait, split in two so a CTA can issue the next phase's loads and
+// prefetches between announcing that it is done (grid_arrive) and waiting for
+// everyone else (grid_wait).  The arrival is a release-add: every write of the
+// CTA made before it (ordered by the preceding __syncthreads) is visible to a
+// CTA whose acquire-load sees the count.  The wait gives up after
+// kSpinLimitCycles and records LB_ERR_TIMEOUT; it returns false if this CTA
+// must stop.
+__device__ __forceinline__ void grid_arrive(WsHeader* hdr) {
     __syncthreads();
+    if (threadIdx.x == 0) red_release_add_u32(&hdr->barrier, 1u);
+}
+
+__device__ bool grid_wait(WsHeader* hdr, unsigned target, int* flag) {
     if (threadIdx.x == 0) {
-        __threadfence();
-        red_release_add_u32(&hdr->barrier, 1u);
         int ok = 1;
         const long long t0 = clock64();
         unsigned spins = 0;
         while (ld_acquire_u32(&hdr->barrier) < target) {
+            __nanosleep(32);
             if ((++spins & 63u) == 0) {
                 if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) { ok = 0; break; }
                 if (clock64() - t0 > kSpinLimitCycles) {
@@ -88,14 +136,15 @@ __device__ __forceinline__ int unit_split(int n, int cta, int G) {
     return (int)(((long long)n * cta) / G);
 }
 
-// Stage v for slice s of job J into shared memory (zero past cols), do the
-// slice owner's side duties, then build the 128 chunk tables.
-__device__ void stage_and_build(const LbJob& J, int s, bool owner, const Smem& sm) {
+// Stage v for slice s of job J into shared memory (zero past cols) and do the
+// slice owner's side duties (sum of squares for RMSNorm, residual seeding).
+__device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm) {
     const int j0 = s * kSliceElems;
     float rs = 1.0f;
     if (J.kind == VK_T && J.norm_sumsq != nullptr)
         rs = rsqrtf(__ldcg(J.norm_sumsq) / (float)J.norm_n + kRmsEps);
     float sq = 0.0f;
+#pragma unroll
     for (int e = threadIdx.x; e < kSliceElems; e += kDecodeThreads) {
         const int j = j0 + e;
         float v = 0.0f;
@@ -151,12 +200,17 @@ __device__ void stage_and_build(const LbJob& J, int s, bool owner, const Smem& s
         }
     }
     __syncthreads();
+}
 
-    // Table build.  Warp wp fills byte position qb = wp/4 of every word and
-    // the 4 high nibbles (wp%4)*4 .. +3; lane = word w of the slice.
+// Build the 64 chunk tables of the staged slice.  Warp wp fills words with
+// reg & 1 == wp & 1 and high nibbles (wp >> 1)*4 .. +3; lane = 8*gam + 4*h2 + qb
+// owns chunk 4*(4*gam + 2*h2 + (wp&1)) + qb, which sits in bank `lane`.
+__device__ void build_lut(const Smem& sm) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int qb = wp >> 2, hb = (wp & 3) * 4;
-    const float* u = sm.vec + 32 * lane + 8 * qb + lane;   // padded index of element 32w+8qb
+    const int gam = lane >> 3, h2 = (lane >> 2) & 1, qb = lane & 3;
+    const int w = 4 * gam + 2 * h2 + (wp & 1);
+    const int e0 = 32 * w + 8 * qb;                    // first element of the chunk
+    const float* u = sm.vec + e0 + (e0 >> 5);
     const float u0 = u[0], u1 = u[1], u2 = u[2], u3 = u[3];
     const float u4 = u[4], u5 = u[5], u6 = u[6], u7 = u[7];
     // bit q of the entry index set <=> element q enters with sign -1
@@ -167,8 +221,8 @@ __device__ void stage_and_build(const LbJob& J, int s, bool owner, const Smem& s
     float lo[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) lo[m] = p01[m & 3] + p23[m >> 2];
-    const uint32_t base = sm.lut + (uint32_t)(qb >> 1) * 65536u + (uint32_t)(qb & 1) * 128u +
-                          (uint32_t)lane * 4u;
+    const uint32_t base = sm.lut + (uint32_t)(wp & 1) * 128u + (uint32_t)lane * 4u;
+    const int hb = (wp >> 1) * 4;
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
         const int hn = hb + n;
@@ -199,80 +253,89 @@ __device__ __forceinline__ uint4 load_group(const LbJob& J, int row, int wbase, 
     return d;
 }
 
-__device__ __forceinline__ void prefetch_rowblock(const LbJob& J, int s, int rb, int lane) {
-    const int row = rb * kRowBlock + lane;
+// L2 prefetch of the slice-s segment of one row.
+__device__ __forceinline__ void prefetch_segment(const LbJob& J, int s, int row) {
     const int w0 = s * kSliceWords;
     if (row < J.rows && w0 < J.ldw) {
         const uint32_t* p = J.P + (size_t)row * (size_t)J.ldw + w0;
         const int nw = min(kSliceWords, J.ldw - w0);
         prefetch_l2(p);
-        const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) >> 7;
-        const uintptr_t a1 = reinterpret_cast<uintptr_t>(p + nw - 1) >> 7;
-        if (a1 != a0) prefetch_l2(p + nw - 1);
+        if ((reinterpret_cast<uintptr_t>(p) >> 7) != (reinterpret_cast<uintptr_t>(p + nw - 1) >> 7))
+            prefetch_l2(p + nw - 1);
     }
 }
 
 // Look up rowblocks [rb0, rb0+nrb) of slice s of job J against the table.
-// Lane l = 8*rho + gam reads words 4*gam..4*gam+3 of row 4*i + rho of the
-// rowblock (i = 0..7) and, in step jj, byte (jj + rho) % 4 of each word, so the
-// 32 lanes of a warp always touch 32 different words.
-__device__ void lookup_rowblocks(const LbJob& J, int s, int rb0, int nrb, const Smem& sm) {
+template <bool kZeroBase>
+__device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0, int nrb,
+                                                 const Smem& sm, uint4 (&cur)[4]) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int rho = lane >> 3, gam = lane & 7;
-    uint32_t B[4], S[4];
+    const int rho = lane >> 2, gam = lane & 3;
+    const uint32_t swap = (uint32_t)(rho >> 2);          // 1: use the group's halves swapped
+    uint32_t B[2][4], S[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
         const uint32_t qbj = (uint32_t)((jj + rho) & 3);
-        B[jj] = ((qbj & 1u) * 128u + 16u * (uint32_t)gam) |
-                (((sm.lut >> 16) + (qbj >> 1)) << 16);
-        S[jj] = 0x7604u | (qbj << 4);
+        S[jj] = 0x7604u | (qbj << 4);                    // [B.b0, word.byte qbj, B.b2, B.b3]
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh)
+            B[rh][jj] = (8u * (uint32_t)gam + 4u * ((uint32_t)rh ^ swap) + qbj) * 4u;
     }
+    const uint32_t tbase = sm.lut;
     const int wbase = s * kSliceWords + 4 * gam;
     const bool vec4 = (J.ldw & 3) == 0;
-    const float hscale_default = 1.0f;
-    for (int rb = rb0 + wp; rb < rb0 + nrb; rb += kDecodeWarps) {
-        if (rb + kPrefetchAhead < rb0 + nrb) prefetch_rowblock(J, s, rb + kPrefetchAhead, lane);
-        const int row0 = rb * kRowBlock;
-        uint4 d[8];
+    const int rb_end = rb0 + nrb;
+
+    uint4 nxt[4];
+    int rb = rb0 + wp;
+    for (; rb < rb_end; rb += kDecodeWarps) {
+        const int rbn = rb + kDecodeWarps;
+        if (rbn < rb_end) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) d[i] = load_group(J, row0 + 4 * i + rho, wbase, vec4);
-        float acc[8];
+            for (int i = 0; i < 4; ++i)
+                nxt[i] = load_group(J, rbn * kRowBlock + 8 * i + rho, wbase, vec4);
+        }
+        if (rb + kPrefetchAhead < rb_end) prefetch_segment(J, s, (rb + kPrefetchAhead) * kRowBlock + lane);
+        float acc[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t w4[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
-            float a = 0.0f;
+        for (int i = 0; i < 4; ++i) {
+            // registers in the order this lane reads them (halves swapped for rho >= 4)
+            const uint32_t w4[4] = {swap ? cur[i].z : cur[i].x, swap ? cur[i].w : cur[i].y,
+                                    swap ? cur[i].x : cur[i].z, swap ? cur[i].y : cur[i].w};
+            float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-            for (int reg = 0; reg < 4; ++reg) {
+            for (int r = 0; r < 4; ++r) {
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    a += lds_f32(prmt(w4[reg], B[jj], S[jj]) + 4u * (uint32_t)reg);
+                for (int jj = 0; jj < 4; ++jj) {
+                    uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) + (uint32_t)(r & 1) * 128u;
+                    if (!kZeroBase) addr += tbase;
+                    const float v = lds_f32(addr);
+                    if (jj & 1) a1 += v; else a0 += v;
+                }
             }
-            acc[i] = a;
+            acc[i] = a0 + a1;
         }
-        // Transpose-reduce over the 8 lanes of a rho group: afterwards lane gam
-        // holds the full slice sum of row-step i = gam.
-        const bool up4 = (gam & 4) != 0, up2 = (gam & 2) != 0, up1 = (gam & 1) != 0;
-        float n4[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float send = up4 ? acc[k] : acc[k + 4];
-            const float keep = up4 ? acc[k + 4] : acc[k];
-            n4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
+        // Transpose-reduce over the 4 lanes of a row (gam = lane bits 0-1):
+        // afterwards lane gam holds the slice sum of row-step i = gam.
+        const bool up2 = (gam & 2) != 0, up1 = (gam & 1) != 0;
         float n2[2];
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-            const float send = up2 ? n4[k] : n4[k + 2];
-            const float keep = up2 ? n4[k + 2] : n4[k];
+            const float send = up2 ? acc[k] : acc[k + 2];
+            const float keep = up2 ? acc[k + 2] : acc[k];
             n2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
         }
         const float send1 = up1 ? n2[0] : n2[1];
         const float keep1 = up1 ? n2[1] : n2[0];
         const float tot = keep1 + __shfl_xor_sync(0xffffffffu, send1, 1);
-        const int row = row0 + 4 * gam + rho;
+        const int row = rb * kRowBlock + 8 * gam + rho;
         if (row < J.rows) {
-            const float hs = J.oscale ? __half2float(__ldg(J.oscale + row)) : hscale_default;
+            const float hs = J.oscale ? __half2float(__ldg(J.oscale + row)) : 1.0f;
             red_add_f32(J.out + row, tot * hs);
+        }
+        if (rbn < rb_end) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
         }
     }
 }
@@ -282,30 +345,24 @@ __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int
     return j;
 }
 
-struct CallArgs {
-    const void* x;
-    float* y;
-};
-
-template <typename T>
-__device__ __forceinline__ T* resolve(T* p, const CallArgs& a) {
-    if ((const void*)p == LB_TAG_X) return (T*)a.x;
-    if ((const void*)p == LB_TAG_Y) return (T*)a.y;
-    return p;
+// Sign words of this warp's first rowblock of a tile (issued before the
+// tile's vector is staged, so the load overlaps the table build).
+__device__ __forceinline__ void first_rows(const LbJob& J, int s, int rb0, int nrb,
+                                           uint4 (&cur)[4]) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const int rho = lane >> 2, gam = lane & 3;
+    const int rb = rb0 + wp;
+    const bool vec4 = (J.ldw & 3) == 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        cur[i] = rb < rb0 + nrb ? load_group(J, rb * kRowBlock + 8 * i + rho,
+                                             s * kSliceWords + 4 * gam, vec4)
+                                : make_uint4(0u, 0u, 0u, 0u);
 }
 
-// Local copy of a job with the call's x / y substituted for their tags.
-__device__ __forceinline__ LbJob fetch_job(const LbJob* jobs, int j, const CallArgs& a) {
-    LbJob J = jobs[j];
-    J.src = resolve(J.src, a);
-    J.out = resolve(J.out, a);
-    J.resid_init = resolve(J.resid_init, a);
-    return J;
-}
-
-__device__ void run_phase(const LbPhase& ph, const LbJob* jobs, const Smem& sm,
-                          const CallArgs& args) {
+__device__ void run_phase(const Smem& sm, const CallArgs& args) {
     const int G = gridDim.x, cta = blockIdx.x;
+    const LbPhase ph = *sm.phase;
     float* zp = resolve(ph.zero_ptr, args);
     if (zp != nullptr) {
         for (int i = cta * kDecodeThreads + threadIdx.x; i < ph.zero_n; i += G * kDecodeThreads)
@@ -313,34 +370,46 @@ __device__ void run_phase(const LbPhase& ph, const LbJob* jobs, const Smem& sm,
     }
     int u = unit_split(ph.n_units, cta, G);
     const int u_end = unit_split(ph.n_units, cta + 1, G);
-    int j = ph.job_begin;
-    const int j_end = ph.job_begin + ph.n_jobs;
+    int j = 0;
     while (u < u_end) {
-        j = find_job(jobs, j, j_end, u);
-        const LbJob J = fetch_job(jobs, j, args);
+        j = find_job(sm.jobs, j, ph.n_jobs, u);
+        const LbJob J = fetch_job(sm.jobs, j, args);
         const int local = u - J.unit_begin;
         const int s = local / J.n_rowblocks;
         const int rb0 = local - s * J.n_rowblocks;
         const int nrb = min(J.n_rowblocks - rb0, u_end - u);
-        stage_and_build(J, s, rb0 == 0, sm);
-        lookup_rowblocks(J, s, rb0, nrb, sm);
+        uint4 cur[4];
+        first_rows(J, s, rb0, nrb, cur);
+        stage_vector(J, s, rb0 == 0, sm);
+        build_lut(sm);
+        if (sm.lut == 0u) lookup_rowblocks<true>(J, s, rb0, nrb, sm, cur);
+        else lookup_rowblocks<false>(J, s, rb0, nrb, sm, cur);
         u += nrb;
         __syncthreads();
     }
 }
 
-// L2 prefetch of the first kPrefetchUnits units this CTA will take in phase ph.
+// L2 prefetch of the sign segments this CTA will read in phase ph (up to
+// kPrefetchSegments of them, in the order it will read them).
 __device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs) {
     const int G = gridDim.x, cta = blockIdx.x;
-    const int u0 = unit_split(ph.n_units, cta, G);
-    const int u1 = min(unit_split(ph.n_units, cta + 1, G), u0 + kPrefetchUnits);
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    for (int u = u0 + wp; u < u1; u += kDecodeWarps) {
-        const int j = find_job(jobs, ph.job_begin, ph.job_begin + ph.n_jobs, u);
+    int u = unit_split(ph.n_units, cta, G);
+    const int u_end = unit_split(ph.n_units, cta + 1, G);
+    int j = ph.job_begin;
+    const int j_end = ph.job_begin + ph.n_jobs;
+    int budget = kPrefetchSegments;
+    while (u < u_end && budget > 0) {
+        j = find_job(jobs, j, j_end, u);
         const LbJob& J = jobs[j];
         const int local = u - J.unit_begin;
         const int s = local / J.n_rowblocks;
-        prefetch_rowblock(J, s, local - s * J.n_rowblocks, lane);
+        const int rb0 = local - s * J.n_rowblocks;
+        const int nrb = min(J.n_rowblocks - rb0, u_end - u);
+        const int rows = min(nrb * kRowBlock, budget);
+        for (int i = threadIdx.x; i < rows; i += kDecodeThreads)
+            prefetch_segment(J, s, rb0 * kRowBlock + i);
+        budget -= rows;
+        u += nrb;
     }
 }
 
@@ -348,22 +417,41 @@ __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jo
                             WsHeader* hdr, const CallArgs& args) {
     const Smem sm = smem_layout();
     const unsigned G = gridDim.x;
+    if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) return;   // sticky after a timeout
+    cache_phase(phases, 0, jobs, sm);
+    prefetch_phase(phases[0], jobs);
+    __syncthreads();
     for (int p = 0; p < n_phases; ++p) {
-        if (p + 1 < n_phases) prefetch_phase(phases[p + 1], jobs);
-        run_phase(phases[p], jobs, sm, args);
+        run_phase(sm, args);
         if (p + 1 < n_phases) {
-            if (!grid_sync(hdr, (unsigned)(p + 1) * G, sm.flag)) return;
+            // Announce completion, then use the wait: copy the next phase's
+            // plan into shared memory and prefetch its sign rows to L2.
+            grid_arrive(hdr);
+            cache_phase(phases, p + 1, jobs, sm);
+            prefetch_phase(phases[p + 1], jobs);
+            if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) return;
+        }
+    }
+    // The last CTA out resets the arrival counter for the next call.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&hdr->exit_count, 1u);
+        if (prev == G - 1) {
+            hdr->barrier = 0u;
+            hdr->exit_count = 0u;
+            __threadfence();
         }
     }
 }
 
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 linear_program_kernel(const __grid_constant__ LinearPlan plan, int n_phases, WsHeader* hdr) {
     const CallArgs args = {nullptr, nullptr};
     run_program(plan.phases, n_phases, plan.jobs, hdr, args);
 }
 
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 stack_program_kernel(const LbPhase* __restrict__ phases, const LbJob* __restrict__ jobs,
                      int n_phases, WsHeader* hdr, const void* x, float* y) {
     const CallArgs args = {x, y};
@@ -372,7 +460,7 @@ stack_program_kernel(const LbPhase* __restrict__ phases, const LbJob* __restrict
 
 cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)device_sm_count());
+    cfg.gridDim = dim3((unsigned)(device_sm_count() * kCtasPerSm));
     cfg.blockDim = dim3(kDecodeThreads);
     cfg.dynamicSmemBytes = kDecodeSmem;
     cfg.stream = s;
@@ -393,11 +481,14 @@ cudaError_t decode_configure() {
     e = cudaFuncSetAttribute(stack_program_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDecodeSmem);
     if (e != cudaSuccess) return e;
-    int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, linear_program_kernel, kDecodeThreads,
-                                                      kDecodeSmem);
-    if (e != cudaSuccess) return e;
-    return nb >= 1 ? cudaSuccess : cudaErrorCooperativeLaunchTooLarge;
+    for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
+                           reinterpret_cast<const void*>(stack_program_kernel)}) {
+        int nb = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kDecodeThreads, kDecodeSmem);
+        if (e != cudaSuccess) return e;
+        if (nb < kCtasPerSm) return cudaErrorCooperativeLaunchTooLarge;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,

@@ -17,15 +17,16 @@
 namespace lb {
 
 // ---------------------------------------------------------------- constants
-constexpr int kDecodeThreads = 512;          // 16 warps per CTA, one CTA per SM
+constexpr int kDecodeThreads = 256;          // 8 warps per CTA
 constexpr int kDecodeWarps = kDecodeThreads / 32;
-constexpr int kSliceElems = 1024;            // columns covered by one lookup table
+constexpr int kCtasPerSm = 2;                // two co-resident CTAs per SM
+constexpr int kSliceElems = 512;             // columns covered by one lookup table
 constexpr int kSliceWords = kSliceElems / 32;
-constexpr int kRowBlock = 32;                // rows per warp work item (8 steps x 4 rows)
-constexpr int kLutBytes = 128 * 1024;        // 128 chunks x 256 entries x fp32
-constexpr int kStageBytes = 8 * 1024;        // staged vector slice + scratch
-constexpr int kDecodeSmem = 64 * 1024 + kLutBytes + kStageBytes;  // worst-case alignment
+constexpr int kRowBlock = 32;                // rows per warp work item (4 steps x 8 rows)
+constexpr int kLutBytes = 64 * 1024;         // 64 chunks x 256 entries x fp32
+constexpr int kVecPad = kSliceElems + kSliceElems / 32;   // staged slice, padded
 constexpr int kMaxLinearJobs = 16;           // per phase in a single-linear call
+constexpr int kMaxPhaseJobs = 16;            // jobs of one phase (stack phases use <= 6)
 constexpr int kMaxDecodeM = 8;               // rows of x the decode path takes at once
 constexpr float kRmsEps = 1e-5f;
 
@@ -73,6 +74,9 @@ struct LbPhase {
 // job pointers that mean "the call's x" or "the call's y" are stored as tags.
 #define LB_TAG_X ((const void*)1)
 #define LB_TAG_Y ((const void*)2)
+
+constexpr int kDecodeSmem = kLutBytes + 4 * kVecPad + 4 * 32 + 64 + (int)sizeof(LbPhase) +
+                            kMaxPhaseJobs * (int)sizeof(LbJob);
 
 // Plan of a single linear call, passed by value as a kernel parameter.
 struct LinearPlan {
@@ -127,6 +131,15 @@ cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phas
                                cudaStream_t s);
 cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, int n_phases,
                               WsHeader* hdr, const void* x, float* y, cudaStream_t s);
+
+// Tensor-core prefill path (lb_prefill.cu).
+constexpr int kPrefillMinM = 16;             // lb_linear_forward uses it from this many rows
+cudaError_t prefill_configure();
+size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r);
+bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r);
+cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int64_t out,
+                           int64_t r, const lb_branch* br, int nb, float* y, void* workspace,
+                           cudaStream_t s);
 
 // Packer (lb_pack.cu).
 cudaError_t launch_pack(const float* latent, int64_t rows, int64_t cols, int64_t ld, int axis,

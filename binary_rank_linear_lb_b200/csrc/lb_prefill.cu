@@ -1,0 +1,609 @@
+// Large-M (prefill) path: the two contractions of the layer as tcgen05 GEMMs.
+//
+// The layer ("Samsung LittleBit: A 13B LLM Under 1 GB ...", "How it works",
+// items 1-3), for a block of M rows of x:
+//   stage 1:  T[m, b*r + k]  = l_b[k] * sum_j x[m, j] * (g_b[j] * sign(V_b[j, k]))
+//   stage 2:  y[m, i]        = sum_b sum_k T[m, b*r + k] * (h_b[i] * sign(U_b[i, k]))
+// Both are dense contractions, so they run on the 5th-generation tensor cores
+// (tcgen05.mma kind::f16: fp16 operands, fp32 accumulation in TMEM).
+//
+// Operands.  A (x, then T) is fp16, row-major, loaded by TMA with the 128-byte
+// swizzle.  B is never stored in HBM: producer warps expand the packed sign
+// bits in shared memory into fp16 tiles, each element a scale with its sign bit
+// flipped (g_b[j] for stage 1, h_b[i] for stage 2), which is exact in fp16.
+// Rows of x are brought into fp16 range by a power of two a_m; stage 1 writes
+// T multiplied by another power of two c_m chosen from the bound
+// |T[m, .]| <= max_k |l_k| * sum_j |g_j x[m, j]|, so T never overflows fp16 and
+// keeps fp16's relative precision.  Stage 2 divides c_m out again.
+//
+// Kernel shape: one CTA per SM, persistent over 128 x 256 output tiles,
+// warp-specialised: warp 0 issues TMA loads of A, warp 1 allocates TMEM and
+// issues the MMAs (one thread), warps 4-7 drain the double-buffered TMEM
+// accumulator, warps 8-11 expand B.  Four pipeline stages of
+// (A 16 KB + B 32 KB) in shared memory, synchronised with mbarriers.
+// Every wait is bounded: on time-out the kernel records LB_ERR_TIMEOUT, lets
+// every role finish, frees its TMEM and returns.
+#include <cuda.h>
+
+#include "lb_internal.cuh"
+
+namespace lb {
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kTileN = 256;
+constexpr int kBlockK = 64;                       // fp16 elements per stage (128 bytes)
+constexpr int kStages = 4;
+constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB
+constexpr int kBBytes = kTileN * kBlockK * 2;     // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kPrefillThreads = 384;              // 12 warps
+constexpr int kExpandWarp0 = 8;                   // warps 8..11 expand B
+constexpr int kExpandThreads = 128;
+constexpr int kEpiWarp0 = 4;                      // warps 4..7 drain TMEM
+constexpr int kTmemCols = 512;                    // two 256-column accumulators
+constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
+constexpr int kPrefillSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+struct Ctl {                 // shared control block
+    uint64_t full_a[kStages], full_b[kStages], empty[kStages];
+    uint64_t acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Bounded wait on an mbarrier phase; on time-out raises the CTA abort flag
+// and the workspace error.  Returns false if the caller must stop.
+__device__ __forceinline__ bool wait_bar(Ctl* c, uint64_t* bar, uint32_t parity, int* err) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&c->abort)) return false;
+        if (clock64() - t0 > kWaitLimit) {
+            atomicExch(&c->abort, 1);
+            atomicExch(err, (int)LB_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes (stride byte offset 1024), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, fp16 A and B, both
+// K-major, M = 128, N = 256.
+constexpr uint32_t kInstrDesc = (1u << 4) | ((uint32_t)(kTileN >> 3) << 17) |
+                                ((uint32_t)(kTileM >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(tmem_d), "l"(a), "l"(b), "r"(kInstrDesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 32 columns of fp32 from TMEM (one row per lane).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ problem
+// One GEMM of the prefill path.  N is cut into segments (stage 1: one per
+// branch, rows of Vp_b; stage 2: one, the output features) and K into segments
+// (stage 1: one, the input features; stage 2: one per branch, rows of T).
+struct PrefillGemm {
+    int M, n_seg_rows, n_nseg, n_kseg, k_seg_len;   // N = n_nseg * n_seg_rows, K = n_kseg * k_seg_len
+    int stage;                                       // 1 or 2
+    const uint32_t* P[2];                            // packed signs per branch
+    int ldw;                                         // words per packed row
+    const __half* bscale[2];                         // stage 1: g_b (per k); stage 2: h_b (per n)
+    const __half* lscale[2];                         // stage 1: l_b (per output column)
+    const float* row_sa;                             // [M] 2^a_m (stage 1 divides it out)
+    const float* row_sc;                             // [M] 2^c_m
+    __half* T;                                       // stage 1 output [M][n_nseg * n_seg_rows]
+    float* y;                                        // stage 2 output [M][n_seg_rows]
+    int* err;
+};
+
+namespace {
+
+__device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb, int& nseg,
+                                            int& nt) {
+    const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
+    const int n_tiles = g.n_nseg * nt_per_seg;
+    mb = t / n_tiles;
+    const int r = t - mb * n_tiles;
+    nseg = r / nt_per_seg;
+    nt = r - nseg * nt_per_seg;
+}
+
+// Expand one 256 x 64 B tile (K-major, 128-byte swizzle) from packed signs.
+// Thread e owns rows e and e + 128.
+__device__ void expand_b(const PrefillGemm& g, uint32_t b_smem, int nseg, int nt, int kseg,
+                         int kb, int e) {
+    const int branch = g.stage == 1 ? nseg : kseg;
+    const uint32_t* P = g.P[branch];
+    const int k0 = kb * kBlockK;                     // k within the segment
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int n = e + half * 128;                // row within the tile
+        const int row = nt * kTileN + n;             // row within the segment
+        uint2 bits = make_uint2(0u, 0u);
+        uint32_t nbase = 0u;                         // stage 2: h[row] in both halves
+        const bool valid = row < g.n_seg_rows;
+        if (valid) {
+            bits = __ldg(reinterpret_cast<const uint2*>(P + (size_t)row * g.ldw + k0 / 32));
+            if (g.stage == 2) {
+                const uint32_t hb = __half_as_ushort(__ldg(g.bscale[branch] + row));
+                nbase = hb | (hb << 16);
+            }
+        }
+        const uint32_t rowoff = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {               // 16-byte chunk: k0 + 8c .. +7
+            const uint32_t byte = ((c < 4 ? bits.x : bits.y) >> (8 * (c & 3))) & 0xFFu;
+            uint4 base;
+            if (g.stage == 1) {
+                base = __ldg(reinterpret_cast<const uint4*>(g.bscale[branch] + k0 + 8 * c));
+            } else {
+                base = make_uint4(nbase, nbase, nbase, nbase);
+            }
+            uint32_t o[4];
+            const uint32_t bw[4] = {base.x, base.y, base.z, base.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t m = ((byte >> (2 * p)) & 3u) * 0x40008000u;
+                o[p] = valid ? (bw[p] ^ (m & 0x80008000u)) : 0u;
+            }
+            const uint32_t addr = b_smem + rowoff + (uint32_t)((c ^ (n & 7)) * 16);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(addr), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ PrefillGemm g) {
+    extern __shared__ __align__(1024) unsigned char dsm[];
+    const uint32_t raw = smem_u32(dsm);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* basep = dsm + (base - raw);
+    Ctl* ctl = reinterpret_cast<Ctl*>(basep + kStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
+    const int n_tiles = ((g.M + kTileM - 1) / kTileM) * g.n_nseg * nt_per_seg;
+    const int kb_per_seg = g.k_seg_len / kBlockK;
+    const int n_kb = g.n_kseg * kb_per_seg;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&ctl->full_a[s]), 1);
+            mbar_init(smem_u32(&ctl->full_b[s]), kExpandThreads);
+            mbar_init(smem_u32(&ctl->empty[s]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&ctl->acc_full[i]), 1);
+            mbar_init(smem_u32(&ctl->acc_empty[i]), 128);
+        }
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(&ctl->tmem_base)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer for A
+        if (lane == 0) {
+            int it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
+                int mb, nseg, nt;
+                tile_coords(g, t, mb, nseg, nt);
+                for (int kb = 0; kb < n_kb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t par = ((it / kStages) & 1) ^ 1;
+                    if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) break;
+                    const uint32_t fb = smem_u32(&ctl->full_a[s]);
+                    mbar_expect_tx(fb, kABytes);
+                    const int kseg = kb / kb_per_seg;
+                    const int kcol = kseg * g.k_seg_len + (kb - kseg * kb_per_seg) * kBlockK;
+                    tma_load_2d(base + s * kStageBytes, &amap, fb, kcol, mb * kTileM);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            int it = 0, tl = 0;
+            for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x, ++tl) {
+                const int buf = tl & 1;
+                if (!wait_bar(ctl, &ctl->acc_empty[buf], ((tl >> 1) & 1) ^ 1, g.err)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * kTileN);
+                bool ok = true;
+                for (int kb = 0; kb < n_kb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t par = (it / kStages) & 1;
+                    if (!wait_bar(ctl, &ctl->full_a[s], par, g.err) ||
+                        !wait_bar(ctl, &ctl->full_b[s], par, g.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_s = base + s * kStageBytes;
+                    const uint64_t ad = sw128_desc(a_s), bd = sw128_desc(a_s + kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; ++kk)
+                        mma_f16(d, ad + 2ull * kk, bd + 2ull * kk, (kb | kk) != 0);
+                    mma_commit(smem_u32(&ctl->empty[s]));
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&ctl->acc_full[buf]));
+            }
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ---------------- epilogue: TMEM -> registers -> global
+        const int q = warp - kEpiWarp0;              // TMEM lane quarter
+        int tl = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+            int mb, nseg, nt;
+            tile_coords(g, t, mb, nseg, nt);
+            const int buf = tl & 1;
+            if (!wait_bar(ctl, &ctl->acc_full[buf], (tl >> 1) & 1, g.err)) break;
+            tc_fence_after();
+            const int m = mb * kTileM + q * 32 + lane;
+            const bool mok = m < g.M;
+            const float sa = mok ? __ldg(g.row_sa + m) : 1.0f;
+            const float sc = mok ? __ldg(g.row_sc + m) : 1.0f;
+            for (int c0 = 0; c0 < kTileN; c0 += 32) {
+                float v[32];
+                __syncwarp();
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTileN + c0), v);
+                const int n0 = nt * kTileN + c0;       // row within the N segment
+                if (!mok || n0 >= g.n_seg_rows) continue;
+                if (g.stage == 1) {
+                    // T = l * t * 2^c with t = D / 2^a
+                    const float f = sc / sa;
+                    __half* dst = g.T + (size_t)m * (g.n_nseg * g.n_seg_rows) +
+                                  (size_t)nseg * g.n_seg_rows + n0;
+                    const __half* lb = g.lscale[nseg] + n0;
+                    if (n0 + 32 <= g.n_seg_rows) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) {
+                                const float a0 = v[i + 2 * p] * f * __half2float(__ldg(lb + i + 2 * p));
+                                const float a1 =
+                                    v[i + 2 * p + 1] * f * __half2float(__ldg(lb + i + 2 * p + 1));
+                                const __half2 h2 = __floats2half2_rn(a0, a1);
+                                w[p] = *reinterpret_cast<const uint32_t*>(&h2);
+                            }
+                            *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        for (int i = 0; i < 32 && n0 + i < g.n_seg_rows; ++i)
+                            dst[i] = __float2half_rn(v[i] * f * __half2float(__ldg(lb + i)));
+                    }
+                } else {
+                    const float f = 1.0f / sc;
+                    float* dst = g.y + (size_t)m * g.n_seg_rows + n0;
+                    if (n0 + 32 <= g.n_seg_rows && (g.n_seg_rows & 3) == 0) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(dst + i) =
+                                make_float4(v[i] * f, v[i + 1] * f, v[i + 2] * f, v[i + 3] * f);
+                    } else {
+                        for (int i = 0; i < 32 && n0 + i < g.n_seg_rows; ++i) dst[i] = v[i] * f;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
+        }
+    } else if (warp >= kExpandWarp0) {
+        // ---------------- B producers: packed signs -> fp16 tile
+        const int e = threadIdx.x - kExpandWarp0 * 32;
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            int mb, nseg, nt;
+            tile_coords(g, t, mb, nseg, nt);
+            for (int kb = 0; kb < n_kb; ++kb, ++it) {
+                const int s = it % kStages;
+                const uint32_t par = ((it / kStages) & 1) ^ 1;
+                if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) { ok = false; break; }
+                const int kseg = kb / kb_per_seg;
+                expand_b(g, base + s * kStageBytes + kABytes, nseg, nt, kseg,
+                         kb - kseg * kb_per_seg, e);
+                fence_async_smem();                  // make the stores visible to the tensor core
+                mbar_arrive(smem_u32(&ctl->full_b[s]));
+            }
+        }
+    }
+
+    // Drain: every role is done (or aborted).  Give in-flight TMA loads time to
+    // land before the shared memory goes away, then free TMEM.
+    __syncthreads();
+    if (ctl->abort && threadIdx.x == 0) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 2000000LL) { }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// Pre-pass: per row m, 2^a_m (brings max|x| into [2^14, 2^15)), the fp16 copy
+// of x * 2^a_m, and 2^c_m (keeps |T| <= 65504; see the header comment).
+__global__ void __launch_bounds__(256) prefill_prepass_kernel(
+    const void* __restrict__ x, int x_kind, int M, int in, int nb,
+    const __half* __restrict__ g0, const __half* __restrict__ g1,
+    const float* __restrict__ lmax, __half* __restrict__ X16, float* __restrict__ row_sa,
+    float* __restrict__ row_sc) {
+    const int m = blockIdx.x;
+    __shared__ float red[3][8];
+    float mx = 0.0f, s0 = 0.0f, s1 = 0.0f;
+    for (int j = threadIdx.x; j < in; j += 256) {
+        float v;
+        if (x_kind == VK_X_F16) v = __half2float(reinterpret_cast<const __half*>(x)[(size_t)m * in + j]);
+        else if (x_kind == VK_X_BF16)
+            v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[(size_t)m * in + j]);
+        else v = reinterpret_cast<const float*>(x)[(size_t)m * in + j];
+        mx = fmaxf(mx, fabsf(v));
+        s0 += fabsf(v * __half2float(g0[j]));
+        if (nb > 1) s1 += fabsf(v * __half2float(g1[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = mx;
+        red[1][threadIdx.x >> 5] = s0;
+        red[2][threadIdx.x >> 5] = s1;
+    }
+    __syncthreads();
+    float M0 = 0.0f, L0 = 0.0f, L1 = 0.0f;
+    for (int w = 0; w < 8; ++w) {
+        M0 = fmaxf(M0, red[0][w]);
+        L0 += red[1][w];
+        L1 += red[2][w];
+    }
+    // 2^a: the largest power of two with max|x| * 2^a < 2^15
+    float sa = 1.0f;
+    if (M0 > 0.0f && isfinite(M0)) sa = exp2f(fminf(fmaxf(14.0f - floorf(log2f(M0)), -126.0f), 126.0f));
+    // 2^c: the largest power of two with bound * 2^c <= 2^15 (< 65504); the
+    // bound is padded by 1/64 for fp32 rounding in the sums.
+    const float bound = fmaxf(L0 * lmax[0], nb > 1 ? L1 * lmax[1] : 0.0f) * (1.0f + 1.0f / 64);
+    float sc = 1.0f;
+    if (bound > 0.0f && isfinite(bound))
+        sc = exp2f(fminf(fmaxf(15.0f - ceilf(log2f(bound)), -126.0f), 126.0f));
+    if (threadIdx.x == 0) {
+        row_sa[m] = sa;
+        row_sc[m] = sc;
+    }
+    for (int j = threadIdx.x; j < in; j += 256) {
+        float v;
+        if (x_kind == VK_X_F16) v = __half2float(reinterpret_cast<const __half*>(x)[(size_t)m * in + j]);
+        else if (x_kind == VK_X_BF16)
+            v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[(size_t)m * in + j]);
+        else v = reinterpret_cast<const float*>(x)[(size_t)m * in + j];
+        X16[(size_t)m * in + j] = __float2half_rn(v * sa);
+    }
+}
+
+// max_k |l_b[k]| for each branch (one block per branch).
+__global__ void __launch_bounds__(256) lmax_kernel(const __half* __restrict__ l0,
+                                                   const __half* __restrict__ l1, int r,
+                                                   float* __restrict__ out) {
+    const __half* l = blockIdx.x == 0 ? l0 : l1;
+    float mx = 0.0f;
+    for (int k = threadIdx.x; k < r; k += 256) mx = fmaxf(mx, fabsf(__half2float(l[k])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.0f;
+        for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+        out[blockIdx.x] = m;
+    }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode() {
+    static EncodeTiled fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+// Row-major fp16 [rows][cols] with a 64 x 128 box and the 128-byte swizzle.
+bool make_amap(CUtensorMap* map, const __half* ptr, int rows, int cols) {
+    EncodeTiled enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {kBlockK, kTileM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(ptr), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t prefill_configure() {
+    return cudaFuncSetAttribute(prefill_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kPrefillSmem);
+}
+
+size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    return up(sizeof(WsHeader)) + up(2 * (size_t)M * in) + up(2 * (size_t)M * 2 * r) +
+           up(8 * (size_t)M) + 256;
+}
+
+bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
+    return M >= 1 && in % kBlockK == 0 && r % kBlockK == 0 && out >= 1 && in <= (1 << 20) &&
+           r <= (1 << 16) && out <= (1 << 24) && M <= (1 << 24);
+}
+
+cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int64_t out,
+                           int64_t r, const lb_branch* br, int nb, float* y, void* workspace,
+                           cudaStream_t s) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    size_t off = up(sizeof(WsHeader));
+    __half* X16 = reinterpret_cast<__half*>(ws + off);
+    off += up(2 * (size_t)M * in);
+    __half* T = reinterpret_cast<__half*>(ws + off);
+    off += up(2 * (size_t)M * 2 * r);
+    float* sa = reinterpret_cast<float*>(ws + off);
+    float* sc = sa + M;
+    off += up(8 * (size_t)M);
+    float* lmax = reinterpret_cast<float*>(ws + off);
+
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
+    if (e != cudaSuccess) return e;
+    const __half* l1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].l);
+    lmax_kernel<<<nb, 256, 0, s>>>(reinterpret_cast<const __half*>(br[0].l), l1, (int)r, lmax);
+    const __half* g1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].g);
+    prefill_prepass_kernel<<<(unsigned)M, 256, 0, s>>>(
+        x, x_kind, (int)M, (int)in, nb, reinterpret_cast<const __half*>(br[0].g), g1, lmax, X16,
+        sa, sc);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const int grid = device_sm_count();
+    // stage 1: T = (x 2^a) (g o sign V)^T, epilogue applies l, 2^-a, 2^c
+    {
+        CUtensorMap amap;
+        if (!make_amap(&amap, X16, (int)M, (int)in)) return cudaErrorInvalidValue;
+        PrefillGemm p = {};
+        p.M = (int)M; p.n_seg_rows = (int)r; p.n_nseg = nb; p.n_kseg = 1; p.k_seg_len = (int)in;
+        p.stage = 1;
+        for (int b = 0; b < 2; ++b) {
+            const lb_branch& B = br[b < nb ? b : 0];
+            p.P[b] = B.Vp;
+            p.bscale[b] = reinterpret_cast<const __half*>(B.g);
+            p.lscale[b] = reinterpret_cast<const __half*>(B.l);
+        }
+        p.ldw = (int)((in + 31) / 32);
+        p.row_sa = sa; p.row_sc = sc; p.T = T; p.y = nullptr; p.err = &hdr->error;
+        prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // stage 2: y = (T) (h o sign U)^T over K = nb * r, epilogue divides 2^c out
+    {
+        CUtensorMap amap;
+        if (!make_amap(&amap, T, (int)M, (int)(nb * r))) return cudaErrorInvalidValue;
+        PrefillGemm p = {};
+        p.M = (int)M; p.n_seg_rows = (int)out; p.n_nseg = 1; p.n_kseg = nb; p.k_seg_len = (int)r;
+        p.stage = 2;
+        for (int b = 0; b < 2; ++b) {
+            const lb_branch& B = br[b < nb ? b : 0];
+            p.P[b] = B.Up;
+            p.bscale[b] = reinterpret_cast<const __half*>(B.h);
+            p.lscale[b] = nullptr;
+        }
+        p.ldw = (int)((r + 31) / 32);
+        p.row_sa = sa; p.row_sc = sc; p.T = nullptr; p.y = y; p.err = &hdr->error;
+        prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace lb

@@ -85,3 +85,53 @@ def test_workspace_reports_ok_and_repeat_calls_agree():
     y2 = lb.linear_forward(x, brs, in_f, out_f, r, workspace=ws)
     assert lb.workspace_status(ws) == lb.LB_OK
     torch.testing.assert_close(y1, y2, rtol=1e-5, atol=1e-4 * y1.abs().max().item())
+
+
+# ---------------------------------------------------------------- tensor-core path
+@pytest.mark.parametrize("shape", [(512, 256, 64), (640, 1000, 192), (1024, 1001, 128),
+                                   (4096, 11008, 128)])
+@pytest.mark.parametrize("M", [16, 100, 256])
+def test_prefill_path_shapes(shape, M):
+    in_f, out_f, r = shape
+    assert lb.linear_path(M, in_f, out_f, r) == 1
+    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=3)
+    for m in (0, M // 2, M - 1):
+        assert_close(got[m], ref[m], what=f"{shape} M={M} row {m}")
+    assert_close(got, ref, what=f"{shape} M={M}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+def test_prefill_path_dtypes_and_one_branch(dtype):
+    got, ref = run_case(768, 512, 128, 64, dtype, nb=1, base=4)
+    assert_close(got, ref, what=f"one branch {dtype}")
+
+
+@pytest.mark.parametrize("bpw", [1.0, 0.1])
+def test_prefill_7b_gate_sampled_rows(bpw):
+    """7B gate projection at M = 512; the oracle evaluates all rows of 8 sampled tokens."""
+    in_f, out_f = 4096, 11008
+    r = rank_for(bpw, in_f, out_f)
+    M = 512
+    brs = build_linear(in_f, out_f, r, base=5)
+    x = synth.activation((M, in_f), 55, torch.bfloat16, "cuda")
+    y = lb.linear_forward(x, brs, in_f, out_f, r)
+    torch.cuda.synchronize()
+    ob = oracle_linear(in_f, out_f, r, 5, 0, 0, 2)
+    toks = [0, 1, 127, 128, 255, 300, 510, 511]
+    ref = oracle.forward(to_f64(x[toks]), ob, in_f, out_f, r)
+    assert_close(y[toks].cpu().numpy(), ref, what=f"7B gate M=512 @ {bpw}")
+
+
+def test_prefill_large_activations_do_not_overflow():
+    """Rows of very different magnitude: the per-row powers of two keep fp16 in range."""
+    in_f, out_f, r = 512, 512, 128
+    brs = build_linear(in_f, out_f, r, base=6)
+    x = synth.activation((32, in_f), 66, torch.float32, "cuda")
+    x = x * torch.logspace(-20, 30, 32, base=2.0, device="cuda")[:, None]
+    y = lb.linear_forward(x, brs, in_f, out_f, r)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all()
+    ob = oracle_linear(in_f, out_f, r, 6, 0, 0, 2)
+    ref = oracle.forward(to_f64(x), ob, in_f, out_f, r)
+    for m in range(32):
+        assert_close(y[m].cpu().numpy(), ref[m], what=f"row {m}")
