@@ -77,7 +77,7 @@ bool branch_ok(const lb_branch& b) {
     return b.Vp && b.Up && b.h && b.g && b.l;
 }
 bool branch_aligned(const lb_branch& b) {
-    return aligned(b.Vp, 16) && aligned(b.Up, 16) && aligned(b.h, 2) && aligned(b.g, 2) &&
+    return aligned(b.Vp, 16) && aligned(b.Up, 16) && aligned(b.h, 4) && aligned(b.g, 2) &&
            aligned(b.l, 2);
 }
 

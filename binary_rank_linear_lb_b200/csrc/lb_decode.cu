@@ -40,11 +40,12 @@ namespace {
 
 constexpr long long kSpinLimitCycles = 4000000000LL;   // ~2 s at 2 GHz
 constexpr int kPrefetchSegments = 2048;                 // next-phase 64-byte segments per CTA
-constexpr int kPrefetchAhead = 2 * kDecodeWarps;        // rowblocks ahead within a tile
+constexpr int kMaxTiles = 4;                            // tiles whose vectors are staged together
 
 struct Smem {
     uint32_t lut;     // shared-window address of the 64 KB table
-    float* vec;       // staged vector slice, index e + e/32
+    uint32_t ring;    // per-warp rings of sign rowblocks (kRingSlots x 2 KB per warp)
+    float* vec;       // staged vector slices (kMaxTiles of them), index e + e/32
     float* red;       // 32 floats of reduction scratch
     int* flag;        // one int
     LbPhase* phase;   // the current phase, copied from the plan
@@ -55,10 +56,11 @@ __device__ __forceinline__ Smem smem_layout() {
     extern __shared__ __align__(16) unsigned char dsmem[];
     Smem s;
     s.lut = (uint32_t)__cvta_generic_to_shared(dsmem);
-    s.vec = reinterpret_cast<float*>(dsmem + kLutBytes);
-    s.red = s.vec + kVecPad;
+    s.ring = s.lut + kLutBytes;
+    s.vec = reinterpret_cast<float*>(dsmem + kLutBytes + kRingBytes);
+    s.red = s.vec + 4 * kVecPad;
     s.flag = reinterpret_cast<int*>(s.red + 32);
-    s.phase = reinterpret_cast<LbPhase*>(dsmem + kLutBytes + 4 * kVecPad + 4 * 32 + 64);
+    s.phase = reinterpret_cast<LbPhase*>(dsmem + kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64);
     s.jobs = reinterpret_cast<LbJob*>(s.phase + 1);
     return s;
 }
@@ -138,7 +140,7 @@ __device__ __forceinline__ int unit_split(int n, int cta, int G) {
 
 // Stage v for slice s of job J into shared memory (zero past cols) and do the
 // slice owner's side duties (sum of squares for RMSNorm, residual seeding).
-__device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm) {
+__device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm, float* vec) {
     const int j0 = s * kSliceElems;
     float rs = 1.0f;
     if (J.kind == VK_T && J.norm_sumsq != nullptr)
@@ -186,7 +188,7 @@ __device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm) 
                 if (J.resid_init != nullptr) J.resid_init[j] = raw;
             }
         }
-        sm.vec[e + (e >> 5)] = v;
+        vec[e + (e >> 5)] = v;
     }
     if (owner && J.acc_sumsq != nullptr) {
 #pragma unroll
@@ -198,19 +200,19 @@ __device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm) 
             for (int w = 0; w < kDecodeWarps; ++w) tot += sm.red[w];
             atomicAdd(J.acc_sumsq, tot);
         }
+        __syncthreads();
     }
-    __syncthreads();
 }
 
 // Build the 64 chunk tables of the staged slice.  Warp wp fills words with
 // reg & 1 == wp & 1 and high nibbles (wp >> 1)*4 .. +3; lane = 8*gam + 4*h2 + qb
 // owns chunk 4*(4*gam + 2*h2 + (wp&1)) + qb, which sits in bank `lane`.
-__device__ void build_lut(const Smem& sm) {
+__device__ void build_lut(const Smem& sm, const float* vec) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int gam = lane >> 3, h2 = (lane >> 2) & 1, qb = lane & 3;
     const int w = 4 * gam + 2 * h2 + (wp & 1);
     const int e0 = 32 * w + 8 * qb;                    // first element of the chunk
-    const float* u = sm.vec + e0 + (e0 >> 5);
+    const float* u = vec + e0 + (e0 >> 5);
     const float u0 = u[0], u1 = u[1], u2 = u[2], u3 = u[3];
     const float u4 = u[4], u5 = u[5], u6 = u[6], u7 = u[7];
     // bit q of the entry index set <=> element q enters with sign -1
@@ -222,9 +224,10 @@ __device__ void build_lut(const Smem& sm) {
 #pragma unroll
     for (int m = 0; m < 16; ++m) lo[m] = p01[m & 3] + p23[m >> 2];
     const uint32_t base = sm.lut + (uint32_t)(wp & 1) * 128u + (uint32_t)lane * 4u;
-    const int hb = (wp >> 1) * 4;
+    constexpr int kNibPerWarp = 16 / (kDecodeWarps / 2);
+    const int hb = (wp >> 1) * kNibPerWarp;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
+    for (int n = 0; n < kNibPerWarp; ++n) {
         const int hn = hb + n;
         const float hi = q45[hn & 3] + q67[hn >> 2];
 #pragma unroll
@@ -236,24 +239,9 @@ __device__ void build_lut(const Smem& sm) {
     __syncthreads();
 }
 
-// Sign words [wbase, wbase+4) of `row`, zero outside the matrix.
-__device__ __forceinline__ uint4 load_group(const LbJob& J, int row, int wbase, bool vec4) {
-    uint4 d = make_uint4(0u, 0u, 0u, 0u);
-    if (row < J.rows && wbase < J.ldw) {
-        const uint32_t* p = J.P + (size_t)row * (size_t)J.ldw + wbase;
-        if (vec4) {
-            d = ld_stream_v4(p);
-        } else {
-            d.x = ld_stream_u32(p);
-            if (wbase + 1 < J.ldw) d.y = ld_stream_u32(p + 1);
-            if (wbase + 2 < J.ldw) d.z = ld_stream_u32(p + 2);
-            if (wbase + 3 < J.ldw) d.w = ld_stream_u32(p + 3);
-        }
-    }
-    return d;
-}
-
-// L2 prefetch of the slice-s segment of one row.
+// L2 prefetch of the slice-s segment of one row (the one or two 128-byte
+// lines it touches; plain prefetches go through the LSU, which issues them far
+// faster than the bulk-copy engine would take one small request at a time).
 __device__ __forceinline__ void prefetch_segment(const LbJob& J, int s, int row) {
     const int w0 = s * kSliceWords;
     if (row < J.rows && w0 < J.ldw) {
@@ -265,13 +253,108 @@ __device__ __forceinline__ void prefetch_segment(const LbJob& J, int s, int row)
     }
 }
 
-// Look up rowblocks [rb0, rb0+nrb) of slice s of job J against the table.
-template <bool kZeroBase>
+// ---- per-warp ring of sign rowblocks, filled with cp.async ----------------
+// Lane l = 4*rho + gam copies exactly the 16 bytes it later reads (words
+// 4*gam .. 4*gam+3 of row 8*i + rho of the rowblock, i = 0..3) to
+// ring + slot*2KB + i*512 + l*16, so no cross-lane synchronisation is needed:
+// cp.async.wait_group on the lane's own groups is enough.  Bytes outside the
+// matrix are zero-filled (source size 0).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" :: "r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
+}
+
+// Slot layout: 4 row-steps x 32 lanes x 16 bytes of signs, then 32 lanes x
+// 4 bytes holding the fp16 row scale h of the lane's output row.
+__device__ __forceinline__ uint32_t ring_slot(const Smem& sm, int slot) {
+    return sm.ring + (uint32_t)((((threadIdx.x >> 5) * kRingSlots) + slot) * kRingSlotBytes) +
+           (uint32_t)(threadIdx.x & 31) * 16u;
+}
+__device__ __forceinline__ uint32_t ring_hslot(uint32_t slot_lane_addr) {
+    // slot base + 2048 + lane*4 (slot_lane_addr = slot base + lane*16)
+    const uint32_t lane = threadIdx.x & 31;
+    return slot_lane_addr - lane * 16u + (uint32_t)kRowBlockBytes + lane * 4u;
+}
+
+// Issue this lane's copies of rowblock rb (slice s) into the ring slot at dst.
+// Lanes with rho >= 4 store the two 8-byte halves of their 16 bytes swapped,
+// which is the order their lookups read them in.  The lane also copies the
+// 4-byte word holding h[row] of its output row (second contraction only).
+__device__ __forceinline__ void issue_rowblock(const LbJob& J, int s, int rb, uint32_t dst) {
+    const int lane = threadIdx.x & 31;
+    const int rho = lane >> 2, gam = lane & 3;
+    const uint32_t sw = (rho >> 2) ? 8u : 0u;
+    const int w = s * kSliceWords + 4 * gam;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int row = rb * kRowBlock + 8 * i + rho;
+        const bool rok = row < J.rows;
+        const uint32_t* p = rok ? J.P + (size_t)row * (size_t)J.ldw + w : J.P;
+        const uint32_t d = dst + (uint32_t)i * 512u;
+        if ((J.ldw & 1) == 0) {
+            cp_async_8(d + sw, p, (rok && w < J.ldw) ? 8u : 0u);
+            cp_async_8(d + (8u - sw), rok && w + 2 < J.ldw ? p + 2 : J.P,
+                       (rok && w + 2 < J.ldw) ? 8u : 0u);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                cp_async_4(d + (((uint32_t)(4 * q) + sw) & 15u), rok && w + q < J.ldw ? p + q : J.P,
+                           (rok && w + q < J.ldw) ? 4u : 0u);
+        }
+    }
+    if (J.oscale != nullptr) {
+        const int orow = rb * kRowBlock + 8 * gam + rho;
+        const int h0 = orow & ~1;                        // h is 4-byte aligned (checked on entry)
+        const uint32_t nb = orow >= J.rows ? 0u : (h0 + 1 < J.rows ? 4u : 2u);
+        cp_async_4(ring_hslot(dst), nb ? J.oscale + h0 : J.oscale, nb);
+    }
+}
+
+// Number of rowblocks warp wp takes in a tile of nrb rowblocks.
+__device__ __forceinline__ int warp_rowblocks(int nrb) {
+    const int wp = threadIdx.x >> 5;
+    return wp < nrb ? (nrb - wp + kDecodeWarps - 1) / kDecodeWarps : 0;
+}
+
+// First kRingDepth rowblocks of this warp's share of a tile (issued before the
+// tile's vector is staged, so the copies overlap staging and table build).
+// Always commits exactly kRingDepth groups.
+__device__ __forceinline__ void ring_prologue(const LbJob& J, int s, int rb0, int nrb,
+                                              const Smem& sm) {
+    const int wp = threadIdx.x >> 5;
+    const int nit = warp_rowblocks(nrb);
+#pragma unroll
+    for (int d = 0; d < kRingDepth; ++d) {
+        if (d < nit) issue_rowblock(J, s, rb0 + wp + d * kDecodeWarps, ring_slot(sm, d));
+        cp_async_commit();
+    }
+}
+
+// Look up this warp's rowblocks of slice s of job J against the table; the
+// rowblocks stream through the warp's ring kRingDepth ahead of use.  kBase is
+// the table's shared-window address when it is the usual 1024 (then it folds
+// into the load's immediate offset), else 0 and tbase is added at run time.
+template <uint32_t kBase>
 __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0, int nrb,
-                                                 const Smem& sm, uint4 (&cur)[4]) {
+                                                 const Smem& sm) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int rho = lane >> 2, gam = lane & 3;
-    const uint32_t swap = (uint32_t)(rho >> 2);          // 1: use the group's halves swapped
+    const uint32_t swap = (uint32_t)(rho >> 2);
     uint32_t B[2][4], S[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -279,41 +362,46 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
         S[jj] = 0x7604u | (qbj << 4);                    // [B.b0, word.byte qbj, B.b2, B.b3]
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh)
-            B[rh][jj] = (8u * (uint32_t)gam + 4u * ((uint32_t)rh ^ swap) + qbj) * 4u;
+            B[rh][jj] = (8u * (uint32_t)gam + 4u * ((uint32_t)rh ^ swap) + qbj) * 4u +
+                        (kBase == 0 ? sm.lut : 0u);
     }
-    const uint32_t tbase = sm.lut;
-    const int wbase = s * kSliceWords + 4 * gam;
-    const bool vec4 = (J.ldw & 3) == 0;
-    const int rb_end = rb0 + nrb;
-
-    uint4 nxt[4];
-    int rb = rb0 + wp;
-    for (; rb < rb_end; rb += kDecodeWarps) {
-        const int rbn = rb + kDecodeWarps;
-        if (rbn < rb_end) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                nxt[i] = load_group(J, rbn * kRowBlock + 8 * i + rho, wbase, vec4);
-        }
-        if (rb + kPrefetchAhead < rb_end) prefetch_segment(J, s, (rb + kPrefetchAhead) * kRowBlock + lane);
+    const int nit = warp_rowblocks(nrb);
+    const bool has_h = J.oscale != nullptr;
+    for (int n = 0; n < nit; ++n) {
+        const int rb = rb0 + wp + n * kDecodeWarps;
+        if (n + kRingDepth < nit)
+            issue_rowblock(J, s, rb + kRingDepth * kDecodeWarps,
+                           ring_slot(sm, (n + kRingDepth) % kRingSlots));
+        cp_async_commit();
+        cp_async_wait<kRingDepth>();                     // rowblock n has landed
+        const uint32_t src = ring_slot(sm, n % kRingSlots);
         float acc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            // registers in the order this lane reads them (halves swapped for rho >= 4)
-            const uint32_t w4[4] = {swap ? cur[i].z : cur[i].x, swap ? cur[i].w : cur[i].y,
-                                    swap ? cur[i].x : cur[i].z, swap ? cur[i].y : cur[i].w};
+            uint32_t w4[4];
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                         : "r"(src + (uint32_t)i * 512u));
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) + (uint32_t)(r & 1) * 128u;
-                    if (!kZeroBase) addr += tbase;
+                    const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) +
+                                          (uint32_t)(r & 1) * 128u + kBase;
                     const float v = lds_f32(addr);
                     if (jj & 1) a1 += v; else a0 += v;
                 }
             }
             acc[i] = a0 + a1;
+        }
+        const int orow = rb * kRowBlock + 8 * gam + rho;   // output row of this lane
+        float hs = 1.0f;
+        if (has_h) {
+            uint32_t hw;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hw) : "r"(ring_hslot(src)));
+            const unsigned short hb = (unsigned short)((orow & 1) ? (hw >> 16) : (hw & 0xFFFFu));
+            hs = __half2float(__ushort_as_half(hb));
         }
         // Transpose-reduce over the 4 lanes of a row (gam = lane bits 0-1):
         // afterwards lane gam holds the slice sum of row-step i = gam.
@@ -328,16 +416,9 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
         const float send1 = up1 ? n2[0] : n2[1];
         const float keep1 = up1 ? n2[1] : n2[0];
         const float tot = keep1 + __shfl_xor_sync(0xffffffffu, send1, 1);
-        const int row = rb * kRowBlock + 8 * gam + rho;
-        if (row < J.rows) {
-            const float hs = J.oscale ? __half2float(__ldg(J.oscale + row)) : 1.0f;
-            red_add_f32(J.out + row, tot * hs);
-        }
-        if (rbn < rb_end) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-        }
+        if (orow < J.rows) red_add_f32(J.out + orow, tot * hs);
     }
+    cp_async_wait<0>();
 }
 
 __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int u) {
@@ -345,19 +426,25 @@ __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int
     return j;
 }
 
-// Sign words of this warp's first rowblock of a tile (issued before the
-// tile's vector is staged, so the load overlaps the table build).
-__device__ __forceinline__ void first_rows(const LbJob& J, int s, int rb0, int nrb,
-                                           uint4 (&cur)[4]) {
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int rho = lane >> 2, gam = lane & 3;
-    const int rb = rb0 + wp;
-    const bool vec4 = (J.ldw & 3) == 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        cur[i] = rb < rb0 + nrb ? load_group(J, rb * kRowBlock + 8 * i + rho,
-                                             s * kSliceWords + 4 * gam, vec4)
-                                : make_uint4(0u, 0u, 0u, 0u);
+struct Tile {
+    int job, slice, rb0, nrb;
+};
+
+// Up to kMaxTiles tiles of this CTA's unit range, starting at unit u.
+__device__ __forceinline__ int collect_tiles(const Smem& sm, int n_jobs, int& j, int u, int u_end,
+                                             Tile (&t)[kMaxTiles]) {
+    int n = 0;
+    while (u < u_end && n < kMaxTiles) {
+        j = find_job(sm.jobs, j, n_jobs, u);
+        const LbJob& J = sm.jobs[j];
+        const int local = u - J.unit_begin;
+        const int s = local / J.n_rowblocks;
+        const int rb0 = local - s * J.n_rowblocks;
+        const int nrb = min(J.n_rowblocks - rb0, u_end - u);
+        t[n++] = Tile{j, s, rb0, nrb};
+        u += nrb;
+    }
+    return n;
 }
 
 __device__ void run_phase(const Smem& sm, const CallArgs& args) {
@@ -372,20 +459,26 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args) {
     const int u_end = unit_split(ph.n_units, cta + 1, G);
     int j = 0;
     while (u < u_end) {
-        j = find_job(sm.jobs, j, ph.n_jobs, u);
-        const LbJob J = fetch_job(sm.jobs, j, args);
-        const int local = u - J.unit_begin;
-        const int s = local / J.n_rowblocks;
-        const int rb0 = local - s * J.n_rowblocks;
-        const int nrb = min(J.n_rowblocks - rb0, u_end - u);
-        uint4 cur[4];
-        first_rows(J, s, rb0, nrb, cur);
-        stage_vector(J, s, rb0 == 0, sm);
-        build_lut(sm);
-        if (sm.lut == 0u) lookup_rowblocks<true>(J, s, rb0, nrb, sm, cur);
-        else lookup_rowblocks<false>(J, s, rb0, nrb, sm, cur);
-        u += nrb;
+        Tile t[kMaxTiles];
+        const int nt = collect_tiles(sm, ph.n_jobs, j, u, u_end, t);
+        {   // the first tile's rows start streaming while every vector is staged
+            const LbJob J = fetch_job(sm.jobs, t[0].job, args);
+            ring_prologue(J, t[0].slice, t[0].rb0, t[0].nrb, sm);
+        }
+        for (int k = 0; k < nt; ++k) {
+            const LbJob J = fetch_job(sm.jobs, t[k].job, args);
+            stage_vector(J, t[k].slice, t[k].rb0 == 0, sm, sm.vec + k * kVecPad);
+        }
         __syncthreads();
+        for (int k = 0; k < nt; ++k) {
+            const LbJob J = fetch_job(sm.jobs, t[k].job, args);
+            if (k > 0) ring_prologue(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
+            build_lut(sm, sm.vec + k * kVecPad);
+            if (sm.lut == 1024u) lookup_rowblocks<1024u>(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
+            else lookup_rowblocks<0u>(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
+            __syncthreads();
+            u += t[k].nrb;
+        }
     }
 }
 
@@ -408,6 +501,17 @@ __device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs) {
         const int rows = min(nrb * kRowBlock, budget);
         for (int i = threadIdx.x; i < rows; i += kDecodeThreads)
             prefetch_segment(J, s, rb0 * kRowBlock + i);
+        // the scales this tile will read: its slice of g or l, its rows of h
+        const int t = threadIdx.x - (kDecodeThreads - 32);          // last warp
+        if (t >= 0) {
+            const int c0 = s * kSliceElems, c1 = min(J.cols, c0 + kSliceElems);
+            if (t < 8 && c0 + 64 * t < c1) prefetch_l2(J.vscale + c0 + 64 * t);
+            if (J.oscale != nullptr) {
+                const int r0 = rb0 * kRowBlock, r1 = min(J.rows, (rb0 + nrb) * kRowBlock);
+                for (int r = r0 + 64 * (t - 8); t >= 8 && r < r1; r += 64 * 24)
+                    prefetch_l2(J.oscale + r);
+            }
+        }
         budget -= rows;
         u += nrb;
     }
@@ -481,6 +585,12 @@ cudaError_t decode_configure() {
     e = cudaFuncSetAttribute(stack_program_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDecodeSmem);
     if (e != cudaSuccess) return e;
+    for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
+                           reinterpret_cast<const void*>(stack_program_kernel)}) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+    }
     for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
                            reinterpret_cast<const void*>(stack_program_kernel)}) {
         int nb = 0;

@@ -17,14 +17,19 @@
 namespace lb {
 
 // ---------------------------------------------------------------- constants
-constexpr int kDecodeThreads = 256;          // 8 warps per CTA
+constexpr int kDecodeThreads = 512;          // 16 warps per CTA, one CTA per SM
 constexpr int kDecodeWarps = kDecodeThreads / 32;
-constexpr int kCtasPerSm = 2;                // two co-resident CTAs per SM
+constexpr int kCtasPerSm = 1;
 constexpr int kSliceElems = 512;             // columns covered by one lookup table
 constexpr int kSliceWords = kSliceElems / 32;
 constexpr int kRowBlock = 32;                // rows per warp work item (4 steps x 8 rows)
 constexpr int kLutBytes = 64 * 1024;         // 64 chunks x 256 entries x fp32
 constexpr int kVecPad = kSliceElems + kSliceElems / 32;   // staged slice, padded
+constexpr int kRingDepth = 3;                // rowblocks each warp has in flight
+constexpr int kRingSlots = kRingDepth + 1;
+constexpr int kRowBlockBytes = kRowBlock * kSliceWords * 4;   // 2 KB of signs
+constexpr int kRingSlotBytes = kRowBlockBytes + 128;          // + the lanes' row scales
+constexpr int kRingBytes = kDecodeWarps * kRingSlots * kRingSlotBytes;   // 130 KB
 constexpr int kMaxLinearJobs = 16;           // per phase in a single-linear call
 constexpr int kMaxPhaseJobs = 16;            // jobs of one phase (stack phases use <= 6)
 constexpr int kMaxDecodeM = 8;               // rows of x the decode path takes at once
@@ -75,8 +80,8 @@ struct LbPhase {
 #define LB_TAG_X ((const void*)1)
 #define LB_TAG_Y ((const void*)2)
 
-constexpr int kDecodeSmem = kLutBytes + 4 * kVecPad + 4 * 32 + 64 + (int)sizeof(LbPhase) +
-                            kMaxPhaseJobs * (int)sizeof(LbJob);
+constexpr int kDecodeSmem = kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64 +
+                            (int)sizeof(LbPhase) + kMaxPhaseJobs * (int)sizeof(LbJob);
 
 // Plan of a single linear call, passed by value as a kernel parameter.
 struct LinearPlan {
@@ -101,6 +106,25 @@ __device__ __forceinline__ void red_add_f32(float* p, float v) {
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" :: "l"(p));
+}
+// Exact-size L2 prefetch (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
+}
+// Read-only sign words through L1 (rows are L1-prefetched a few steps ahead).
+__device__ __forceinline__ uint4 ld_sign_v4(const uint32_t* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_sign_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
 }
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;

@@ -36,11 +36,14 @@ constexpr int kBlockK = 64;                       // fp16 elements per stage (12
 constexpr int kStages = 4;
 constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB
 constexpr int kBBytes = kTileN * kBlockK * 2;     // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kPrefillThreads = 384;              // 12 warps
-constexpr int kExpandWarp0 = 8;                   // warps 8..11 expand B
-constexpr int kExpandThreads = 128;
-constexpr int kEpiWarp0 = 4;                      // warps 4..7 drain TMEM
+constexpr int kGBytes = kBlockK * 2;              // g slice of the K block (stage 1)
+constexpr int kStageBytes = kABytes + kBBytes + 1024;   // keeps every tile 1024-aligned
+constexpr int kPrefillThreads = 512;              // 16 warps
+constexpr int kEpiWarp0 = 0;                      // warps 0..3 drain TMEM (lane quarter = warp)
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kExpandWarp0 = 8;                   // warps 8..15 expand B, one row per thread
+constexpr int kExpandThreads = 256;
 constexpr int kTmemCols = 512;                    // two 256-column accumulators
 constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
 constexpr int kPrefillSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
@@ -99,6 +102,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];"
         :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
@@ -185,49 +195,41 @@ __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb
     nt = r - nseg * nt_per_seg;
 }
 
-// Expand one 256 x 64 B tile (K-major, 128-byte swizzle) from packed signs.
-// Thread e owns rows e and e + 128.
-__device__ void expand_b(const PrefillGemm& g, uint32_t b_smem, int nseg, int nt, int kseg,
-                         int kb, int e) {
-    const int branch = g.stage == 1 ? nseg : kseg;
-    const uint32_t* P = g.P[branch];
-    const int k0 = kb * kBlockK;                     // k within the segment
+// Expand row n of one 256 x 64 B tile (K-major, 128-byte swizzle) from its 64
+// packed sign bits.  Element k is the scale with its sign bit flipped when the
+// bit is set: stage 1 scales per k (g slice staged in shared memory next to
+// the tile), stage 2 per row (hh = h[row] in both halves).  Bits of a byte are
+// spread to the top bit of each byte of a word by one multiply, and PRMT moves
+// two of them to bits 15 and 31 of the fp16 pair they sign.
+__device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int n, uint2 bits,
+                                           bool valid, bool per_k, uint32_t hh) {
+    const uint32_t rowoff = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int n = e + half * 128;                // row within the tile
-        const int row = nt * kTileN + n;             // row within the segment
-        uint2 bits = make_uint2(0u, 0u);
-        uint32_t nbase = 0u;                         // stage 2: h[row] in both halves
-        const bool valid = row < g.n_seg_rows;
-        if (valid) {
-            bits = __ldg(reinterpret_cast<const uint2*>(P + (size_t)row * g.ldw + k0 / 32));
-            if (g.stage == 2) {
-                const uint32_t hb = __half_as_ushort(__ldg(g.bscale[branch] + row));
-                nbase = hb | (hb << 16);
-            }
+    for (int c = 0; c < 8; ++c) {                    // 16-byte chunk: k = 8c .. 8c+7
+        const uint32_t byte = ((c < 4 ? bits.x : bits.y) >> (8 * (c & 3))) & 0xFFu;
+        const uint32_t rlo = ((byte & 0xFu) * 0x10204080u) & 0x80808080u;
+        const uint32_t rhi = ((byte >> 4) * 0x10204080u) & 0x80808080u;
+        const uint32_t m0 = prmt(rlo, 0u, 0x1404u), m1 = prmt(rlo, 0u, 0x3424u);
+        const uint32_t m2 = prmt(rhi, 0u, 0x1404u), m3 = prmt(rhi, 0u, 0x3424u);
+        uint4 base;
+        if (per_k) {
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(base.x), "=r"(base.y), "=r"(base.z), "=r"(base.w)
+                         : "r"(g_smem + 16u * (uint32_t)c));
+        } else {
+            base = make_uint4(hh, hh, hh, hh);
         }
-        const uint32_t rowoff = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {               // 16-byte chunk: k0 + 8c .. +7
-            const uint32_t byte = ((c < 4 ? bits.x : bits.y) >> (8 * (c & 3))) & 0xFFu;
-            uint4 base;
-            if (g.stage == 1) {
-                base = __ldg(reinterpret_cast<const uint4*>(g.bscale[branch] + k0 + 8 * c));
-            } else {
-                base = make_uint4(nbase, nbase, nbase, nbase);
-            }
-            uint32_t o[4];
-            const uint32_t bw[4] = {base.x, base.y, base.z, base.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const uint32_t m = ((byte >> (2 * p)) & 3u) * 0x40008000u;
-                o[p] = valid ? (bw[p] ^ (m & 0x80008000u)) : 0u;
-            }
-            const uint32_t addr = b_smem + rowoff + (uint32_t)((c ^ (n & 7)) * 16);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                         :: "r"(addr), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
-        }
+        const uint32_t o0 = valid ? base.x ^ m0 : 0u, o1 = valid ? base.y ^ m1 : 0u;
+        const uint32_t o2 = valid ? base.z ^ m2 : 0u, o3 = valid ? base.w ^ m3 : 0u;
+        const uint32_t addr = b_smem + rowoff + (uint32_t)((c ^ (n & 7)) * 16);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(addr), "r"(o0), "r"(o1), "r"(o2), "r"(o3) : "memory");
     }
+}
+
+__device__ __forceinline__ uint2 load_bits(const PrefillGemm& g, int branch, int row, int kb) {
+    if (row >= g.n_seg_rows) return make_uint2(0u, 0u);
+    return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + (size_t)row * g.ldw + kb * 2));
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -257,7 +259,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      :: "r"(smem_u32(&ctl->tmem_base)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -267,8 +269,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp == 0) {
-        // ---------------- TMA producer for A
+    if (warp == kTmaWarp) {
+        // ---------------- TMA producer for A (and the g slice of stage 1)
         if (lane == 0) {
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
@@ -279,14 +281,21 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                     const uint32_t par = ((it / kStages) & 1) ^ 1;
                     if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) break;
                     const uint32_t fb = smem_u32(&ctl->full_a[s]);
-                    mbar_expect_tx(fb, kABytes);
                     const int kseg = kb / kb_per_seg;
-                    const int kcol = kseg * g.k_seg_len + (kb - kseg * kb_per_seg) * kBlockK;
+                    const int kloc = (kb - kseg * kb_per_seg) * kBlockK;
+                    const int kcol = kseg * g.k_seg_len + kloc;
+                    if (g.stage == 1) {
+                        mbar_expect_tx(fb, kABytes + kGBytes);
+                        bulk_load(base + s * kStageBytes + kABytes + kBBytes,
+                                  g.bscale[nseg] + kloc, kGBytes, fb);
+                    } else {
+                        mbar_expect_tx(fb, kABytes);
+                    }
                     tma_load_2d(base + s * kStageBytes, &amap, fb, kcol, mb * kTileM);
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer
         if (lane == 0) {
             int it = 0, tl = 0;
@@ -313,7 +322,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                 mma_commit(smem_u32(&ctl->acc_full[buf]));
             }
         }
-    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    } else if (warp < kEpiWarp0 + 4) {
         // ---------------- epilogue: TMEM -> registers -> global
         const int q = warp - kEpiWarp0;              // TMEM lane quarter
         int tl = 0;
@@ -374,20 +383,43 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
         }
     } else if (warp >= kExpandWarp0) {
-        // ---------------- B producers: packed signs -> fp16 tile
+        // ---------------- B producers: packed signs -> fp16 tile, one row per thread
         const int e = threadIdx.x - kExpandWarp0 * 32;
         int it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             int mb, nseg, nt;
             tile_coords(g, t, mb, nseg, nt);
+            const int row = nt * kTileN + e;
+            const bool valid = row < g.n_seg_rows;
+            uint32_t hh[2] = {0u, 0u};
+            if (g.stage == 2 && valid) {
+                for (int b = 0; b < g.n_kseg; ++b) {
+                    const uint32_t hb = __half_as_ushort(__ldg(g.bscale[b] + row));
+                    hh[b] = hb | (hb << 16);
+                }
+            }
+            const int br0 = g.stage == 1 ? nseg : 0;
+            uint2 nxt = load_bits(g, br0, row, 0);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
                 const int s = it % kStages;
-                const uint32_t par = ((it / kStages) & 1) ^ 1;
-                if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) { ok = false; break; }
                 const int kseg = kb / kb_per_seg;
-                expand_b(g, base + s * kStageBytes + kABytes, nseg, nt, kseg,
-                         kb - kseg * kb_per_seg, e);
+                const int klocb = kb - kseg * kb_per_seg;
+                const int branch = g.stage == 1 ? nseg : kseg;
+                const uint2 cur = nxt;
+                if (kb + 1 < n_kb) {
+                    const int ks1 = (kb + 1) / kb_per_seg;
+                    nxt = load_bits(g, g.stage == 1 ? nseg : ks1, row, kb + 1 - ks1 * kb_per_seg);
+                }
+                if (!wait_bar(ctl, &ctl->empty[s], ((it / kStages) & 1) ^ 1, g.err)) { ok = false; break; }
+                if (g.stage == 1 && !wait_bar(ctl, &ctl->full_a[s], (it / kStages) & 1, g.err)) {
+                    ok = false;
+                    break;
+                }
+                (void)klocb;
+                const uint32_t sb = base + s * kStageBytes;
+                expand_row(sb + kABytes, sb + kABytes + kBBytes, e, cur, valid, g.stage == 1,
+                           hh[branch & 1]);
                 fence_async_smem();                  // make the stores visible to the tensor core
                 mbar_arrive(smem_u32(&ctl->full_b[s]));
             }
@@ -402,7 +434,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         while (clock64() - t0 < 2000000LL) { }
     }
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      :: "r"(tmem), "r"(kTmemCols) : "memory");

@@ -85,7 +85,7 @@ lb_status lb_pack_signs(const float *latent, int64_t rows, int64_t cols, int64_t
 typedef struct {
     const uint32_t *Vp;   /* [r][ld_v] signs of V_b packed along in          */
     const uint32_t *Up;   /* [out][ld_u] signs of U_b packed along r         */
-    const uint16_t *h;    /* [out] FP16 row scale (IEEE binary16 bits)       */
+    const uint16_t *h;    /* [out] FP16 row scale (IEEE binary16 bits), 4-byte aligned */
     const uint16_t *g;    /* [in]  FP16 column scale                         */
     const uint16_t *l;    /* [r]   FP16 latent scale                         */
 } lb_branch;
@@ -104,8 +104,10 @@ typedef struct {
  * tensor-core kernels.  Both accumulate in fp32.
  * Errors: LB_ERR_INVALID_ARG (null pointer, M/in/out/r <= 0, n_branches not 1
  * or 2, bad dtype), LB_ERR_ALIGNMENT (x, y, workspace or a packed pointer not
- * 16-byte aligned), LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED (no sm_100 device),
- * LB_ERR_CUDA.
+ * 16-byte aligned, h not 4-byte aligned, g or l not 2-byte aligned),
+ * LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED (no sm_100 device), LB_ERR_CUDA.
+ * (The tensor-core path also reads g in 16-byte vectors; a g that is not
+ * 16-byte aligned keeps the call on the lookup-table kernels.)
  */
 lb_status lb_linear_forward(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
                             int64_t out, int64_t r, const lb_branch *br, int n_branches,
