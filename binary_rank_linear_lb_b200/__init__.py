@@ -40,7 +40,8 @@ class LbError(RuntimeError):
 
 class lb_branch(ctypes.Structure):
     _fields_ = [("Vp", ctypes.c_void_p), ("Up", ctypes.c_void_p), ("h", ctypes.c_void_p),
-                ("g", ctypes.c_void_p), ("l", ctypes.c_void_p)]
+                ("g", ctypes.c_void_p), ("l", ctypes.c_void_p), ("ld_v", ctypes.c_int64),
+                ("ld_u", ctypes.c_int64)]
 
 
 class lb_stack_desc(ctypes.Structure):
@@ -149,7 +150,8 @@ class Branch:
         self.Vp, self.Up, self.h, self.g, self.l = Vp, Up, h, g, l
 
     def c_struct(self) -> lb_branch:
-        return lb_branch(_ptr(self.Vp), _ptr(self.Up), _ptr(self.h), _ptr(self.g), _ptr(self.l))
+        return lb_branch(_ptr(self.Vp), _ptr(self.Up), _ptr(self.h), _ptr(self.g), _ptr(self.l),
+                         self.Vp.shape[1], self.Up.shape[1])
 
     @property
     def nbytes(self) -> int:

@@ -56,14 +56,21 @@ int vec_kind_for(lb_dtype t) {
     }
 }
 
-// Fill the size fields of a job whose matrix has `rows` packed rows of `cols` signs.
-void set_job_shape(LbJob& J, int64_t rows, int64_t cols) {
+// Fill the size fields of a job whose matrix has `rows` packed rows of `cols`
+// signs with a pitch of `ld` words (0: unpadded), and its TMA descriptor when
+// the pitch allows one (16-byte rows).
+void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld) {
     J.rows = (int)rows;
     J.cols = (int)cols;
-    J.ldw = (int)cdiv(cols, 32);
+    J.ldw = (int)(ld ? ld : cdiv(cols, 32));
     J.n_slices = (int)cdiv(cols, kSliceElems);
     J.n_rowblocks = (int)cdiv(rows, kRowBlock);
+    J.use_tma = 0;
+    if ((J.ldw & 3) == 0 && (reinterpret_cast<uintptr_t>(J.P) & 15) == 0)
+        J.use_tma = make_sign_tmap(&J.tmap, J.P, J.rows, J.ldw) ? 1 : 0;
 }
+
+bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <= (1 << 26)); }
 
 // Append `J` to phase `ph`, assigning its unit range.
 void add_job(LbPhase& ph, std::vector<LbJob>& jobs, LbJob J) {
@@ -74,7 +81,7 @@ void add_job(LbPhase& ph, std::vector<LbJob>& jobs, LbJob J) {
 }
 
 bool branch_ok(const lb_branch& b) {
-    return b.Vp && b.Up && b.h && b.g && b.l;
+    return b.Vp && b.Up && b.h && b.g && b.l && b.ld_v >= 0 && b.ld_u >= 0;
 }
 bool branch_aligned(const lb_branch& b) {
     return aligned(b.Vp, 16) && aligned(b.Up, 16) && aligned(b.h, 4) && aligned(b.g, 2) &&
@@ -100,6 +107,18 @@ struct StackLayout {
     size_t total;
 };
 
+// in / out features of projection p.
+void proj_shape(const lb_stack_desc* d, int p, int64_t& in, int64_t& out) {
+    const int64_t kv = (int64_t)d->n_kv_heads * d->head_dim;
+    switch (p) {
+        case LB_Q: in = d->hidden; out = d->hidden; break;
+        case LB_K: case LB_V: in = d->hidden; out = kv; break;
+        case LB_O: in = d->hidden; out = d->hidden; break;
+        case LB_GATE: case LB_UP: in = d->hidden; out = d->inter; break;
+        default: in = d->inter; out = d->hidden; break;
+    }
+}
+
 bool stack_desc_ok(const lb_stack_desc* d) {
     if (!d || !d->lin || !d->ranks) return false;
     if (d->n_layers <= 0 || d->hidden <= 0 || d->inter <= 0) return false;
@@ -120,22 +139,15 @@ bool stack_desc_ok(const lb_stack_desc* d) {
             if (!used) continue;
             if (d->ranks[L * LB_N_PROJ + p] <= 0 || d->ranks[L * LB_N_PROJ + p] > (1 << 24))
                 return false;
-            for (int b = 0; b < d->n_branches; ++b)
-                if (!branch_ok(d->lin[(L * LB_N_PROJ + p) * d->n_branches + b])) return false;
+            int64_t in, out;
+            proj_shape(d, p, in, out);
+            const int64_t r = d->ranks[L * LB_N_PROJ + p];
+            for (int b = 0; b < d->n_branches; ++b) {
+                const lb_branch& B = d->lin[(L * LB_N_PROJ + p) * d->n_branches + b];
+                if (!branch_ok(B) || !ld_ok(B.ld_v, in) || !ld_ok(B.ld_u, r)) return false;
+            }
         }
     return true;
-}
-
-// in / out features of projection p.
-void proj_shape(const lb_stack_desc* d, int p, int64_t& in, int64_t& out) {
-    const int64_t kv = (int64_t)d->n_kv_heads * d->head_dim;
-    switch (p) {
-        case LB_Q: in = d->hidden; out = d->hidden; break;
-        case LB_K: case LB_V: in = d->hidden; out = kv; break;
-        case LB_O: in = d->hidden; out = d->hidden; break;
-        case LB_GATE: case LB_UP: in = d->hidden; out = d->inter; break;
-        default: in = d->inter; out = d->hidden; break;
-    }
 }
 
 bool proj_used(const lb_stack_desc* d, int p) {
@@ -245,7 +257,7 @@ void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
                     LbJob J = {};
                     if (ps.first) {
                         J.P = br(l, p, b).Vp;
-                        set_job_shape(J, r, in);
+                        set_job_shape(J, r, in, br(l, p, b).ld_v);
                         J.vscale = reinterpret_cast<const __half*>(br(l, p, b).g);
                         J.out = tptr(l, p, b);
                         if (p == LB_O) {
@@ -269,7 +281,7 @@ void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
                         if (first_job && norm) J.acc_sumsq = norm;
                     } else {
                         J.P = br(l, p, b).Up;
-                        set_job_shape(J, out, r);
+                        set_job_shape(J, out, r, br(l, p, b).ld_u);
                         J.kind = VK_T;
                         J.src = tptr(l, p, b);
                         J.vscale = reinterpret_cast<const __half*>(br(l, p, b).l);
@@ -374,7 +386,8 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
     if (n_branches < 1 || n_branches > 2) return LB_ERR_INVALID_ARG;
     if (x_dtype != LB_F16 && x_dtype != LB_BF16 && x_dtype != LB_F32) return LB_ERR_INVALID_ARG;
     for (int b = 0; b < n_branches; ++b)
-        if (!branch_ok(br[b])) return LB_ERR_INVALID_ARG;
+        if (!branch_ok(br[b]) || !ld_ok(br[b].ld_v, in) || !ld_ok(br[b].ld_u, r))
+            return LB_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(workspace, 16)) return LB_ERR_ALIGNMENT;
     for (int b = 0; b < n_branches; ++b)
         if (!branch_aligned(br[b])) return LB_ERR_ALIGNMENT;
@@ -384,9 +397,12 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (use_prefill(M, in, out, r)) {
-        bool scales16 = true;   // the tensor-core path reads g in 16-byte vectors
-        for (int b = 0; b < n_branches; ++b) scales16 = scales16 && aligned(br[b].g, 16);
-        if (scales16)
+        // the tensor-core path reads g in 16-byte vectors and sign words in pairs
+        bool ok = true;
+        for (int b = 0; b < n_branches; ++b)
+            ok = ok && aligned(br[b].g, 16) && ((br[b].ld_v ? br[b].ld_v : cdiv(in, 32)) & 1) == 0 &&
+                 ((br[b].ld_u ? br[b].ld_u : cdiv(r, 32)) & 1) == 0;
+        if (ok)
             return launch_prefill(x, vec_kind_for(x_dtype), M, in, out, r, br, n_branches, y,
                                   workspace, s) == cudaSuccess
                        ? LB_OK
@@ -407,7 +423,7 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
             for (int b = 0; b < n_branches; ++b) {
                 LbJob J = {};
                 J.P = br[b].Vp;
-                set_job_shape(J, r, in);
+                set_job_shape(J, r, in, br[b].ld_v);
                 J.kind = vec_kind_for(x_dtype);
                 J.src = static_cast<const char*>(x) + (size_t)(m0 + m) * (size_t)in * xsz;
                 J.vscale = reinterpret_cast<const __half*>(br[b].g);
@@ -422,7 +438,7 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
             for (int b = 0; b < n_branches; ++b) {
                 LbJob J = {};
                 J.P = br[b].Up;
-                set_job_shape(J, out, r);
+                set_job_shape(J, out, r, br[b].ld_u);
                 J.kind = VK_T;
                 J.src = t + ((size_t)m * n_branches + b) * (size_t)r;
                 J.vscale = reinterpret_cast<const __half*>(br[b].l);

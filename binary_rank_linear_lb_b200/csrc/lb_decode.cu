@@ -50,6 +50,7 @@ struct Smem {
     int* flag;        // one int
     LbPhase* phase;   // the current phase, copied from the plan
     LbJob* jobs;      // its jobs (at most kMaxPhaseJobs), copied from the plan
+    uint32_t bars;    // per-warp ring mbarriers (kRingSlots per warp), shared address
 };
 
 __device__ __forceinline__ Smem smem_layout() {
@@ -61,7 +62,8 @@ __device__ __forceinline__ Smem smem_layout() {
     s.red = s.vec + 4 * kVecPad;
     s.flag = reinterpret_cast<int*>(s.red + 32);
     s.phase = reinterpret_cast<LbPhase*>(dsmem + kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64);
-    s.jobs = reinterpret_cast<LbJob*>(s.phase + 1);
+    s.jobs = reinterpret_cast<LbJob*>(reinterpret_cast<unsigned char*>(s.phase) + 64);
+    s.bars = (uint32_t)__cvta_generic_to_shared(s.jobs + kMaxPhaseJobs);
     return s;
 }
 
@@ -325,6 +327,46 @@ __device__ __forceinline__ void issue_rowblock(const LbJob& J, int s, int rb, ui
     }
 }
 
+// ---- TMA-fed ring (rows with a 16-byte pitch) -----------------------------
+// Lane 0 of a warp loads a whole rowblock (32 rows x 16 words, 2 KB) with one
+// 2-D tensor copy into the warp's ring slot; the slot's mbarrier counts the
+// bytes.  The box lands row-major, 64 bytes per row, which is the same layout
+// the cp.async path writes (minus the half swap of rows 4..7 of each step).
+// ring_it counts the rowblocks this warp has consumed so far in this launch;
+// slot = it % kRingSlots, mbarrier phase parity = (it / kRingSlots) & 1.
+__device__ __forceinline__ uint32_t ring_bar(const Smem& sm, uint32_t it) {
+    return sm.bars + (uint32_t)(((threadIdx.x >> 5) * kRingSlots + (int)(it % kRingSlots)) * 8);
+}
+__device__ __forceinline__ uint32_t ring_slot_base(const Smem& sm, uint32_t it) {
+    return sm.ring + (uint32_t)((((threadIdx.x >> 5) * kRingSlots) + (int)(it % kRingSlots)) *
+                                kRingSlotBytes);
+}
+// Issue (lane 0) the TMA of rowblock rb of slice s as ring entry `it`.  The
+// slot was last read by this warp: every lane has passed __syncwarp, and the
+// proxy fence orders those reads before the tensor copy's writes.
+__device__ __forceinline__ void tma_issue(const LbJob* Jg, int s, int rb, const Smem& sm,
+                                          uint32_t it) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        fence_proxy_async_smem();
+        const uint32_t bar = ring_bar(sm, it);
+        mbar_expect_tx(bar, (uint32_t)kRowBlockBytes);
+        tma_load_2d(ring_slot_base(sm, it), &Jg->tmap, bar, s * kSliceWords, rb * kRowBlock);
+    }
+}
+// Bounded wait for ring entry `it`; on time-out records LB_ERR_TIMEOUT.
+__device__ __forceinline__ void tma_wait(const Smem& sm, uint32_t it, int* err) {
+    const uint32_t bar = ring_bar(sm, it), par = (it / kRingSlots) & 1u;
+    if (mbar_try_wait(bar, par)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, par)) {
+        if (clock64() - t0 > kSpinLimitCycles) {
+            atomicExch(err, (int)LB_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
 // Number of rowblocks warp wp takes in a tile of nrb rowblocks.
 __device__ __forceinline__ int warp_rowblocks(int nrb) {
     const int wp = threadIdx.x >> 5;
@@ -333,11 +375,16 @@ __device__ __forceinline__ int warp_rowblocks(int nrb) {
 
 // First kRingDepth rowblocks of this warp's share of a tile (issued before the
 // tile's vector is staged, so the copies overlap staging and table build).
-// Always commits exactly kRingDepth groups.
-__device__ __forceinline__ void ring_prologue(const LbJob& J, int s, int rb0, int nrb,
-                                              const Smem& sm) {
+// The cp.async path always commits exactly kRingDepth groups.
+__device__ __forceinline__ void ring_prologue(const LbJob& J, const LbJob* Jg, int s, int rb0,
+                                              int nrb, const Smem& sm, uint32_t ring_it) {
     const int wp = threadIdx.x >> 5;
     const int nit = warp_rowblocks(nrb);
+    if (J.use_tma) {
+        for (int d = 0; d < kRingDepth && d < nit; ++d)
+            tma_issue(Jg, s, rb0 + wp + d * kDecodeWarps, sm, ring_it + d);
+        return;
+    }
 #pragma unroll
     for (int d = 0; d < kRingDepth; ++d) {
         if (d < nit) issue_rowblock(J, s, rb0 + wp + d * kDecodeWarps, ring_slot(sm, d));
@@ -349,9 +396,10 @@ __device__ __forceinline__ void ring_prologue(const LbJob& J, int s, int rb0, in
 // rowblocks stream through the warp's ring kRingDepth ahead of use.  kBase is
 // the table's shared-window address when it is the usual 1024 (then it folds
 // into the load's immediate offset), else 0 and tbase is added at run time.
-template <uint32_t kBase>
-__device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0, int nrb,
-                                                 const Smem& sm) {
+template <uint32_t kBase, bool kTma>
+__device__ __forceinline__ void lookup_rowblocks(const LbJob& J, const LbJob* Jg, int s, int rb0,
+                                                 int nrb, const Smem& sm, uint32_t& ring_it,
+                                                 int* err) {
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int rho = lane >> 2, gam = lane & 3;
     const uint32_t swap = (uint32_t)(rho >> 2);
@@ -369,12 +417,23 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
     const bool has_h = J.oscale != nullptr;
     for (int n = 0; n < nit; ++n) {
         const int rb = rb0 + wp + n * kDecodeWarps;
-        if (n + kRingDepth < nit)
-            issue_rowblock(J, s, rb + kRingDepth * kDecodeWarps,
-                           ring_slot(sm, (n + kRingDepth) % kRingSlots));
-        cp_async_commit();
-        cp_async_wait<kRingDepth>();                     // rowblock n has landed
-        const uint32_t src = ring_slot(sm, n % kRingSlots);
+        uint32_t src;
+        float hs_early = 1.0f;
+        const int orow_e = rb * kRowBlock + 8 * gam + rho;
+        if (kTma) {
+            if (n + kRingDepth < nit)
+                tma_issue(Jg, s, rb + kRingDepth * kDecodeWarps, sm, ring_it + n + kRingDepth);
+            if (has_h && orow_e < J.rows) hs_early = __half2float(__ldg(J.oscale + orow_e));
+            tma_wait(sm, ring_it + n, err);
+            src = ring_slot_base(sm, ring_it + n) + (uint32_t)lane * 16u;
+        } else {
+            if (n + kRingDepth < nit)
+                issue_rowblock(J, s, rb + kRingDepth * kDecodeWarps,
+                               ring_slot(sm, (n + kRingDepth) % kRingSlots));
+            cp_async_commit();
+            cp_async_wait<kRingDepth>();                 // rowblock n has landed
+            src = ring_slot(sm, n % kRingSlots);
+        }
         float acc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -382,6 +441,10 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
                          : "r"(src + (uint32_t)i * 512u));
+            if (kTma && swap) {                          // rows 4..7 read the halves swapped
+                const uint32_t t0 = w4[0], t1 = w4[1];
+                w4[0] = w4[2]; w4[1] = w4[3]; w4[2] = t0; w4[3] = t1;
+            }
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -395,9 +458,9 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
             }
             acc[i] = a0 + a1;
         }
-        const int orow = rb * kRowBlock + 8 * gam + rho;   // output row of this lane
-        float hs = 1.0f;
-        if (has_h) {
+        const int orow = orow_e;                           // output row of this lane
+        float hs = hs_early;
+        if (!kTma && has_h) {
             uint32_t hw;
             asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hw) : "r"(ring_hslot(src)));
             const unsigned short hb = (unsigned short)((orow & 1) ? (hw >> 16) : (hw & 0xFFFFu));
@@ -418,7 +481,8 @@ __device__ __forceinline__ void lookup_rowblocks(const LbJob& J, int s, int rb0,
         const float tot = keep1 + __shfl_xor_sync(0xffffffffu, send1, 1);
         if (orow < J.rows) red_add_f32(J.out + orow, tot * hs);
     }
-    cp_async_wait<0>();
+    if (kTma) ring_it += (uint32_t)nit;
+    else cp_async_wait<0>();
 }
 
 __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int u) {
@@ -447,7 +511,8 @@ __device__ __forceinline__ int collect_tiles(const Smem& sm, int n_jobs, int& j,
     return n;
 }
 
-__device__ void run_phase(const Smem& sm, const CallArgs& args) {
+__device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
+                          uint32_t& ring_it, int* err) {
     const int G = gridDim.x, cta = blockIdx.x;
     const LbPhase ph = *sm.phase;
     float* zp = resolve(ph.zero_ptr, args);
@@ -463,7 +528,8 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args) {
         const int nt = collect_tiles(sm, ph.n_jobs, j, u, u_end, t);
         {   // the first tile's rows start streaming while every vector is staged
             const LbJob J = fetch_job(sm.jobs, t[0].job, args);
-            ring_prologue(J, t[0].slice, t[0].rb0, t[0].nrb, sm);
+            ring_prologue(J, jobs_g + ph.job_begin + t[0].job, t[0].slice, t[0].rb0, t[0].nrb, sm,
+                          ring_it);
         }
         for (int k = 0; k < nt; ++k) {
             const LbJob J = fetch_job(sm.jobs, t[k].job, args);
@@ -472,10 +538,17 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args) {
         __syncthreads();
         for (int k = 0; k < nt; ++k) {
             const LbJob J = fetch_job(sm.jobs, t[k].job, args);
-            if (k > 0) ring_prologue(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
+            const LbJob* Jg = jobs_g + ph.job_begin + t[k].job;
+            if (k > 0) ring_prologue(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it);
             build_lut(sm, sm.vec + k * kVecPad);
-            if (sm.lut == 1024u) lookup_rowblocks<1024u>(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
-            else lookup_rowblocks<0u>(J, t[k].slice, t[k].rb0, t[k].nrb, sm);
+            const bool b1024 = sm.lut == 1024u;
+            if (J.use_tma) {
+                if (b1024) lookup_rowblocks<1024u, true>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+                else lookup_rowblocks<0u, true>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+            } else {
+                if (b1024) lookup_rowblocks<1024u, false>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+                else lookup_rowblocks<0u, false>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+            }
             __syncthreads();
             u += t[k].nrb;
         }
@@ -522,11 +595,14 @@ __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jo
     const Smem sm = smem_layout();
     const unsigned G = gridDim.x;
     if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) return;   // sticky after a timeout
+    if (threadIdx.x < kDecodeWarps * kRingSlots) mbar_init(sm.bars + 8u * threadIdx.x, 1u);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     cache_phase(phases, 0, jobs, sm);
     prefetch_phase(phases[0], jobs);
     __syncthreads();
+    uint32_t ring_it = 0;
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args);
+        run_phase(sm, args, jobs, ring_it, &hdr->error);
         if (p + 1 < n_phases) {
             // Announce completion, then use the wait: copy the next phase's
             // plan into shared memory and prefetch its sign rows to L2.
@@ -577,6 +653,33 @@ cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
 }
 
 }  // namespace
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw) {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    if (!fn || rows <= 0 || ldw <= 0 || (ldw & 3) != 0) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)ldw, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldw * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)kSliceWords, (cuuint32_t)kRowBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(P), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
 
 cudaError_t decode_configure() {
     cudaError_t e = cudaFuncSetAttribute(linear_program_kernel,

@@ -8,6 +8,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -28,7 +29,7 @@ constexpr int kVecPad = kSliceElems + kSliceElems / 32;   // staged slice, padde
 constexpr int kRingDepth = 3;                // rowblocks each warp has in flight
 constexpr int kRingSlots = kRingDepth + 1;
 constexpr int kRowBlockBytes = kRowBlock * kSliceWords * 4;   // 2 KB of signs
-constexpr int kRingSlotBytes = kRowBlockBytes + 128;          // + the lanes' row scales
+constexpr int kRingSlotBytes = kRowBlockBytes + 128;          // + the lanes' row scales (128-aligned)
 constexpr int kRingBytes = kDecodeWarps * kRingSlots * kRingSlotBytes;   // 130 KB
 constexpr int kMaxLinearJobs = 16;           // per phase in a single-linear call
 constexpr int kMaxPhaseJobs = 16;            // jobs of one phase (stack phases use <= 6)
@@ -54,8 +55,9 @@ enum VecKind : int {
     VK_SILU_MUL = 5,   // v = g[j] * silu(src[j]) * src2[j]
 };
 
-struct LbJob {
-    const uint32_t* P;        // packed rows [rows][ldw]
+struct alignas(64) LbJob {
+    CUtensorMap tmap;         // 2-D TMA descriptor of P (32-row x 16-word boxes), if use_tma
+    const uint32_t* P;        // packed rows [rows][ldw] (ldw = row pitch in words)
     const void* src;          // vector source
     const float* src2;        // second source (VK_SILU_MUL)
     const __half* vscale;     // g (first contraction) or l (second)
@@ -66,7 +68,7 @@ struct LbJob {
     float* resid_init;        // owner of a slice writes float(src) of the slice here
     int rows, cols, ldw, kind;
     int n_slices, n_rowblocks, unit_begin, norm_n;
-    int gqa_ghd, gqa_hd, pad0, pad1;
+    int gqa_ghd, gqa_hd, use_tma, pad1;
 };
 
 struct LbPhase {
@@ -80,8 +82,9 @@ struct LbPhase {
 #define LB_TAG_X ((const void*)1)
 #define LB_TAG_Y ((const void*)2)
 
-constexpr int kDecodeSmem = kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64 +
-                            (int)sizeof(LbPhase) + kMaxPhaseJobs * (int)sizeof(LbJob);
+constexpr int kDecodeSmem = kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64 + 64 +
+                            kMaxPhaseJobs * (int)sizeof(LbJob) + 8 * kDecodeWarps * kRingSlots;
+static_assert(kDecodeSmem <= 227 * 1024, "decode kernel shared memory over the per-CTA limit");
 
 // Plan of a single linear call, passed by value as a kernel parameter.
 struct LinearPlan {
@@ -145,10 +148,42 @@ __device__ __forceinline__ float lds_f32(uint32_t saddr) {
     return v;
 }
 
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------ host helpers
 int device_sm_count();               // SMs of the current device (cached per device)
 bool device_is_sm100();
 cudaError_t decode_configure();      // one-time kernel attribute setup per device
+// 2-D TMA descriptor of a packed sign matrix (rows x ldw words, 16-byte pitch).
+bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw);
 
 // Decode phase program launches (lb_decode.cu).
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,

@@ -52,26 +52,6 @@ constexpr int kPrefillSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barr
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
 struct Ctl {                 // shared control block
     uint64_t full_a[kStages], full_b[kStages], empty[kStages];
     uint64_t acc_full[2], acc_empty[2];
@@ -94,14 +74,6 @@ __device__ __forceinline__ bool wait_bar(Ctl* c, uint64_t* bar, uint32_t parity,
             return false;
         }
     }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -173,7 +145,7 @@ struct PrefillGemm {
     int M, n_seg_rows, n_nseg, n_kseg, k_seg_len;   // N = n_nseg * n_seg_rows, K = n_kseg * k_seg_len
     int stage;                                       // 1 or 2
     const uint32_t* P[2];                            // packed signs per branch
-    int ldw;                                         // words per packed row
+    int ldw[2];                                      // words per packed row, per branch
     const __half* bscale[2];                         // stage 1: g_b (per k); stage 2: h_b (per n)
     const __half* lscale[2];                         // stage 1: l_b (per output column)
     const float* row_sa;                             // [M] 2^a_m (stage 1 divides it out)
@@ -229,7 +201,7 @@ __device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int
 
 __device__ __forceinline__ uint2 load_bits(const PrefillGemm& g, int branch, int row, int kb) {
     if (row >= g.n_seg_rows) return make_uint2(0u, 0u);
-    return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + (size_t)row * g.ldw + kb * 2));
+    return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + (size_t)row * g.ldw[branch] + kb * 2));
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -609,10 +581,10 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         for (int b = 0; b < 2; ++b) {
             const lb_branch& B = br[b < nb ? b : 0];
             p.P[b] = B.Vp;
+            p.ldw[b] = (int)(B.ld_v ? B.ld_v : (in + 31) / 32);
             p.bscale[b] = reinterpret_cast<const __half*>(B.g);
             p.lscale[b] = reinterpret_cast<const __half*>(B.l);
         }
-        p.ldw = (int)((in + 31) / 32);
         p.row_sa = sa; p.row_sc = sc; p.T = T; p.y = nullptr; p.err = &hdr->error;
         prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -627,10 +599,10 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         for (int b = 0; b < 2; ++b) {
             const lb_branch& B = br[b < nb ? b : 0];
             p.P[b] = B.Up;
+            p.ldw[b] = (int)(B.ld_u ? B.ld_u : (r + 31) / 32);
             p.bscale[b] = reinterpret_cast<const __half*>(B.h);
             p.lscale[b] = nullptr;
         }
-        p.ldw = (int)((r + 31) / 32);
         p.row_sa = sa; p.row_sc = sc; p.T = nullptr; p.y = y; p.err = &hdr->error;
         prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

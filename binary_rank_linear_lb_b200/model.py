@@ -1,7 +1,9 @@
 """Device-resident factorised linears and decoder stacks built from seeded inputs.
 
 Each branch is generated from its own seeds (``synth``) and binarised on the GPU
-with ``lb_pack_signs``; the fp32 latents are dropped right after packing.
+with ``lb_pack_signs``; the fp32 latents are dropped right after packing.  Rows
+are packed with a 16-byte pitch (``ld_words`` a multiple of 4, zero padding),
+which lets the decode kernels stream them with TMA.
 
 ``signs="bits"`` instead draws the packed words directly from a uniform bit
 source.  The signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so the
@@ -19,28 +21,35 @@ from . import Branch, Stack, pack_signs, synth
 from .configs import Model, proj_shape
 
 
+def padded_words(k: int, pad: bool = True) -> int:
+    """Words per packed row of k signs: ceil(k/32), rounded up to a multiple of 4 if pad."""
+    w = (k + 31) // 32
+    return (w + 3) // 4 * 4 if pad else w
+
+
 def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int, branch: int,
-                 device="cuda", signs: str = "latent") -> Branch:
+                 device="cuda", signs: str = "latent", pad: bool = True) -> Branch:
     s = lambda k: synth.tensor_seed(base, layer, proj, branch, k)
     h = synth.scale(out_f, s(synth.KIND_H), device)
     g = synth.scale(in_f, s(synth.KIND_G), device)
     l = synth.scale(r, s(synth.KIND_L), device)
     if signs == "latent":
         V = synth.latent(in_f, r, s(synth.KIND_V), device)
-        Vp = pack_signs(V, axis=0)
+        Vp = pack_signs(V, axis=0, ld_words=padded_words(in_f, pad))
         del V
         U = synth.latent(out_f, r, s(synth.KIND_U), device)
-        Up = pack_signs(U, axis=1)
+        Up = pack_signs(U, axis=1, ld_words=padded_words(r, pad))
         del U
     elif signs == "bits":
         def words(n_rows, k, seed):
             gen = torch.Generator(device=device)
             gen.manual_seed(seed)
-            ldw = (k + 31) // 32
-            w = torch.randint(-2 ** 31, 2 ** 31, (n_rows, ldw), generator=gen, device=device,
-                              dtype=torch.int64).to(torch.int32)
+            nw = (k + 31) // 32
+            w = torch.zeros((n_rows, padded_words(k, pad)), dtype=torch.int32, device=device)
+            w[:, :nw] = torch.randint(-2 ** 31, 2 ** 31, (n_rows, nw), generator=gen,
+                                      device=device, dtype=torch.int64).to(torch.int32)
             if k % 32:
-                w[:, -1] &= (1 << (k % 32)) - 1
+                w[:, nw - 1] &= (1 << (k % 32)) - 1
             return w
         Vp = words(r, in_f, s(synth.KIND_V))
         Up = words(out_f, r, s(synth.KIND_U))
@@ -50,8 +59,9 @@ def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int
 
 
 def build_linear(in_f: int, out_f: int, r: int, base: int = 0, layer: int = 0, proj: int = 0,
-                 n_branches: int = 2, device="cuda", signs: str = "latent") -> List[Branch]:
-    return [build_branch(in_f, out_f, r, base, layer, proj, b, device, signs)
+                 n_branches: int = 2, device="cuda", signs: str = "latent",
+                 pad: bool = True) -> List[Branch]:
+    return [build_branch(in_f, out_f, r, base, layer, proj, b, device, signs, pad)
             for b in range(n_branches)]
 
 

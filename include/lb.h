@@ -81,13 +81,19 @@ int lb_version(void);
 lb_status lb_pack_signs(const float *latent, int64_t rows, int64_t cols, int64_t ld,
                         int axis, uint32_t *packed, int64_t ld_words, void *stream);
 
-/* One branch of a factorised layer (all device pointers). */
+/* One branch of a factorised layer (device pointers and row pitches).
+ * ld_v / ld_u are the words per packed row of Vp / Up (0 means the unpadded
+ * ceil(in/32) / ceil(r/32)).  Rows padded to a multiple of 4 words (16 bytes)
+ * let the decode kernels stream them with the tensor-memory accelerator; other
+ * pitches take a slower copy path.  Padding words are never read for results. */
 typedef struct {
     const uint32_t *Vp;   /* [r][ld_v] signs of V_b packed along in          */
     const uint32_t *Up;   /* [out][ld_u] signs of U_b packed along r         */
     const uint16_t *h;    /* [out] FP16 row scale (IEEE binary16 bits), 4-byte aligned */
     const uint16_t *g;    /* [in]  FP16 column scale                         */
     const uint16_t *l;    /* [r]   FP16 latent scale                         */
+    int64_t ld_v;         /* words per packed row of Vp, 0 or >= ceil(in/32) */
+    int64_t ld_u;         /* words per packed row of Up, 0 or >= ceil(r/32)  */
 } lb_branch;
 
 /*
@@ -95,7 +101,7 @@ typedef struct {
  *
  *   x         : device, M x in, dtype x_dtype (LB_F16, LB_BF16 or LB_F32)
  *   br        : host array of n_branches (1 or 2) lb_branch; every branch shares
- *               in, out, r, ld_v = ceil(in/32) and ld_u = ceil(r/32)
+ *               in, out and r (each branch has its own row pitches)
  *   y         : device, M x out fp32, overwritten
  *   workspace : device scratch of at least lb_linear_workspace_size(...) bytes,
  *               16-byte aligned; contents need not be initialised and are
