@@ -72,6 +72,20 @@ void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld) {
 
 bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <= (1 << 26)); }
 
+// Give each phase a cost-balanced split of its units over G CTAs, written to
+// `split` (kMaxGrid+1 ints per phase); phases keep the even split if G does
+// not fit the table.
+void plan_splits(LbPhase* phases, int n_phases, const LbJob* jobs, int G, int* split) {
+    for (int p = 0; p < n_phases; ++p) {
+        phases[p].split_off = p * (kMaxGrid + 1);
+        phases[p].split_g = -1;
+        if (G < 1 || G > kMaxGrid) continue;
+        balanced_split(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units, G,
+                       split + phases[p].split_off);
+        phases[p].split_g = G;
+    }
+}
+
 // Append `J` to phase `ph`, assigning its unit range.
 void add_job(LbPhase& ph, std::vector<LbJob>& jobs, LbJob J) {
     J.unit_begin = ph.n_units;
@@ -102,7 +116,7 @@ struct StackLayout {
     std::vector<size_t> region_len;  // [phase] bytes (0: nothing, or y for MLP-only)
     size_t acc_end;                  // end of the accumulator area
     size_t x_dev, y_dev;             // staging for lb_stack_forward_host
-    size_t phases, jobs;             // plan
+    size_t phases, jobs, splits;     // plan
     int n_phases, n_jobs;
     size_t total;
 };
@@ -221,6 +235,8 @@ StackLayout stack_layout(const lb_stack_desc* d) {
     off = round_up(off + sizeof(LbPhase) * (size_t)L.n_phases, 256);
     L.jobs = off;
     off = round_up(off + sizeof(LbJob) * (size_t)L.n_jobs, 256);
+    L.splits = off;
+    off = round_up(off + sizeof(int) * (size_t)(kMaxGrid + 1) * (size_t)L.n_phases, 256);
     L.total = off;
     return L;
 }
@@ -450,6 +466,7 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
         plan.phases[0] = p0;
         plan.phases[1] = p1;
         std::copy(jobs.begin(), jobs.end(), plan.jobs);
+        plan_splits(plan.phases, 2, plan.jobs, decode_grid(), plan.split);
         const size_t zero_bytes = sizeof(WsHeader) + sizeof(float) * (size_t)mc * n_branches * r;
         if (cudaMemsetAsync(workspace, 0, zero_bytes, s) != cudaSuccess) return LB_ERR_CUDA;
         if (launch_linear_plan(plan, hdr, 2, s) != cudaSuccess) return LB_ERR_CUDA;
@@ -482,6 +499,8 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
     std::vector<LbJob> jobs;
     build_stack_plan(d, L, static_cast<char*>(workspace), phases, jobs);
     if ((int)phases.size() != L.n_phases || (int)jobs.size() != L.n_jobs) return LB_ERR_CUDA;
+    std::vector<int> split((size_t)(kMaxGrid + 1) * L.n_phases, 0);
+    plan_splits(phases.data(), L.n_phases, jobs.data(), decode_grid(), split.data());
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
@@ -489,6 +508,9 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
     if (cudaMemcpyAsync(ws + L.jobs, jobs.data(), sizeof(LbJob) * jobs.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return LB_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + L.splits, split.data(), sizeof(int) * split.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
@@ -506,7 +528,8 @@ lb_status lb_stack_forward(const lb_stack_desc* d, void* workspace, size_t ws_by
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     if (launch_stack_plan(reinterpret_cast<const LbPhase*>(ws + L.phases),
-                          reinterpret_cast<const LbJob*>(ws + L.jobs), L.n_phases,
+                          reinterpret_cast<const LbJob*>(ws + L.jobs),
+                          reinterpret_cast<const int*>(ws + L.splits), L.n_phases,
                           reinterpret_cast<WsHeader*>(ws), x, y, s) != cudaSuccess)
         return LB_ERR_CUDA;
     return LB_OK;

@@ -135,9 +135,11 @@ __device__ bool grid_wait(WsHeader* hdr, unsigned target, int* flag) {
     return *flag != 0;
 }
 
-// First unit of CTA `cta` in a phase with n units over G CTAs.
-__device__ __forceinline__ int unit_split(int n, int cta, int G) {
-    return (int)(((long long)n * cta) / G);
+// First unit of CTA `cta` in phase ph: from the host's cost-balanced split
+// table when there is one, else an even split of the units.
+__device__ __forceinline__ int unit_split(const LbPhase& ph, const int* splits, int cta, int G) {
+    if (ph.split_g == G) return splits[ph.split_off + cta];
+    return (int)(((long long)ph.n_units * cta) / G);
 }
 
 // Stage v for slice s of job J into shared memory (zero past cols) and do the
@@ -512,7 +514,7 @@ __device__ __forceinline__ int collect_tiles(const Smem& sm, int n_jobs, int& j,
 }
 
 __device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
-                          uint32_t& ring_it, int* err) {
+                          const int* splits, uint32_t& ring_it, int* err) {
     const int G = gridDim.x, cta = blockIdx.x;
     const LbPhase ph = *sm.phase;
     float* zp = resolve(ph.zero_ptr, args);
@@ -520,8 +522,8 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* job
         for (int i = cta * kDecodeThreads + threadIdx.x; i < ph.zero_n; i += G * kDecodeThreads)
             zp[i] = 0.0f;
     }
-    int u = unit_split(ph.n_units, cta, G);
-    const int u_end = unit_split(ph.n_units, cta + 1, G);
+    int u = unit_split(ph, splits, cta, G);
+    const int u_end = unit_split(ph, splits, cta + 1, G);
     int j = 0;
     while (u < u_end) {
         Tile t[kMaxTiles];
@@ -557,10 +559,10 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* job
 
 // L2 prefetch of the sign segments this CTA will read in phase ph (up to
 // kPrefetchSegments of them, in the order it will read them).
-__device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs) {
+__device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs, const int* splits) {
     const int G = gridDim.x, cta = blockIdx.x;
-    int u = unit_split(ph.n_units, cta, G);
-    const int u_end = unit_split(ph.n_units, cta + 1, G);
+    int u = unit_split(ph, splits, cta, G);
+    const int u_end = unit_split(ph, splits, cta + 1, G);
     int j = ph.job_begin;
     const int j_end = ph.job_begin + ph.n_jobs;
     int budget = kPrefetchSegments;
@@ -591,24 +593,24 @@ __device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs) {
 }
 
 __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jobs,
-                            WsHeader* hdr, const CallArgs& args) {
+                            const int* splits, WsHeader* hdr, const CallArgs& args) {
     const Smem sm = smem_layout();
     const unsigned G = gridDim.x;
     if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) return;   // sticky after a timeout
     if (threadIdx.x < kDecodeWarps * kRingSlots) mbar_init(sm.bars + 8u * threadIdx.x, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     cache_phase(phases, 0, jobs, sm);
-    prefetch_phase(phases[0], jobs);
+    prefetch_phase(phases[0], jobs, splits);
     __syncthreads();
     uint32_t ring_it = 0;
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args, jobs, ring_it, &hdr->error);
+        run_phase(sm, args, jobs, splits, ring_it, &hdr->error);
         if (p + 1 < n_phases) {
             // Announce completion, then use the wait: copy the next phase's
             // plan into shared memory and prefetch its sign rows to L2.
             grid_arrive(hdr);
             cache_phase(phases, p + 1, jobs, sm);
-            prefetch_phase(phases[p + 1], jobs);
+            prefetch_phase(phases[p + 1], jobs, splits);
             if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) return;
         }
     }
@@ -628,14 +630,15 @@ __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jo
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 linear_program_kernel(const __grid_constant__ LinearPlan plan, int n_phases, WsHeader* hdr) {
     const CallArgs args = {nullptr, nullptr};
-    run_program(plan.phases, n_phases, plan.jobs, hdr, args);
+    run_program(plan.phases, n_phases, plan.jobs, plan.split, hdr, args);
 }
 
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 stack_program_kernel(const LbPhase* __restrict__ phases, const LbJob* __restrict__ jobs,
-                     int n_phases, WsHeader* hdr, const void* x, float* y) {
+                     const int* __restrict__ splits, int n_phases, WsHeader* hdr, const void* x,
+                     float* y) {
     const CallArgs args = {x, y};
-    run_program(phases, n_phases, jobs, hdr, args);
+    run_program(phases, n_phases, jobs, splits, hdr, args);
 }
 
 cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
@@ -681,6 +684,59 @@ bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw) {
            CUDA_SUCCESS;
 }
 
+int decode_grid() { return device_sm_count() * kCtasPerSm; }
+
+// Contiguous unit ranges for G CTAs with the smallest largest cost.  The
+// warps of a CTA take a tile's rowblocks kDecodeWarps at a time, so a CTA
+// that takes k rowblocks of a tile spends ceil(k / kDecodeWarps) warp
+// iterations on them, plus kTileCost (in 1/kDecodeWarps iterations) to stage
+// the tile's vector and build its tables.  Units run job by job, slice-major
+// inside a job, so a phase is a list of tiles of n_rowblocks units each; a
+// greedy fill is optimal for a given bound, which a bisection minimises.
+namespace {
+template <class F>
+void for_each_tile(const LbJob* jobs, int n_jobs, F f) {
+    for (int j = 0; j < n_jobs; ++j)
+        for (int s = 0; s < jobs[j].n_slices; ++s) f(jobs[j].n_rowblocks);
+}
+long long take_cost(long long k) {
+    return kTileCost + (k + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps;
+}
+// CTAs a greedy fill under cost bound T needs; boundaries go to `out` if set.
+int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
+    int used = 1, u = 0;
+    long long cost = 0;
+    for_each_tile(jobs, n_jobs, [&](int n) {
+        while (n > 0) {
+            if (cost + take_cost(1) > T) {
+                if (out) out[used] = u;
+                ++used;
+                cost = 0;
+            }
+            const long long room = (T - cost - kTileCost) / kDecodeWarps * kDecodeWarps;
+            const int take = (int)std::min<long long>(n, room);
+            cost += take_cost(take);
+            n -= take;
+            u += take;
+        }
+    });
+    return used;
+}
+}  // namespace
+
+void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out) {
+    long long lo = take_cost(1), hi = lo;
+    for_each_tile(jobs, n_jobs, [&](int n) { hi += take_cost(n); });
+    while (lo < hi) {   // smallest bound a fill of at most G CTAs meets
+        const long long mid = (lo + hi) / 2;
+        if (greedy_fill(jobs, n_jobs, mid, nullptr) <= G) hi = mid;
+        else lo = mid + 1;
+    }
+    const int used = greedy_fill(jobs, n_jobs, lo, out);
+    out[0] = 0;
+    for (int c = used; c <= G; ++c) out[c] = n_units;
+}
+
 cudaError_t decode_configure() {
     cudaError_t e = cudaFuncSetAttribute(linear_program_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDecodeSmem);
@@ -710,9 +766,10 @@ cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phas
     return launch_coop(reinterpret_cast<const void*>(linear_program_kernel), args, s);
 }
 
-cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, int n_phases,
-                              WsHeader* hdr, const void* x, float* y, cudaStream_t s) {
-    void* args[] = {&phases, &jobs, &n_phases, &hdr, &x, &y};
+cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const int* splits,
+                              int n_phases, WsHeader* hdr, const void* x, float* y,
+                              cudaStream_t s) {
+    void* args[] = {&phases, &jobs, &splits, &n_phases, &hdr, &x, &y};
     return launch_coop(reinterpret_cast<const void*>(stack_program_kernel), args, s);
 }
 

@@ -74,7 +74,8 @@ struct alignas(64) LbJob {
 struct LbPhase {
     int job_begin, n_jobs, n_units, zero_n;
     float* zero_ptr;          // if set, the CTAs zero zero_n floats here during the phase
-    long long pad;
+    int split_off;            // offset of this phase's split_g+1 unit boundaries in the split table
+    int split_g;              // CTAs the split was made for (-1 or another grid: even split)
 };
 
 // Stack plans are prepared once and reused with different x / y buffers, so
@@ -87,9 +88,13 @@ constexpr int kDecodeSmem = kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 
 static_assert(kDecodeSmem <= 227 * 1024, "decode kernel shared memory over the per-CTA limit");
 
 // Plan of a single linear call, passed by value as a kernel parameter.
+constexpr int kMaxGrid = 256;                // CTAs a split table has room for
+constexpr int kTileCost = 40;                // vector stage + table build, in 1/16 warp iterations
+
 struct LinearPlan {
-    LbPhase phases[2];
     LbJob jobs[2 * kMaxLinearJobs];
+    LbPhase phases[2];
+    int split[2 * (kMaxGrid + 1)];           // per-phase unit boundaries of the CTAs
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -188,8 +193,12 @@ bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw);
 // Decode phase program launches (lb_decode.cu).
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,
                                cudaStream_t s);
-cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, int n_phases,
-                              WsHeader* hdr, const void* x, float* y, cudaStream_t s);
+cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const int* splits,
+                              int n_phases, WsHeader* hdr, const void* x, float* y,
+                              cudaStream_t s);
+int decode_grid();                   // CTAs of a decode launch on the current device
+// Cost-balanced contiguous unit ranges for the G CTAs of a phase (out: G+1 boundaries).
+void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
 
 // Tensor-core prefill path (lb_prefill.cu).
 constexpr int kPrefillMinM = 16;             // lb_linear_forward uses it from this many rows
