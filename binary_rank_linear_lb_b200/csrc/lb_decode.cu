@@ -142,69 +142,22 @@ __device__ __forceinline__ int unit_split(const LbPhase& ph, const int* splits, 
     return (int)(((long long)ph.n_units * cta) / G);
 }
 
-// Stage v for slice s of job J into shared memory (zero past cols) and do the
-// slice owner's side duties (sum of squares for RMSNorm, residual seeding).
-__device__ void stage_vector(const LbJob& J, int s, bool owner, const Smem& sm, float* vec) {
-    const int j0 = s * kSliceElems;
-    float rs = 1.0f;
-    if (J.kind == VK_T && J.norm_sumsq != nullptr)
-        rs = rsqrtf(__ldcg(J.norm_sumsq) / (float)J.norm_n + kRmsEps);
-    float sq = 0.0f;
-#pragma unroll
-    for (int e = threadIdx.x; e < kSliceElems; e += kDecodeThreads) {
-        const int j = j0 + e;
-        float v = 0.0f;
-        if (j < J.cols) {
-            float raw;
-            switch (J.kind) {
-                case VK_X_F16:
-                    raw = __half2float(reinterpret_cast<const __half*>(J.src)[j]);
-                    v = __half2float(__ldg(J.vscale + j)) * raw;
-                    break;
-                case VK_X_BF16:
-                    raw = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(J.src)[j]);
-                    v = __half2float(__ldg(J.vscale + j)) * raw;
-                    break;
-                case VK_X_F32:
-                    raw = __ldcg(reinterpret_cast<const float*>(J.src) + j);
-                    v = __half2float(__ldg(J.vscale + j)) * raw;
-                    break;
-                case VK_T:
-                    raw = __ldcg(reinterpret_cast<const float*>(J.src) + j);
-                    v = __half2float(__ldg(J.vscale + j)) * (raw * rs);
-                    break;
-                case VK_GQA: {
-                    const int head = j / J.gqa_ghd;
-                    raw = __ldcg(reinterpret_cast<const float*>(J.src) + head * J.gqa_hd +
-                                 (j % J.gqa_hd));
-                    v = __half2float(__ldg(J.vscale + j)) * raw;
-                    break;
-                }
-                default: {  // VK_SILU_MUL
-                    const float gt = __ldcg(reinterpret_cast<const float*>(J.src) + j);
-                    raw = silu(gt) * __ldcg(J.src2 + j);
-                    v = __half2float(__ldg(J.vscale + j)) * raw;
-                    break;
-                }
-            }
-            if (owner) {
-                sq += raw * raw;
-                if (J.resid_init != nullptr) J.resid_init[j] = raw;
-            }
-        }
-        vec[e + (e >> 5)] = v;
-    }
-    if (owner && J.acc_sumsq != nullptr) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        if ((threadIdx.x & 31) == 0) sm.red[threadIdx.x >> 5] = sq;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float tot = 0.0f;
-            for (int w = 0; w < kDecodeWarps; ++w) tot += sm.red[w];
-            atomicAdd(J.acc_sumsq, tot);
-        }
-        __syncthreads();
+// Element j of a job's vector source, before its scale: a is the source
+// value (the gate for VK_SILU_MUL, whose up value goes to b).
+__device__ __forceinline__ void load_src(const LbJob& J, int j, float& a, float& b) {
+    switch (J.kind) {
+        case VK_X_F16: a = __half2float(reinterpret_cast<const __half*>(J.src)[j]); break;
+        case VK_X_BF16: a = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(J.src)[j]); break;
+        case VK_X_F32:
+        case VK_T: a = __ldcg(reinterpret_cast<const float*>(J.src) + j); break;
+        case VK_GQA:
+            a = __ldcg(reinterpret_cast<const float*>(J.src) + (j / J.gqa_ghd) * J.gqa_hd +
+                       (j % J.gqa_hd));
+            break;
+        default:  // VK_SILU_MUL
+            a = __ldcg(reinterpret_cast<const float*>(J.src) + j);
+            b = __ldcg(J.src2 + j);
+            break;
     }
 }
 
@@ -513,8 +466,122 @@ __device__ __forceinline__ int collect_tiles(const Smem& sm, int n_jobs, int& j,
     return n;
 }
 
-__device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
-                          const int* splits, uint32_t& ring_it, int* err) {
+// A batch of up to kMaxTiles tiles whose vectors are staged together.  sc[k]
+// is this thread's element of tile k's vector scale (g or l), which does not
+// depend on earlier phases and is loaded before the grid-wide wait.
+struct Batch {
+    int nt;
+    Tile t[kMaxTiles];
+    float sc[kMaxTiles];
+};
+static_assert(kSliceElems == kDecodeThreads, "one slice element per thread");
+
+// This CTA's place in a phase: units [u, u_end), the job cursor, the batch
+// about to run and how many TMA ring entries this warp has in flight for it.
+struct Cursor {
+    int u, u_end, j, in_flight;
+    Batch b;
+};
+
+// Collect the next batch at c.u, start its first tile's rows streaming and
+// load its scale elements.
+__device__ void batch_begin(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
+                            uint32_t ring_it, Cursor& c) {
+    const LbPhase& ph = *sm.phase;
+    Batch& b = c.b;
+    b.nt = collect_tiles(sm, ph.n_jobs, c.j, c.u, c.u_end, b.t);
+    const LbJob J0 = fetch_job(sm.jobs, b.t[0].job, args);
+    ring_prologue(J0, jobs_g + ph.job_begin + b.t[0].job, b.t[0].slice, b.t[0].rb0, b.t[0].nrb,
+                  sm, ring_it);
+    c.in_flight = J0.use_tma ? min(kRingDepth, warp_rowblocks(b.t[0].nrb)) : 0;
+#pragma unroll
+    for (int k = 0; k < kMaxTiles; ++k) {
+        b.sc[k] = 0.0f;
+        if (k < b.nt) {
+            const LbJob& J = sm.jobs[b.t[k].job];
+            const int col = b.t[k].slice * kSliceElems + (int)threadIdx.x;
+            if (col < J.cols) b.sc[k] = __half2float(__ldg(J.vscale + col));
+        }
+    }
+}
+
+// Stage the batch's vector slices into shared memory (zero past cols): all
+// source loads are issued before any is used, so the batch costs one round
+// trip to L2.  The owner of a slice (the CTA holding its first rowblock) also
+// seeds the residual and adds the slice's sum of squares for RMSNorm; only
+// the first job of a phase carries acc_sumsq, so there is one sum per batch.
+__device__ void stage_batch(const Smem& sm, const CallArgs& args, const Batch& b) {
+    const int e = threadIdx.x;
+    float a[kMaxTiles], a2[kMaxTiles], nrm[kMaxTiles];
+#pragma unroll
+    for (int k = 0; k < kMaxTiles; ++k) {
+        a[k] = 0.0f;
+        a2[k] = 0.0f;
+        nrm[k] = -1.0f;
+        if (k < b.nt) {
+            const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
+            const int col = b.t[k].slice * kSliceElems + e;
+            if (col < J.cols) load_src(J, col, a[k], a2[k]);
+            if (J.kind == VK_T && J.norm_sumsq != nullptr) nrm[k] = __ldcg(J.norm_sumsq);
+        }
+    }
+    float sq = 0.0f;
+    float* acc = nullptr;
+#pragma unroll
+    for (int k = 0; k < kMaxTiles; ++k) {
+        if (k >= b.nt) break;
+        const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
+        const int col = b.t[k].slice * kSliceElems + e;
+        float v = 0.0f;
+        if (col < J.cols) {
+            const float raw = J.kind == VK_SILU_MUL ? silu(a[k]) * a2[k] : a[k];
+            const float rs = nrm[k] >= 0.0f ? rsqrtf(nrm[k] / (float)J.norm_n + kRmsEps) : 1.0f;
+            v = b.sc[k] * (raw * rs);
+            if (b.t[k].rb0 == 0) {
+                if (J.acc_sumsq != nullptr) sq += raw * raw;
+                if (J.resid_init != nullptr) J.resid_init[col] = raw;
+            }
+        }
+        if (b.t[k].rb0 == 0 && J.acc_sumsq != nullptr) acc = J.acc_sumsq;
+        sm.vec[k * kVecPad + e + (e >> 5)] = v;
+    }
+    if (acc != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if ((threadIdx.x & 31) == 0) sm.red[threadIdx.x >> 5] = sq;
+    }
+    __syncthreads();
+    if (acc != nullptr && threadIdx.x == 0) {
+        float tot = 0.0f;
+        for (int w = 0; w < kDecodeWarps; ++w) tot += sm.red[w];
+        atomicAdd(acc, tot);
+    }
+}
+
+// The part of a phase that does not depend on earlier phases, run before the
+// grid-wide wait: this CTA's unit range and its first batch (rows in flight,
+// scales loaded).  sm.phase / sm.jobs must hold the phase.
+__device__ void phase_begin(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
+                            const int* splits, uint32_t ring_it, Cursor& c) {
+    const LbPhase& ph = *sm.phase;
+    c.u = unit_split(ph, splits, blockIdx.x, gridDim.x);
+    c.u_end = unit_split(ph, splits, blockIdx.x + 1, gridDim.x);
+    c.j = 0;
+    c.in_flight = 0;
+    c.b.nt = 0;
+    if (c.u < c.u_end) batch_begin(sm, args, jobs_g, ring_it, c);
+}
+
+// Wait (bounded) for the ring entries a cursor has in flight, before leaving
+// the kernel early: no copy may still be writing this CTA's shared memory.
+__device__ void drain_ring(const Smem& sm, const Cursor& c, uint32_t ring_it, int* err) {
+    for (int d = 0; d < c.in_flight; ++d) tma_wait(sm, ring_it + d, err);
+    cp_async_wait<0>();
+}
+
+// The rest of the phase, after the grid-wide wait.
+__device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g, Cursor& c,
+                          uint32_t& ring_it, int* err) {
     const int G = gridDim.x, cta = blockIdx.x;
     const LbPhase ph = *sm.phase;
     float* zp = resolve(ph.zero_ptr, args);
@@ -522,39 +589,30 @@ __device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* job
         for (int i = cta * kDecodeThreads + threadIdx.x; i < ph.zero_n; i += G * kDecodeThreads)
             zp[i] = 0.0f;
     }
-    int u = unit_split(ph, splits, cta, G);
-    const int u_end = unit_split(ph, splits, cta + 1, G);
-    int j = 0;
-    while (u < u_end) {
-        Tile t[kMaxTiles];
-        const int nt = collect_tiles(sm, ph.n_jobs, j, u, u_end, t);
-        {   // the first tile's rows start streaming while every vector is staged
-            const LbJob J = fetch_job(sm.jobs, t[0].job, args);
-            ring_prologue(J, jobs_g + ph.job_begin + t[0].job, t[0].slice, t[0].rb0, t[0].nrb, sm,
-                          ring_it);
-        }
-        for (int k = 0; k < nt; ++k) {
-            const LbJob J = fetch_job(sm.jobs, t[k].job, args);
-            stage_vector(J, t[k].slice, t[k].rb0 == 0, sm, sm.vec + k * kVecPad);
-        }
-        __syncthreads();
-        for (int k = 0; k < nt; ++k) {
-            const LbJob J = fetch_job(sm.jobs, t[k].job, args);
-            const LbJob* Jg = jobs_g + ph.job_begin + t[k].job;
-            if (k > 0) ring_prologue(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it);
+    bool first = true;
+    while (c.u < c.u_end) {
+        if (!first) batch_begin(sm, args, jobs_g, ring_it, c);
+        first = false;
+        const Batch& b = c.b;
+        stage_batch(sm, args, b);
+        for (int k = 0; k < b.nt; ++k) {
+            const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
+            const LbJob* Jg = jobs_g + ph.job_begin + b.t[k].job;
+            if (k > 0) ring_prologue(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it);
             build_lut(sm, sm.vec + k * kVecPad);
             const bool b1024 = sm.lut == 1024u;
             if (J.use_tma) {
-                if (b1024) lookup_rowblocks<1024u, true>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
-                else lookup_rowblocks<0u, true>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+                if (b1024) lookup_rowblocks<1024u, true>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
+                else lookup_rowblocks<0u, true>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
             } else {
-                if (b1024) lookup_rowblocks<1024u, false>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
-                else lookup_rowblocks<0u, false>(J, Jg, t[k].slice, t[k].rb0, t[k].nrb, sm, ring_it, err);
+                if (b1024) lookup_rowblocks<1024u, false>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
+                else lookup_rowblocks<0u, false>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
             }
             __syncthreads();
-            u += t[k].nrb;
+            c.u += b.t[k].nrb;
         }
     }
+    c.in_flight = 0;
 }
 
 // L2 prefetch of the sign segments this CTA will read in phase ph (up to
@@ -600,18 +658,26 @@ __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jo
     if (threadIdx.x < kDecodeWarps * kRingSlots) mbar_init(sm.bars + 8u * threadIdx.x, 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     cache_phase(phases, 0, jobs, sm);
-    prefetch_phase(phases[0], jobs, splits);
     __syncthreads();
     uint32_t ring_it = 0;
+    Cursor cur;
+    phase_begin(sm, args, jobs, splits, ring_it, cur);
+    prefetch_phase(phases[0], jobs, splits);
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args, jobs, splits, ring_it, &hdr->error);
+        run_phase(sm, args, jobs, cur, ring_it, &hdr->error);
         if (p + 1 < n_phases) {
-            // Announce completion, then use the wait: copy the next phase's
-            // plan into shared memory and prefetch its sign rows to L2.
+            // Announce completion, then use the wait: bring in the next
+            // phase's plan, start its first rows streaming into the ring and
+            // prefetch the rest of this CTA's rows to L2.
             grid_arrive(hdr);
             cache_phase(phases, p + 1, jobs, sm);
+            __syncthreads();
+            phase_begin(sm, args, jobs, splits, ring_it, cur);
             prefetch_phase(phases[p + 1], jobs, splits);
-            if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) return;
+            if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) {
+                drain_ring(sm, cur, ring_it, &hdr->error);
+                return;
+            }
         }
     }
     // The last CTA out resets the arrival counter for the next call.
