@@ -65,9 +65,10 @@ void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld) {
     J.ldw = (int)(ld ? ld : cdiv(cols, 32));
     J.n_slices = (int)cdiv(cols, kSliceElems);
     J.n_rowblocks = (int)cdiv(rows, kRowBlock);
+    J.rg = J.n_rowblocks;
     J.use_tma = 0;
     if ((J.ldw & 3) == 0 && (reinterpret_cast<uintptr_t>(J.P) & 15) == 0)
-        J.use_tma = make_sign_tmap(&J.tmap, J.P, J.rows, J.ldw) ? 1 : 0;
+        J.use_tma = make_sign_tmap(&J.tmap, J.P, J.rows, J.ldw, (int)cdiv(cols, 32)) ? 1 : 0;
 }
 
 bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <= (1 << 26)); }
@@ -75,10 +76,14 @@ bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <
 // Give each phase a cost-balanced split of its units over G CTAs, written to
 // `split` (kMaxGrid+1 ints per phase); phases keep the even split if G does
 // not fit the table.
-void plan_splits(LbPhase* phases, int n_phases, const LbJob* jobs, int G, int* split) {
+void plan_splits(LbPhase* phases, int n_phases, LbJob* jobs, int G, int* split) {
     for (int p = 0; p < n_phases; ++p) {
+        phases[p].next_job_begin = p + 1 < n_phases ? phases[p + 1].job_begin : 0;
+        phases[p].next_n_jobs = p + 1 < n_phases ? phases[p + 1].n_jobs : 0;
         phases[p].split_off = p * (kMaxGrid + 1);
         phases[p].split_g = -1;
+        plan_row_groups(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units,
+                        std::max(G, 1));
         if (G < 1 || G > kMaxGrid) continue;
         balanced_split(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units, G,
                        split + phases[p].split_off);

@@ -11,72 +11,145 @@
 // chunk of 8 consecutive columns, all 256 signed sums  T_c[e] = sum_q (bit q of
 // e ? -v_q : +v_q).  One byte of a packed row then costs one shared-memory load
 // and one add.  With chunk c = 4w + qb (word w = 4*gam + reg of the slice, byte
-// qb of the word) the table entry lives at byte
+// qb of the word) the entry lives at byte
 //     e*256 + (reg&1)*128 + 4*(8*gam + 4*(reg>>1) + qb)
-// of the 64 KB table, i.e. in bank 8*gam + 4*(reg>>1) + qb.
+// of the 64 KB table, i.e. in bank 8*gam + 4*(reg>>1) + qb.  Two tables are
+// resident, at shared-window addresses 64 KB and 128 KB, so bits 16-17 of a
+// lookup address pick the table and a CTA can run the rowblocks of two tiles
+// (two slices or two matrices) as one stream.
 //
 // Lane mapping of the lookups.  Lane l = 4*rho + gam (rho = 0..7 picks one of 8
 // rows of a step, gam = 0..3 one of four 16-byte word groups of the row).  At
 // step (r, jj) the lane reads register r of its group (with the two halves of
 // the group swapped when rho >= 4) and byte (jj + rho) % 4 of that word, so
 // the 32 lanes touch 32 chunks in 32 different banks.  A single PRMT merges the
-// sign byte (the entry index) with a per-lane constant into the address, so a
-// lookup is PRMT + LDS + FADD.
+// sign byte (the entry index) with a per-lane constant that also carries the
+// table's address bits, so a lookup is PRMT + LDS + FADD.
+//
+// Sign words are loaded straight into registers with 128-bit non-allocating
+// loads, kDepth rowblocks ahead of their use; shared memory only holds the
+// tables, whose bandwidth the lookups need.
 //
 // Work split.  A job (one matrix) is cut into units of 32 rows x one slice.
-// The units of a phase are dealt to the CTAs in contiguous, equal ranges; a CTA
-// rebuilds its table whenever its range enters a new (job, slice).  Partial
-// row sums over a slice go to the fp32 output with red.global.add, so the
-// V-contraction result t stays in L2 between the two phases.
+// The host deals each CTA a contiguous, cost-balanced range of units; a CTA
+// takes its range in batches of at most two tiles (a tile = the units of one
+// slice of one job), stages the batch's vector slices, builds their tables
+// and streams the rowblocks.  Partial row sums over a slice go to the fp32
+// output with red.global.add, so the V-contraction result t stays in L2
+// between the two phases.
 //
 // Phases are separated by a grid-wide wait (bounded spin); the kernel is
-// launched cooperatively so that every CTA is resident.  At the start of each
-// phase a CTA issues L2 prefetches for the sign rows it will read in the next
-// phase, so HBM keeps streaming through the waits.
+// launched cooperatively so that every CTA is resident.  Between announcing
+// the end of a phase and waiting for the others, a CTA switches to the next
+// phase's plan (fetched asynchronously one phase ahead) and loads the scales
+// it will stage.  It keeps bulk loads out of the memory queues until the wait
+// and the staging loads after it, which are on the critical path, have been
+// issued.
 #include "lb_internal.cuh"
 
 namespace lb {
 namespace {
 
 constexpr long long kSpinLimitCycles = 4000000000LL;   // ~2 s at 2 GHz
-constexpr int kPrefetchSegments = 2048;                 // next-phase 64-byte segments per CTA
-constexpr int kMaxTiles = 4;                            // tiles whose vectors are staged together
+constexpr int kMaxTiles = kTables;                      // tiles of one batch
+constexpr int kPrefetchDepth = 4;                       // rowblocks a warp has requested ahead (L2)
+constexpr int kEarlyPrefetch = 1;                       // of them, requested before a phase's wait
 
 struct Smem {
-    uint32_t lut;     // shared-window address of the 64 KB table
-    uint32_t ring;    // per-warp rings of sign rowblocks (kRingSlots x 2 KB per warp)
-    float* vec;       // staged vector slices (kMaxTiles of them), index e + e/32
+    float* vec;       // kTables staged slices; element j at j + 4*(j/64)
     float* red;       // 32 floats of reduction scratch
     int* flag;        // one int
     LbPhase* phase;   // the current phase, copied from the plan
+    int* range;       // this CTA's unit range in it (from the split table)
     LbJob* jobs;      // its jobs (at most kMaxPhaseJobs), copied from the plan
-    uint32_t bars;    // per-warp ring mbarriers (kRingSlots per warp), shared address
 };
 
+// Two plan buffers (phase header, unit range, jobs): the current phase's and
+// the next one's, which is copied in while the current phase runs.
+constexpr int kOffPlan = 4 * kTables * kVecPad + 4 * 32 + 64;
+constexpr int kPlanBufBytes = 64 + kMaxPhaseJobs * (int)sizeof(LbJob);
+static_assert(kOffPlan % 64 == 0, "plan buffers must be 64-byte aligned");
+static_assert(kOffPlan + 2 * kPlanBufBytes == kMiscBytes, "shared layout out of step");
+
+__device__ __forceinline__ unsigned char* dyn_smem() {
+    extern __shared__ __align__(64) unsigned char dsmem[];
+    return dsmem;
+}
+
+__device__ __forceinline__ void use_plan_buf(Smem& s, int b) {
+    unsigned char* base = dyn_smem() + kOffPlan + b * kPlanBufBytes;
+    s.phase = reinterpret_cast<LbPhase*>(base);
+    s.range = reinterpret_cast<int*>(base + sizeof(LbPhase));
+    s.jobs = reinterpret_cast<LbJob*>(base + 64);
+}
+
 __device__ __forceinline__ Smem smem_layout() {
-    extern __shared__ __align__(16) unsigned char dsmem[];
+    unsigned char* dsmem = dyn_smem();
     Smem s;
-    s.lut = (uint32_t)__cvta_generic_to_shared(dsmem);
-    s.ring = s.lut + kLutBytes;
-    s.vec = reinterpret_cast<float*>(dsmem + kLutBytes + kRingBytes);
-    s.red = s.vec + 4 * kVecPad;
+    s.vec = reinterpret_cast<float*>(dsmem);
+    s.red = s.vec + kTables * kVecPad;
     s.flag = reinterpret_cast<int*>(s.red + 32);
-    s.phase = reinterpret_cast<LbPhase*>(dsmem + kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64);
-    s.jobs = reinterpret_cast<LbJob*>(reinterpret_cast<unsigned char*>(s.phase) + 64);
-    s.bars = (uint32_t)__cvta_generic_to_shared(s.jobs + kMaxPhaseJobs);
+    use_plan_buf(s, 0);
     return s;
 }
 
-// Copy phase ph and its jobs into shared memory (plan data never changes
-// during a call, so this can run before the grid-wide wait).
-__device__ void cache_phase(const LbPhase* phases, int p, const LbJob* jobs, const Smem& sm) {
-    const LbPhase ph = phases[p];
-    if (threadIdx.x == 0) *sm.phase = ph;
+__device__ __forceinline__ int vpad(int j) { return j + 4 * (j >> 6); }
+
+// Index of this CTA's first unit of phase q in the split table, or -1 when
+// the table has no room for the grid.
+__device__ __forceinline__ int split_index(int q) {
+    return blockIdx.x + 1 <= kMaxGrid ? q * (kMaxGrid + 1) + (int)blockIdx.x : -1;
+}
+
+// Copy phase q, its jobs and this CTA's unit range into plan buffer b, with
+// every thread of the CTA (plan data never changes during a call).
+__device__ void cache_plan(const LbPhase* phases, int q, const LbJob* jobs, const int* splits,
+                           int b) {
+    Smem s;
+    use_plan_buf(s, b);
+    const LbPhase ph = phases[q];
+    if (threadIdx.x == 0) *s.phase = ph;
+    const int si = split_index(q);
+    if (threadIdx.x < 2) s.range[threadIdx.x] = si >= 0 ? splits[si + threadIdx.x] : 0;
     const int n_words = ph.n_jobs * (int)(sizeof(LbJob) / 4);
     const uint32_t* src = reinterpret_cast<const uint32_t*>(jobs + ph.job_begin);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(sm.jobs);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(s.jobs);
     for (int i = threadIdx.x; i < n_words; i += kDecodeThreads) dst[i] = src[i];
 }
+
+__device__ __forceinline__ void cp_async(void* dst, const void* src, int bytes) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    if (bytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(d), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" :: "r"(d), "l"(src) : "memory");
+}
+
+// The same copy done asynchronously by one warp (the plan must be in global
+// memory); the job range comes from the previous phase's header.  Completed
+// by plan_wait in the same warp before a CTA barrier.
+__device__ void cache_plan_async(const LbPhase* phases, int q, int job_begin, int n_jobs,
+                                 const LbJob* jobs, const int* splits, int b) {
+    Smem s;
+    use_plan_buf(s, b);
+    const int lane = threadIdx.x & 31;
+    constexpr int kHdrPieces = (int)sizeof(LbPhase) / 16;
+    constexpr int kJobPieces = (int)sizeof(LbJob) / 16;
+    const int n = kHdrPieces + n_jobs * kJobPieces;
+    for (int i = lane; i < n; i += 32) {
+        if (i < kHdrPieces)
+            cp_async(reinterpret_cast<uint4*>(s.phase) + i,
+                     reinterpret_cast<const uint4*>(phases + q) + i, 16);
+        else
+            cp_async(reinterpret_cast<uint4*>(s.jobs) + (i - kHdrPieces),
+                     reinterpret_cast<const uint4*>(jobs + job_begin) + (i - kHdrPieces), 16);
+    }
+    const int si = split_index(q);
+    if (lane < 2 && si >= 0) cp_async(s.range + lane, splits + si + lane, 4);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void plan_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
 
@@ -90,15 +163,6 @@ __device__ __forceinline__ T* resolve(T* p, const CallArgs& a) {
     if ((const void*)p == LB_TAG_X) return (T*)a.x;
     if ((const void*)p == LB_TAG_Y) return (T*)a.y;
     return p;
-}
-
-// Local copy of a job with the call's x / y substituted for their tags.
-__device__ __forceinline__ LbJob fetch_job(const LbJob* jobs, int j, const CallArgs& a) {
-    LbJob J = jobs[j];
-    J.src = resolve(J.src, a);
-    J.out = resolve(J.out, a);
-    J.resid_init = resolve(J.resid_init, a);
-    return J;
 }
 
 // Grid-wide wait, split in two so a CTA can issue the next phase's loads and
@@ -135,311 +199,70 @@ __device__ bool grid_wait(WsHeader* hdr, unsigned target, int* flag) {
     return *flag != 0;
 }
 
-// First unit of CTA `cta` in phase ph: from the host's cost-balanced split
-// table when there is one, else an even split of the units.
-__device__ __forceinline__ int unit_split(const LbPhase& ph, const int* splits, int cta, int G) {
-    if (ph.split_g == G) return splits[ph.split_off + cta];
-    return (int)(((long long)ph.n_units * cta) / G);
+// This CTA's unit range of the phase in sm: from the host's cost-balanced
+// split table when it was made for this grid, else an even split.
+__device__ __forceinline__ void unit_range(const Smem& sm, int& u, int& u_end) {
+    const LbPhase& ph = *sm.phase;
+    const int G = gridDim.x, cta = blockIdx.x;
+    if (ph.split_g == G) {
+        u = sm.range[0];
+        u_end = sm.range[1];
+    } else {
+        u = (int)(((long long)ph.n_units * cta) / G);
+        u_end = (int)(((long long)ph.n_units * (cta + 1)) / G);
+    }
 }
 
 // Element j of a job's vector source, before its scale: a is the source
 // value (the gate for VK_SILU_MUL, whose up value goes to b).
-__device__ __forceinline__ void load_src(const LbJob& J, int j, float& a, float& b) {
+__device__ __forceinline__ void load_src(const LbJob& J, const void* src, int j, float& a,
+                                         float& b) {
     switch (J.kind) {
-        case VK_X_F16: a = __half2float(reinterpret_cast<const __half*>(J.src)[j]); break;
-        case VK_X_BF16: a = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(J.src)[j]); break;
+        case VK_X_F16: a = __half2float(reinterpret_cast<const __half*>(src)[j]); break;
+        case VK_X_BF16: a = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[j]); break;
         case VK_X_F32:
-        case VK_T: a = __ldcg(reinterpret_cast<const float*>(J.src) + j); break;
+        case VK_T: a = __ldcg(reinterpret_cast<const float*>(src) + j); break;
         case VK_GQA:
-            a = __ldcg(reinterpret_cast<const float*>(J.src) + (j / J.gqa_ghd) * J.gqa_hd +
+            a = __ldcg(reinterpret_cast<const float*>(src) + (j / J.gqa_ghd) * J.gqa_hd +
                        (j % J.gqa_hd));
             break;
         default:  // VK_SILU_MUL
-            a = __ldcg(reinterpret_cast<const float*>(J.src) + j);
+            a = __ldcg(reinterpret_cast<const float*>(src) + j);
             b = __ldcg(J.src2 + j);
             break;
     }
 }
 
-// Build the 64 chunk tables of the staged slice.  Warp wp fills words with
-// reg & 1 == wp & 1 and high nibbles (wp >> 1)*4 .. +3; lane = 8*gam + 4*h2 + qb
-// owns chunk 4*(4*gam + 2*h2 + (wp&1)) + qb, which sits in bank `lane`.
-__device__ void build_lut(const Smem& sm, const float* vec) {
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int gam = lane >> 3, h2 = (lane >> 2) & 1, qb = lane & 3;
-    const int w = 4 * gam + 2 * h2 + (wp & 1);
-    const int e0 = 32 * w + 8 * qb;                    // first element of the chunk
-    const float* u = vec + e0 + (e0 >> 5);
-    const float u0 = u[0], u1 = u[1], u2 = u[2], u3 = u[3];
-    const float u4 = u[4], u5 = u[5], u6 = u[6], u7 = u[7];
+// Build the table of one staged slice at shared address taddr.  Thread t owns
+// chunk c (slot i = t & 63: qb = i&3, wb1 = (i>>2)&1, gam = (i>>3)&3,
+// reg&1 = i>>5) and the 32 entries e = 32*(t>>6) + m, m = 0..31; a warp's 32
+// lanes write one entry of 32 chunks in 32 different banks.  Entry
+// e = L(m) + H(t>>6) with L the signed sum of elements 0..4 and H that of 5..7.
+__device__ __forceinline__ void build_table(const float* vec, uint32_t taddr) {
+    const int t = threadIdx.x;
+    const int i = t & 63, k = t >> 6;
+    const int qb = i & 3, wb1 = (i >> 2) & 1, gam = (i >> 3) & 3, w0 = i >> 5;
+    const int c = 4 * (4 * gam + 2 * wb1 + w0) + qb;
+    const float4 lo = *reinterpret_cast<const float4*>(vec + vpad(8 * c));
+    const float4 hi = *reinterpret_cast<const float4*>(vec + vpad(8 * c) + 4);
     // bit q of the entry index set <=> element q enters with sign -1
-    const float p01[4] = {u0 + u1, u1 - u0, u0 - u1, -u0 - u1};
-    const float p23[4] = {u2 + u3, u3 - u2, u2 - u3, -u2 - u3};
-    const float q45[4] = {u4 + u5, u5 - u4, u4 - u5, -u4 - u5};
-    const float q67[4] = {u6 + u7, u7 - u6, u6 - u7, -u6 - u7};
-    float lo[16];
+    const float p01[4] = {lo.x + lo.y, lo.y - lo.x, lo.x - lo.y, -lo.x - lo.y};
+    const float p23[4] = {lo.z + lo.w, lo.w - lo.z, lo.z - lo.w, -lo.z - lo.w};
+    const float hk = ((k & 1) ? -hi.y : hi.y) + ((k & 2) ? -hi.z : hi.z) + ((k & 4) ? -hi.w : hi.w);
+    const float c0 = hk + hi.x, c1 = hk - hi.x;
+    const uint32_t base = taddr + (uint32_t)k * (32u * 256u) + (uint32_t)w0 * 128u +
+                          (uint32_t)(32 * gam + 16 * wb1 + 4 * qb);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) lo[m] = p01[m & 3] + p23[m >> 2];
-    const uint32_t base = sm.lut + (uint32_t)(wp & 1) * 128u + (uint32_t)lane * 4u;
-    constexpr int kNibPerWarp = 16 / (kDecodeWarps / 2);
-    const int hb = (wp >> 1) * kNibPerWarp;
-#pragma unroll
-    for (int n = 0; n < kNibPerWarp; ++n) {
-        const int hn = hb + n;
-        const float hi = q45[hn & 3] + q67[hn >> 2];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const uint32_t addr = base + (uint32_t)(hn * 16 + m) * 256u;
-            asm volatile("st.shared.f32 [%0], %1;" :: "r"(addr), "f"(hi + lo[m]) : "memory");
-        }
-    }
-    __syncthreads();
-}
-
-// L2 prefetch of the slice-s segment of one row (the one or two 128-byte
-// lines it touches; plain prefetches go through the LSU, which issues them far
-// faster than the bulk-copy engine would take one small request at a time).
-__device__ __forceinline__ void prefetch_segment(const LbJob& J, int s, int row) {
-    const int w0 = s * kSliceWords;
-    if (row < J.rows && w0 < J.ldw) {
-        const uint32_t* p = J.P + (size_t)row * (size_t)J.ldw + w0;
-        const int nw = min(kSliceWords, J.ldw - w0);
-        prefetch_l2(p);
-        if ((reinterpret_cast<uintptr_t>(p) >> 7) != (reinterpret_cast<uintptr_t>(p + nw - 1) >> 7))
-            prefetch_l2(p + nw - 1);
+    for (int m = 0; m < 16; ++m) {
+        const float l4 = p01[m & 3] + p23[m >> 2];
+        asm volatile("st.shared.f32 [%0], %1;" :: "r"(base + (uint32_t)m * 256u), "f"(l4 + c0)
+                     : "memory");
+        asm volatile("st.shared.f32 [%0], %1;" :: "r"(base + (uint32_t)(m + 16) * 256u),
+                     "f"(l4 + c1) : "memory");
     }
 }
 
-// ---- per-warp ring of sign rowblocks, filled with cp.async ----------------
-// Lane l = 4*rho + gam copies exactly the 16 bytes it later reads (words
-// 4*gam .. 4*gam+3 of row 8*i + rho of the rowblock, i = 0..3) to
-// ring + slot*2KB + i*512 + l*16, so no cross-lane synchronisation is needed:
-// cp.async.wait_group on the lane's own groups is enough.  Bytes outside the
-// matrix are zero-filled (source size 0).
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t n) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src, uint32_t n) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" :: "r"(dst), "l"(src), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t n) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
-}
-
-// Slot layout: 4 row-steps x 32 lanes x 16 bytes of signs, then 32 lanes x
-// 4 bytes holding the fp16 row scale h of the lane's output row.
-__device__ __forceinline__ uint32_t ring_slot(const Smem& sm, int slot) {
-    return sm.ring + (uint32_t)((((threadIdx.x >> 5) * kRingSlots) + slot) * kRingSlotBytes) +
-           (uint32_t)(threadIdx.x & 31) * 16u;
-}
-__device__ __forceinline__ uint32_t ring_hslot(uint32_t slot_lane_addr) {
-    // slot base + 2048 + lane*4 (slot_lane_addr = slot base + lane*16)
-    const uint32_t lane = threadIdx.x & 31;
-    return slot_lane_addr - lane * 16u + (uint32_t)kRowBlockBytes + lane * 4u;
-}
-
-// Issue this lane's copies of rowblock rb (slice s) into the ring slot at dst.
-// Lanes with rho >= 4 store the two 8-byte halves of their 16 bytes swapped,
-// which is the order their lookups read them in.  The lane also copies the
-// 4-byte word holding h[row] of its output row (second contraction only).
-__device__ __forceinline__ void issue_rowblock(const LbJob& J, int s, int rb, uint32_t dst) {
-    const int lane = threadIdx.x & 31;
-    const int rho = lane >> 2, gam = lane & 3;
-    const uint32_t sw = (rho >> 2) ? 8u : 0u;
-    const int w = s * kSliceWords + 4 * gam;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int row = rb * kRowBlock + 8 * i + rho;
-        const bool rok = row < J.rows;
-        const uint32_t* p = rok ? J.P + (size_t)row * (size_t)J.ldw + w : J.P;
-        const uint32_t d = dst + (uint32_t)i * 512u;
-        if ((J.ldw & 1) == 0) {
-            cp_async_8(d + sw, p, (rok && w < J.ldw) ? 8u : 0u);
-            cp_async_8(d + (8u - sw), rok && w + 2 < J.ldw ? p + 2 : J.P,
-                       (rok && w + 2 < J.ldw) ? 8u : 0u);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                cp_async_4(d + (((uint32_t)(4 * q) + sw) & 15u), rok && w + q < J.ldw ? p + q : J.P,
-                           (rok && w + q < J.ldw) ? 4u : 0u);
-        }
-    }
-    if (J.oscale != nullptr) {
-        const int orow = rb * kRowBlock + 8 * gam + rho;
-        const int h0 = orow & ~1;                        // h is 4-byte aligned (checked on entry)
-        const uint32_t nb = orow >= J.rows ? 0u : (h0 + 1 < J.rows ? 4u : 2u);
-        cp_async_4(ring_hslot(dst), nb ? J.oscale + h0 : J.oscale, nb);
-    }
-}
-
-// ---- TMA-fed ring (rows with a 16-byte pitch) -----------------------------
-// Lane 0 of a warp loads a whole rowblock (32 rows x 16 words, 2 KB) with one
-// 2-D tensor copy into the warp's ring slot; the slot's mbarrier counts the
-// bytes.  The box lands row-major, 64 bytes per row, which is the same layout
-// the cp.async path writes (minus the half swap of rows 4..7 of each step).
-// ring_it counts the rowblocks this warp has consumed so far in this launch;
-// slot = it % kRingSlots, mbarrier phase parity = (it / kRingSlots) & 1.
-__device__ __forceinline__ uint32_t ring_bar(const Smem& sm, uint32_t it) {
-    return sm.bars + (uint32_t)(((threadIdx.x >> 5) * kRingSlots + (int)(it % kRingSlots)) * 8);
-}
-__device__ __forceinline__ uint32_t ring_slot_base(const Smem& sm, uint32_t it) {
-    return sm.ring + (uint32_t)((((threadIdx.x >> 5) * kRingSlots) + (int)(it % kRingSlots)) *
-                                kRingSlotBytes);
-}
-// Issue (lane 0) the TMA of rowblock rb of slice s as ring entry `it`.  The
-// slot was last read by this warp: every lane has passed __syncwarp, and the
-// proxy fence orders those reads before the tensor copy's writes.
-__device__ __forceinline__ void tma_issue(const LbJob* Jg, int s, int rb, const Smem& sm,
-                                          uint32_t it) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) {
-        fence_proxy_async_smem();
-        const uint32_t bar = ring_bar(sm, it);
-        mbar_expect_tx(bar, (uint32_t)kRowBlockBytes);
-        tma_load_2d(ring_slot_base(sm, it), &Jg->tmap, bar, s * kSliceWords, rb * kRowBlock);
-    }
-}
-// Bounded wait for ring entry `it`; on time-out records LB_ERR_TIMEOUT.
-__device__ __forceinline__ void tma_wait(const Smem& sm, uint32_t it, int* err) {
-    const uint32_t bar = ring_bar(sm, it), par = (it / kRingSlots) & 1u;
-    if (mbar_try_wait(bar, par)) return;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, par)) {
-        if (clock64() - t0 > kSpinLimitCycles) {
-            atomicExch(err, (int)LB_ERR_TIMEOUT);
-            return;
-        }
-    }
-}
-
-// Number of rowblocks warp wp takes in a tile of nrb rowblocks.
-__device__ __forceinline__ int warp_rowblocks(int nrb) {
-    const int wp = threadIdx.x >> 5;
-    return wp < nrb ? (nrb - wp + kDecodeWarps - 1) / kDecodeWarps : 0;
-}
-
-// First kRingDepth rowblocks of this warp's share of a tile (issued before the
-// tile's vector is staged, so the copies overlap staging and table build).
-// The cp.async path always commits exactly kRingDepth groups.
-__device__ __forceinline__ void ring_prologue(const LbJob& J, const LbJob* Jg, int s, int rb0,
-                                              int nrb, const Smem& sm, uint32_t ring_it) {
-    const int wp = threadIdx.x >> 5;
-    const int nit = warp_rowblocks(nrb);
-    if (J.use_tma) {
-        for (int d = 0; d < kRingDepth && d < nit; ++d)
-            tma_issue(Jg, s, rb0 + wp + d * kDecodeWarps, sm, ring_it + d);
-        return;
-    }
-#pragma unroll
-    for (int d = 0; d < kRingDepth; ++d) {
-        if (d < nit) issue_rowblock(J, s, rb0 + wp + d * kDecodeWarps, ring_slot(sm, d));
-        cp_async_commit();
-    }
-}
-
-// Look up this warp's rowblocks of slice s of job J against the table; the
-// rowblocks stream through the warp's ring kRingDepth ahead of use.  kBase is
-// the table's shared-window address when it is the usual 1024 (then it folds
-// into the load's immediate offset), else 0 and tbase is added at run time.
-template <uint32_t kBase, bool kTma>
-__device__ __forceinline__ void lookup_rowblocks(const LbJob& J, const LbJob* Jg, int s, int rb0,
-                                                 int nrb, const Smem& sm, uint32_t& ring_it,
-                                                 int* err) {
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int rho = lane >> 2, gam = lane & 3;
-    const uint32_t swap = (uint32_t)(rho >> 2);
-    uint32_t B[2][4], S[4];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        const uint32_t qbj = (uint32_t)((jj + rho) & 3);
-        S[jj] = 0x7604u | (qbj << 4);                    // [B.b0, word.byte qbj, B.b2, B.b3]
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh)
-            B[rh][jj] = (8u * (uint32_t)gam + 4u * ((uint32_t)rh ^ swap) + qbj) * 4u +
-                        (kBase == 0 ? sm.lut : 0u);
-    }
-    const int nit = warp_rowblocks(nrb);
-    const bool has_h = J.oscale != nullptr;
-    for (int n = 0; n < nit; ++n) {
-        const int rb = rb0 + wp + n * kDecodeWarps;
-        uint32_t src;
-        float hs_early = 1.0f;
-        const int orow_e = rb * kRowBlock + 8 * gam + rho;
-        if (kTma) {
-            if (n + kRingDepth < nit)
-                tma_issue(Jg, s, rb + kRingDepth * kDecodeWarps, sm, ring_it + n + kRingDepth);
-            if (has_h && orow_e < J.rows) hs_early = __half2float(__ldg(J.oscale + orow_e));
-            tma_wait(sm, ring_it + n, err);
-            src = ring_slot_base(sm, ring_it + n) + (uint32_t)lane * 16u;
-        } else {
-            if (n + kRingDepth < nit)
-                issue_rowblock(J, s, rb + kRingDepth * kDecodeWarps,
-                               ring_slot(sm, (n + kRingDepth) % kRingSlots));
-            cp_async_commit();
-            cp_async_wait<kRingDepth>();                 // rowblock n has landed
-            src = ring_slot(sm, n % kRingSlots);
-        }
-        float acc[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t w4[4];
-            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                         : "r"(src + (uint32_t)i * 512u));
-            if (kTma && swap) {                          // rows 4..7 read the halves swapped
-                const uint32_t t0 = w4[0], t1 = w4[1];
-                w4[0] = w4[2]; w4[1] = w4[3]; w4[2] = t0; w4[3] = t1;
-            }
-            float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) +
-                                          (uint32_t)(r & 1) * 128u + kBase;
-                    const float v = lds_f32(addr);
-                    if (jj & 1) a1 += v; else a0 += v;
-                }
-            }
-            acc[i] = a0 + a1;
-        }
-        const int orow = orow_e;                           // output row of this lane
-        float hs = hs_early;
-        if (!kTma && has_h) {
-            uint32_t hw;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(hw) : "r"(ring_hslot(src)));
-            const unsigned short hb = (unsigned short)((orow & 1) ? (hw >> 16) : (hw & 0xFFFFu));
-            hs = __half2float(__ushort_as_half(hb));
-        }
-        // Transpose-reduce over the 4 lanes of a row (gam = lane bits 0-1):
-        // afterwards lane gam holds the slice sum of row-step i = gam.
-        const bool up2 = (gam & 2) != 0, up1 = (gam & 1) != 0;
-        float n2[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const float send = up2 ? acc[k] : acc[k + 2];
-            const float keep = up2 ? acc[k + 2] : acc[k];
-            n2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-        }
-        const float send1 = up1 ? n2[0] : n2[1];
-        const float keep1 = up1 ? n2[1] : n2[0];
-        const float tot = keep1 + __shfl_xor_sync(0xffffffffu, send1, 1);
-        if (orow < J.rows) red_add_f32(J.out + orow, tot * hs);
-    }
-    if (kTma) ring_it += (uint32_t)nit;
-    else cp_async_wait<0>();
-}
-
+// ---- tiles and batches ----------------------------------------------------
 __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int u) {
     while (j + 1 < j_end && jobs[j + 1].unit_begin <= u) ++j;
     return j;
@@ -449,68 +272,285 @@ struct Tile {
     int job, slice, rb0, nrb;
 };
 
-// Up to kMaxTiles tiles of this CTA's unit range, starting at unit u.
-__device__ __forceinline__ int collect_tiles(const Smem& sm, int n_jobs, int& j, int u, int u_end,
-                                             Tile (&t)[kMaxTiles]) {
-    int n = 0;
-    while (u < u_end && n < kMaxTiles) {
-        j = find_job(sm.jobs, j, n_jobs, u);
-        const LbJob& J = sm.jobs[j];
-        const int local = u - J.unit_begin;
-        const int s = local / J.n_rowblocks;
-        const int rb0 = local - s * J.n_rowblocks;
-        const int nrb = min(J.n_rowblocks - rb0, u_end - u);
-        t[n++] = Tile{j, s, rb0, nrb};
-        u += nrb;
-    }
-    return n;
+// The tile of this CTA's unit range that starts at unit u (u < u_end).  A
+// job's units run row group by row group, slice by slice inside a group, so
+// the CTAs holding the slices of one group stream the same rows together and
+// each DRAM page is read while it is open.
+__device__ __forceinline__ Tile next_tile(const LbJob* jobs, int n_jobs, int& j, int u, int u_end) {
+    j = find_job(jobs, j, n_jobs, u);
+    const LbJob& J = jobs[j];
+    const int local = u - J.unit_begin;
+    const int per_group = J.rg * J.n_slices;
+    const int g = local / per_group;
+    const int off = local - g * per_group;
+    const int rows_g = min(J.rg, J.n_rowblocks - g * J.rg);
+    const int s = off / rows_g;
+    const int rbi = off - s * rows_g;
+    return Tile{j, s, g * J.rg + rbi, min(rows_g - rbi, u_end - u)};
 }
 
-// A batch of up to kMaxTiles tiles whose vectors are staged together.  sc[k]
-// is this thread's element of tile k's vector scale (g or l), which does not
-// depend on earlier phases and is loaded before the grid-wide wait.
-struct Batch {
-    int nt;
-    Tile t[kMaxTiles];
-    float sc[kMaxTiles];
+// What the lookup loop needs of one tile of the current batch.
+struct TileRt {
+    const uint32_t* P;       // first word of the slice in row 0
+    const __half* h;         // row scales (second contraction) or nullptr
+    float* out;
+    int ldw, rows, wrem;     // row pitch, rows, words of the slice holding signs (<= 16)
+    int rb0, nrb;
+    uint32_t tb;             // table address bits (kTableAddr0 + t * 64 KB)
+    const CUtensorMap* tmap; // the job's tensor map (in the plan), or nullptr: no L2 prefetch
+    int x;                   // the slice's first word (tensor-map coordinate)
 };
-static_assert(kSliceElems == kDecodeThreads, "one slice element per thread");
 
-// This CTA's place in a phase: units [u, u_end), the job cursor, the batch
-// about to run and how many TMA ring entries this warp has in flight for it.
+// This CTA's place in a phase and the batch about to run.  sc[k] is this
+// thread's element of tile k's vector scale (g or l), which does not depend
+// on earlier phases and is loaded before the grid-wide wait.
 struct Cursor {
-    int u, u_end, j, in_flight;
-    Batch b;
+    int u, u_end, j;
+    int nt, n_rb;
+    int pf0;                 // rowblock steps of the batch already prefetched to L2
+    Tile t[kMaxTiles];
+    TileRt rt[kMaxTiles];
+    unsigned short sc[kMaxTiles];   // fp16 bits
 };
 
-// Collect the next batch at c.u, start its first tile's rows streaming and
-// load its scale elements.
-__device__ void batch_begin(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
-                            uint32_t ring_it, Cursor& c) {
-    const LbPhase& ph = *sm.phase;
-    Batch& b = c.b;
-    b.nt = collect_tiles(sm, ph.n_jobs, c.j, c.u, c.u_end, b.t);
-    const LbJob J0 = fetch_job(sm.jobs, b.t[0].job, args);
-    ring_prologue(J0, jobs_g + ph.job_begin + b.t[0].job, b.t[0].slice, b.t[0].rb0, b.t[0].nrb,
-                  sm, ring_it);
-    c.in_flight = J0.use_tma ? min(kRingDepth, warp_rowblocks(b.t[0].nrb)) : 0;
+// One rowblock (32 rows x 16 words of a slice) as this lane holds it: row
+// step i covers rows 4*rho + i, the lane's words 4*gam .. 4*gam+3; h is the
+// row scale of the lane's output row (row `lane` of the rowblock).
+struct RB {
+    uint4 d[4];
+    unsigned short h;   // fp16 bits, converted at use so the load does not stall the warp
+};
+
+__device__ __forceinline__ uint2 ld_stream_v2(const uint32_t* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+
+// Load rowblock rb of tile T into R.  Rows past the matrix and words past the
+// signs are zero (their vector elements are zero, so any value would do; the
+// point is to read neither outside the matrix nor a padded row's pitch).
+__device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
+    const int lane = threadIdx.x & 31;
+    const int rho = lane >> 2, gam = lane & 3;
+    const int w = 4 * gam;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int row = rb * kRowBlock + 4 * rho + i;
+        uint4 d = make_uint4(0u, 0u, 0u, 0u);
+        if (row < T.rows && w < T.wrem) {
+            const uint32_t* p = T.P + (size_t)row * (size_t)T.ldw + w;
+            if ((T.ldw & 3) == 0 && w + 4 <= T.wrem) {
+                d = ld_stream_v4(p);
+            } else if ((T.ldw & 1) == 0) {
+                const uint2 a = ld_stream_v2(p);
+                d.x = a.x; d.y = a.y;
+                if (w + 2 < T.wrem) {
+                    const uint2 b = ld_stream_v2(p + 2);
+                    d.z = b.x; d.w = b.y;
+                }
+            } else {
+                d.x = ld_stream_u32(p);
+                if (w + 1 < T.wrem) d.y = ld_stream_u32(p + 1);
+                if (w + 2 < T.wrem) d.z = ld_stream_u32(p + 2);
+                if (w + 3 < T.wrem) d.w = ld_stream_u32(p + 3);
+            }
+        }
+        R.d[i] = d;
+    }
+    R.h = 0x3C00u;   // 1.0
+    if (T.h != nullptr) {
+        const int orow = rb * kRowBlock + lane;
+        R.h = orow < T.rows ? __ldg(reinterpret_cast<const unsigned short*>(T.h) + orow) : 0u;
+    }
+}
+
+// Look up rowblock R against the table at address bits tb and add the row
+// sums (times the row scale) to out.
+__device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
+                                           const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
+    const int lane = threadIdx.x & 31;
+    const int rho = lane >> 2, gam = lane & 3;
+    const bool swap = rho >= 4;
+    uint32_t B[2][4];
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) B[rh][jj] = Bc[rh][jj] + T.tb;
+    float acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t w4[4];
+        w4[0] = swap ? R.d[i].z : R.d[i].x;
+        w4[1] = swap ? R.d[i].w : R.d[i].y;
+        w4[2] = swap ? R.d[i].x : R.d[i].z;
+        w4[3] = swap ? R.d[i].y : R.d[i].w;
+        float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) + (uint32_t)(r & 1) * 128u;
+                const float v = lds_f32(addr);
+                if (jj & 1) a1 += v; else a0 += v;
+            }
+        }
+        acc[i] = a0 + a1;
+    }
+    // Transpose-reduce over the 4 lanes of a row group (gam = lane bits 0-1):
+    // afterwards lane gam of group rho holds the slice sum of row 4*rho + gam,
+    // i.e. lane l holds row l of the rowblock.
+    const bool up2 = (gam & 2) != 0, up1 = (gam & 1) != 0;
+    float n2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float send = up2 ? acc[k] : acc[k + 2];
+        const float keep = up2 ? acc[k + 2] : acc[k];
+        n2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    const float send1 = up1 ? n2[0] : n2[1];
+    const float keep1 = up1 ? n2[1] : n2[0];
+    const float tot = (keep1 + __shfl_xor_sync(0xffffffffu, send1, 1)) *
+                      __half2float(__ushort_as_half(R.h));
+    // Lane 4q adds rows 4q..4q+3 with one vector reduction (the L2 takes a
+    // 16-byte reduction at the rate of a 4-byte one); partial or unaligned
+    // groups fall back to one reduction per row.
+    const float t1 = __shfl_down_sync(0xffffffffu, tot, 1);
+    const float t2 = __shfl_down_sync(0xffffffffu, tot, 2);
+    const float t3 = __shfl_down_sync(0xffffffffu, tot, 3);
+    const int g0 = rb * kRowBlock + 4 * rho;             // first row of the lane's group
+    float* og = T.out + g0;
+    if (g0 + 4 <= T.rows && (reinterpret_cast<uintptr_t>(og) & 15u) == 0) {
+        if (gam == 0) red_add_v4_f32(og, tot, t1, t2, t3);
+    } else if (g0 + gam < T.rows) {
+        red_add_f32(og + gam, tot);
+    }
+}
+
+// Rowblock n of a batch (n < n_rb): its tile (selected field by field, so
+// the cursor stays in registers) and its rowblock index.
+__device__ __forceinline__ TileRt batch_tile(const Cursor& c, int n, int& rb) {
+    const bool k = c.nt > 1 && n >= c.rt[0].nrb;
+    TileRt T;
+    T.P = k ? c.rt[1].P : c.rt[0].P;
+    T.h = k ? c.rt[1].h : c.rt[0].h;
+    T.out = k ? c.rt[1].out : c.rt[0].out;
+    T.ldw = k ? c.rt[1].ldw : c.rt[0].ldw;
+    T.rows = k ? c.rt[1].rows : c.rt[0].rows;
+    T.wrem = k ? c.rt[1].wrem : c.rt[0].wrem;
+    T.rb0 = k ? c.rt[1].rb0 : c.rt[0].rb0;
+    T.nrb = k ? c.rt[1].nrb : c.rt[0].nrb;
+    T.tb = k ? c.rt[1].tb : c.rt[0].tb;
+    T.tmap = k ? c.rt[1].tmap : c.rt[0].tmap;
+    T.x = k ? c.rt[1].x : c.rt[0].x;
+    rb = T.rb0 + (k ? n - c.rt[0].nrb : n);
+    return T;
+}
+
+// Lane 0 asks the TMA unit to bring rowblock n of the batch into L2 (no data
+// comes back to the SM; the register loads kDepth rowblocks later then hit L2).
+__device__ __forceinline__ void prefetch_rb(const Cursor& c, int n) {
+    if ((threadIdx.x & 31) == 0 && n < c.n_rb) {
+        int rb;
+        const TileRt T = batch_tile(c, n, rb);
+        if (T.tmap != nullptr) tma_prefetch_2d(T.tmap, T.x, rb * kRowBlock);
+    }
+}
+
+// L2 prefetches for this warp's rowblocks d = from .. to-1 steps ahead
+// (n = wp + d * kDecodeWarps).  They never stall the warp: the TMA unit
+// takes them, and no data returns to the SM.
+__device__ __forceinline__ void batch_prefetch(const Cursor& c, int from, int to) {
+    const int wp = threadIdx.x >> 5;
+    for (int d = from; d < to; ++d) prefetch_rb(c, wp + d * kDecodeWarps);
+}
+
+// Issue this warp's first kDepth rowblocks of the batch into buf.  Register
+// loads can stall a warp at issue once the SM's outstanding misses fill up,
+// so they are issued only after the batch's tables are built.
+__device__ __forceinline__ void batch_loads(const Cursor& c, RB (&buf)[kDepth]) {
+    const int wp = threadIdx.x >> 5;
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+        const int n = wp + d * kDecodeWarps;
+        if (n < c.n_rb) {
+            int rb;
+            const TileRt T = batch_tile(c, n, rb);
+            load_rb(T, rb, buf[d]);
+        }
+    }
+}
+
+// Stream this warp's rowblocks of the batch (n = wp, wp + 16, ...) through
+// the register ring buf, kDepth ahead of their use; the first kDepth were
+// issued by batch_loads.
+__device__ __forceinline__ void batch_lookups(const Cursor& c, RB (&buf)[kDepth],
+                                              const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
+    const int wp = threadIdx.x >> 5;
+    for (int n0 = wp; n0 < c.n_rb; n0 += kDepth * kDecodeWarps) {
+#pragma unroll
+        for (int d = 0; d < kDepth; ++d) {
+            const int n = n0 + d * kDecodeWarps;
+            if (n < c.n_rb) {
+                int rb;
+                const TileRt T = batch_tile(c, n, rb);
+                consume_rb(buf[d], T, rb, Bc, S);
+                prefetch_rb(c, n + kPrefetchDepth * kDecodeWarps);
+                const int nn = n + kDepth * kDecodeWarps;
+                if (nn < c.n_rb) {
+                    int rb2;
+                    const TileRt T2 = batch_tile(c, nn, rb2);
+                    load_rb(T2, rb2, buf[d]);
+                }
+            }
+        }
+    }
+}
+
+// Collect the next batch at c.u and load this thread's scale elements.
+// Reads only plan data and weights.
+__device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args,
+                                            const LbJob* jobs_g, Cursor& c) {
+    c.nt = 0;
+    c.n_rb = 0;
+    c.pf0 = 0;
 #pragma unroll
     for (int k = 0; k < kMaxTiles; ++k) {
-        b.sc[k] = 0.0f;
-        if (k < b.nt) {
-            const LbJob& J = sm.jobs[b.t[k].job];
-            const int col = b.t[k].slice * kSliceElems + (int)threadIdx.x;
-            if (col < J.cols) b.sc[k] = __half2float(__ldg(J.vscale + col));
+        c.sc[k] = 0u;
+        if (c.u + c.n_rb < c.u_end) {
+            c.t[k] = next_tile(sm.jobs, sm.phase->n_jobs, c.j, c.u + c.n_rb, c.u_end);
+            c.nt = k + 1;
+            const Tile& t = c.t[k];
+            const LbJob& J = sm.jobs[t.job];
+            TileRt& T = c.rt[k];
+            T.P = J.P + (size_t)t.slice * kSliceWords;
+            T.h = J.oscale;
+            T.out = resolve(J.out, args);
+            T.ldw = J.ldw;
+            T.rows = J.rows;
+            T.wrem = min(kSliceWords, (J.cols + 31) / 32 - t.slice * kSliceWords);
+            T.rb0 = t.rb0;
+            T.nrb = t.nrb;
+            T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
+            T.tmap = J.use_tma ? &jobs_g[sm.phase->job_begin + t.job].tmap : nullptr;
+            T.x = t.slice * kSliceWords;
+            c.n_rb += t.nrb;
+            const int col = t.slice * kSliceElems + (int)threadIdx.x;
+            if (col < J.cols) c.sc[k] = __ldg(reinterpret_cast<const unsigned short*>(J.vscale) + col);
         }
     }
 }
 
 // Stage the batch's vector slices into shared memory (zero past cols): all
 // source loads are issued before any is used, so the batch costs one round
-// trip to L2.  The owner of a slice (the CTA holding its first rowblock) also
+// trip to L2, and L2 prefetches for this warp's first rowblocks of the batch
+// follow them.  The owner of a slice (the CTA holding its first rowblock) also
 // seeds the residual and adds the slice's sum of squares for RMSNorm; only
 // the first job of a phase carries acc_sumsq, so there is one sum per batch.
-__device__ void stage_batch(const Smem& sm, const CallArgs& args, const Batch& b) {
+// Ends with a CTA barrier.
+__device__ __forceinline__ void stage_batch(const Smem& sm, const CallArgs& args, const Cursor& c) {
+    static_assert(kSliceElems == kDecodeThreads, "one slice element per thread");
     const int e = threadIdx.x;
     float a[kMaxTiles], a2[kMaxTiles], nrm[kMaxTiles];
 #pragma unroll
@@ -518,32 +558,36 @@ __device__ void stage_batch(const Smem& sm, const CallArgs& args, const Batch& b
         a[k] = 0.0f;
         a2[k] = 0.0f;
         nrm[k] = -1.0f;
-        if (k < b.nt) {
-            const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
-            const int col = b.t[k].slice * kSliceElems + e;
-            if (col < J.cols) load_src(J, col, a[k], a2[k]);
+        if (k < c.nt) {
+            const LbJob& J = sm.jobs[c.t[k].job];
+            const int col = c.t[k].slice * kSliceElems + e;
+            if (col < J.cols) load_src(J, resolve(J.src, args), col, a[k], a2[k]);
             if (J.kind == VK_T && J.norm_sumsq != nullptr) nrm[k] = __ldcg(J.norm_sumsq);
         }
     }
+    // the batch's first rowblocks head for L2 behind the (latency-critical) source loads
+    batch_prefetch(c, c.pf0, kPrefetchDepth);
     float sq = 0.0f;
     float* acc = nullptr;
 #pragma unroll
     for (int k = 0; k < kMaxTiles; ++k) {
-        if (k >= b.nt) break;
-        const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
-        const int col = b.t[k].slice * kSliceElems + e;
+        if (k >= c.nt) break;
+        const LbJob& J = sm.jobs[c.t[k].job];
+        const int col = c.t[k].slice * kSliceElems + e;
+        const bool owner = c.t[k].rb0 == 0;
         float v = 0.0f;
         if (col < J.cols) {
             const float raw = J.kind == VK_SILU_MUL ? silu(a[k]) * a2[k] : a[k];
             const float rs = nrm[k] >= 0.0f ? rsqrtf(nrm[k] / (float)J.norm_n + kRmsEps) : 1.0f;
-            v = b.sc[k] * (raw * rs);
-            if (b.t[k].rb0 == 0) {
+            v = __half2float(__ushort_as_half(c.sc[k])) * (raw * rs);
+            if (owner) {
                 if (J.acc_sumsq != nullptr) sq += raw * raw;
-                if (J.resid_init != nullptr) J.resid_init[col] = raw;
+                float* ri = resolve(J.resid_init, args);
+                if (ri != nullptr) ri[col] = raw;
             }
         }
-        if (b.t[k].rb0 == 0 && J.acc_sumsq != nullptr) acc = J.acc_sumsq;
-        sm.vec[k * kVecPad + e + (e >> 5)] = v;
+        if (owner && J.acc_sumsq != nullptr) acc = J.acc_sumsq;
+        sm.vec[k * kVecPad + vpad(e)] = v;
     }
     if (acc != nullptr) {
 #pragma unroll
@@ -558,124 +602,100 @@ __device__ void stage_batch(const Smem& sm, const CallArgs& args, const Batch& b
     }
 }
 
-// The part of a phase that does not depend on earlier phases, run before the
-// grid-wide wait: this CTA's unit range and its first batch (rows in flight,
-// scales loaded).  sm.phase / sm.jobs must hold the phase.
-__device__ void phase_begin(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
-                            const int* splits, uint32_t ring_it, Cursor& c) {
-    const LbPhase& ph = *sm.phase;
-    c.u = unit_split(ph, splits, blockIdx.x, gridDim.x);
-    c.u_end = unit_split(ph, splits, blockIdx.x + 1, gridDim.x);
+// The part of a phase that does not depend on earlier phases: this CTA's
+// unit range and its first batch.  sm.phase / sm.jobs must hold the phase.
+__device__ __forceinline__ void phase_begin(const Smem& sm, const CallArgs& args,
+                                            const LbJob* jobs_g, Cursor& c) {
+    unit_range(sm, c.u, c.u_end);
     c.j = 0;
-    c.in_flight = 0;
-    c.b.nt = 0;
-    if (c.u < c.u_end) batch_begin(sm, args, jobs_g, ring_it, c);
-}
-
-// Wait (bounded) for the ring entries a cursor has in flight, before leaving
-// the kernel early: no copy may still be writing this CTA's shared memory.
-__device__ void drain_ring(const Smem& sm, const Cursor& c, uint32_t ring_it, int* err) {
-    for (int d = 0; d < c.in_flight; ++d) tma_wait(sm, ring_it + d, err);
-    cp_async_wait<0>();
+    c.nt = 0;
+    c.n_rb = 0;
+    if (c.u < c.u_end) batch_begin(sm, args, jobs_g, c);
 }
 
 // The rest of the phase, after the grid-wide wait.
-__device__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g, Cursor& c,
-                          uint32_t& ring_it, int* err) {
+__device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
+                                          Cursor& c, RB (&buf)[kDepth],
+                          const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
     const int G = gridDim.x, cta = blockIdx.x;
-    const LbPhase ph = *sm.phase;
-    float* zp = resolve(ph.zero_ptr, args);
+    float* zp = resolve(sm.phase->zero_ptr, args);
+    const int zn = sm.phase->zero_n;
     if (zp != nullptr) {
-        for (int i = cta * kDecodeThreads + threadIdx.x; i < ph.zero_n; i += G * kDecodeThreads)
+        for (int i = cta * kDecodeThreads + threadIdx.x; i < zn; i += G * kDecodeThreads)
             zp[i] = 0.0f;
     }
-    bool first = true;
     while (c.u < c.u_end) {
-        if (!first) batch_begin(sm, args, jobs_g, ring_it, c);
-        first = false;
-        const Batch& b = c.b;
-        stage_batch(sm, args, b);
-        for (int k = 0; k < b.nt; ++k) {
-            const LbJob J = fetch_job(sm.jobs, b.t[k].job, args);
-            const LbJob* Jg = jobs_g + ph.job_begin + b.t[k].job;
-            if (k > 0) ring_prologue(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it);
-            build_lut(sm, sm.vec + k * kVecPad);
-            const bool b1024 = sm.lut == 1024u;
-            if (J.use_tma) {
-                if (b1024) lookup_rowblocks<1024u, true>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
-                else lookup_rowblocks<0u, true>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
-            } else {
-                if (b1024) lookup_rowblocks<1024u, false>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
-                else lookup_rowblocks<0u, false>(J, Jg, b.t[k].slice, b.t[k].rb0, b.t[k].nrb, sm, ring_it, err);
-            }
-            __syncthreads();
-            c.u += b.t[k].nrb;
-        }
-    }
-    c.in_flight = 0;
-}
-
-// L2 prefetch of the sign segments this CTA will read in phase ph (up to
-// kPrefetchSegments of them, in the order it will read them).
-__device__ void prefetch_phase(const LbPhase& ph, const LbJob* jobs, const int* splits) {
-    const int G = gridDim.x, cta = blockIdx.x;
-    int u = unit_split(ph, splits, cta, G);
-    const int u_end = unit_split(ph, splits, cta + 1, G);
-    int j = ph.job_begin;
-    const int j_end = ph.job_begin + ph.n_jobs;
-    int budget = kPrefetchSegments;
-    while (u < u_end && budget > 0) {
-        j = find_job(jobs, j, j_end, u);
-        const LbJob& J = jobs[j];
-        const int local = u - J.unit_begin;
-        const int s = local / J.n_rowblocks;
-        const int rb0 = local - s * J.n_rowblocks;
-        const int nrb = min(J.n_rowblocks - rb0, u_end - u);
-        const int rows = min(nrb * kRowBlock, budget);
-        for (int i = threadIdx.x; i < rows; i += kDecodeThreads)
-            prefetch_segment(J, s, rb0 * kRowBlock + i);
-        // the scales this tile will read: its slice of g or l, its rows of h
-        const int t = threadIdx.x - (kDecodeThreads - 32);          // last warp
-        if (t >= 0) {
-            const int c0 = s * kSliceElems, c1 = min(J.cols, c0 + kSliceElems);
-            if (t < 8 && c0 + 64 * t < c1) prefetch_l2(J.vscale + c0 + 64 * t);
-            if (J.oscale != nullptr) {
-                const int r0 = rb0 * kRowBlock, r1 = min(J.rows, (rb0 + nrb) * kRowBlock);
-                for (int r = r0 + 64 * (t - 8); t >= 8 && r < r1; r += 64 * 24)
-                    prefetch_l2(J.oscale + r);
-            }
-        }
-        budget -= rows;
-        u += nrb;
+        stage_batch(sm, args, c);
+        for (int k = 0; k < c.nt; ++k)
+            build_table(sm.vec + k * kVecPad, kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes);
+        batch_loads(c, buf);
+        __syncthreads();
+        batch_lookups(c, buf, Bc, S);
+        c.u += c.n_rb;
+        if (c.u < c.u_end) batch_begin(sm, args, jobs_g, c);
+        __syncthreads();
     }
 }
 
-__device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jobs,
-                            const int* splits, WsHeader* hdr, const CallArgs& args) {
-    const Smem sm = smem_layout();
+template <bool kAsyncPlan>
+__device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jobs,
+                                            const int* splits, WsHeader* hdr,
+                                            const CallArgs& args) {
+    Smem sm = smem_layout();
     const unsigned G = gridDim.x;
     if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) return;   // sticky after a timeout
-    if (threadIdx.x < kDecodeWarps * kRingSlots) mbar_init(sm.bars + 8u * threadIdx.x, 1u);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    cache_phase(phases, 0, jobs, sm);
+    // the tables must sit above the plan cache at their fixed addresses
+    if ((uint32_t)__cvta_generic_to_shared(dyn_smem()) + (uint32_t)kMiscBytes > kTableAddr0) {
+        if (threadIdx.x == 0) atomicExch(&hdr->error, (int)LB_ERR_UNSUPPORTED);
+        return;
+    }
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const int rho = lane >> 2, gam = lane & 3;
+    const uint32_t swap = (uint32_t)(rho >> 2);
+    uint32_t Bc[2][4], S[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t qbj = (uint32_t)((jj + rho) & 3);
+        S[jj] = 0x7604u | (qbj << 4);                    // [B.b0, word.byte qbj, B.b2, B.b3]
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh)
+            Bc[rh][jj] = (8u * (uint32_t)gam + 4u * ((uint32_t)rh ^ swap) + qbj) * 4u;
+    }
+    // The first two phases' plans are copied in by the whole CTA; each later
+    // one is fetched asynchronously by the last warp one phase ahead.
+    cache_plan(phases, 0, jobs, splits, 0);
+    if (n_phases > 1) cache_plan(phases, 1, jobs, splits, 1);
     __syncthreads();
-    uint32_t ring_it = 0;
     Cursor cur;
-    phase_begin(sm, args, jobs, splits, ring_it, cur);
-    prefetch_phase(phases[0], jobs, splits);
+    RB buf[kDepth];
+    phase_begin(sm, args, jobs, cur);
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args, jobs, cur, ring_it, &hdr->error);
+        run_phase(sm, args, jobs, cur, buf, Bc, S);
         if (p + 1 < n_phases) {
-            // Announce completion, then use the wait: bring in the next
-            // phase's plan, start its first rows streaming into the ring and
-            // prefetch the rest of this CTA's rows to L2.
+            // Announce completion, then use the wait: switch to the next
+            // phase's plan, load the scales of its first batch and fetch the
+            // plan of the phase after it into the buffer this phase used.
+            // Nothing bulky is in flight while the CTA waits: the wait and
+            // the staging loads after it are the latency-critical requests.
             grid_arrive(hdr);
-            cache_phase(phases, p + 1, jobs, sm);
+            if (wp == kDecodeWarps - 1) plan_wait();
             __syncthreads();
-            phase_begin(sm, args, jobs, splits, ring_it, cur);
-            prefetch_phase(phases[p + 1], jobs, splits);
+            const int nb = (p + 1) & 1;
+            use_plan_buf(sm, nb);
+            phase_begin(sm, args, jobs, cur);
+            if (cur.u < cur.u_end) {   // a little of the next phase heads for L2 during the wait
+                batch_prefetch(cur, 0, kEarlyPrefetch);
+                cur.pf0 = kEarlyPrefetch;
+            }
+            if (kAsyncPlan && wp == kDecodeWarps - 1 && p + 2 < n_phases)
+                cache_plan_async(phases, p + 2, sm.phase->next_job_begin, sm.phase->next_n_jobs,
+                                 jobs, splits, nb ^ 1);
+            if (!kAsyncPlan && p + 2 < n_phases) {   // (not reached: such plans have two phases)
+                __syncthreads();
+                cache_plan(phases, p + 2, jobs, splits, nb ^ 1);
+            }
             if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) {
-                drain_ring(sm, cur, ring_it, &hdr->error);
+                if (wp == kDecodeWarps - 1) plan_wait();
                 return;
             }
         }
@@ -696,7 +716,7 @@ __device__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jo
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 linear_program_kernel(const __grid_constant__ LinearPlan plan, int n_phases, WsHeader* hdr) {
     const CallArgs args = {nullptr, nullptr};
-    run_program(plan.phases, n_phases, plan.jobs, plan.split, hdr, args);
+    run_program<false>(plan.phases, n_phases, plan.jobs, plan.split, hdr, args);
 }
 
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
@@ -704,7 +724,7 @@ stack_program_kernel(const LbPhase* __restrict__ phases, const LbJob* __restrict
                      const int* __restrict__ splits, int n_phases, WsHeader* hdr, const void* x,
                      float* y) {
     const CallArgs args = {x, y};
-    run_program(phases, n_phases, jobs, splits, hdr, args);
+    run_program<true>(phases, n_phases, jobs, splits, hdr, args);
 }
 
 cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
@@ -728,7 +748,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw) {
+// 2-D tensor map of a packed sign matrix with 32-row x 16-word boxes (one
+// rowblock of one slice), used for L2 prefetches of whole rowblocks.
+bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw, int words) {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
     if (!tried) {
@@ -739,49 +761,70 @@ bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw) {
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<EncodeTiledFn>(p);
     }
-    if (!fn || rows <= 0 || ldw <= 0 || (ldw & 3) != 0) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)ldw, (cuuint64_t)rows};
+    if (!fn || rows <= 0 || ldw <= 0 || (ldw & 3) != 0 || words <= 0 || words > ldw) return false;
+    // the tensor's width is the words holding signs, so boxes stop before a padded pitch
+    const cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)ldw * 4};
     const cuuint32_t box[2] = {(cuuint32_t)kSliceWords, (cuuint32_t)kRowBlock};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(P), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+              CU_TENSOR_MAP_L2_PROMOTION_L2_64B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
 
 int decode_grid() { return device_sm_count() * kCtasPerSm; }
 
-// Contiguous unit ranges for G CTAs with the smallest largest cost.  The
-// warps of a CTA take a tile's rowblocks kDecodeWarps at a time, so a CTA
-// that takes k rowblocks of a tile spends ceil(k / kDecodeWarps) warp
-// iterations on them, plus kTileCost (in 1/kDecodeWarps iterations) to stage
-// the tile's vector and build its tables.  Units run job by job, slice-major
+// Contiguous unit ranges for G CTAs with the smallest largest cost.  A CTA
+// takes its tiles in batches of up to kTables; a batch costs kTileCost per
+// tile (vector stage + table build, in 1/kDecodeWarps warp iterations) plus
+// ceil(rowblocks / kDecodeWarps) warp iterations, since its warps take the
+// batch's rowblocks kDecodeWarps at a time.  Units run job by job, slice-major
 // inside a job, so a phase is a list of tiles of n_rowblocks units each; a
 // greedy fill is optimal for a given bound, which a bisection minimises.
 namespace {
 template <class F>
 void for_each_tile(const LbJob* jobs, int n_jobs, F f) {
     for (int j = 0; j < n_jobs; ++j)
-        for (int s = 0; s < jobs[j].n_slices; ++s) f(jobs[j].n_rowblocks);
+        for (int g0 = 0; g0 < jobs[j].n_rowblocks; g0 += jobs[j].rg)
+            for (int s = 0; s < jobs[j].n_slices; ++s)
+                f(std::min(jobs[j].rg, jobs[j].n_rowblocks - g0));
 }
-long long take_cost(long long k) {
-    return kTileCost + (k + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps;
+long long ceil_warps(long long k) { return (k + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps; }
+struct Fill {
+    long long closed;   // cost of the CTA's finished batches
+    int tiles;          // tiles in its open batch
+    long long rb;       // rowblocks in its open batch
+};
+// The CTA's state and cost once `take` rowblocks of a new tile join it.
+long long join(const Fill& f, long long take, Fill& g) {
+    g = f;
+    if (g.tiles == kTables) {
+        g.closed += g.tiles * kTileCost + ceil_warps(g.rb);
+        g.tiles = 0;
+        g.rb = 0;
+    }
+    g.tiles += 1;
+    g.rb += take;
+    return g.closed + g.tiles * kTileCost + ceil_warps(g.rb);
 }
 // CTAs a greedy fill under cost bound T needs; boundaries go to `out` if set.
 int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
     int used = 1, u = 0;
-    long long cost = 0;
+    Fill f = {0, 0, 0};
     for_each_tile(jobs, n_jobs, [&](int n) {
         while (n > 0) {
-            if (cost + take_cost(1) > T) {
+            Fill g;
+            if (join(f, 1, g) > T) {
                 if (out) out[used] = u;
                 ++used;
-                cost = 0;
+                f = Fill{0, 0, 0};
             }
-            const long long room = (T - cost - kTileCost) / kDecodeWarps * kDecodeWarps;
-            const int take = (int)std::min<long long>(n, room);
-            cost += take_cost(take);
+            join(f, 0, g);
+            const long long room =
+                (T - g.closed - g.tiles * kTileCost) / kDecodeWarps * kDecodeWarps - g.rb;
+            const int take = (int)std::max<long long>(1, std::min<long long>(n, room));
+            join(f, take, f);
             n -= take;
             u += take;
         }
@@ -790,9 +833,25 @@ int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
 }
 }  // namespace
 
+// A job gets about as many row groups as the CTAs its share of the phase's
+// units would occupy, divided by its slices, so that a CTA's range is
+// usually one tile and the n_slices CTAs of a group read the same rows.
+void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G) {
+    for (int j = 0; j < n_jobs; ++j) {
+        LbJob& J = jobs[j];
+        const double ctas = (double)G * (double)(J.n_slices * J.n_rowblocks) / (double)n_units;
+        const int groups = std::max(1, (int)(ctas / J.n_slices + 0.5));
+        J.rg = (J.n_rowblocks + groups - 1) / groups;
+    }
+}
+
 void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out) {
-    long long lo = take_cost(1), hi = lo;
-    for_each_tile(jobs, n_jobs, [&](int n) { hi += take_cost(n); });
+    long long lo = kTileCost + kDecodeWarps, hi = lo;
+    {
+        Fill f = {0, 0, 0};
+        for_each_tile(jobs, n_jobs, [&](int n) { hi = join(f, n, f); });
+        hi = std::max(hi, lo);
+    }
     while (lo < hi) {   // smallest bound a fill of at most G CTAs meets
         const long long mid = (lo + hi) / 2;
         if (greedy_fill(jobs, n_jobs, mid, nullptr) <= G) hi = mid;
@@ -804,20 +863,14 @@ void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out)
 }
 
 cudaError_t decode_configure() {
-    cudaError_t e = cudaFuncSetAttribute(linear_program_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kDecodeSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(stack_program_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kDecodeSmem);
-    if (e != cudaSuccess) return e;
     for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
                            reinterpret_cast<const void*>(stack_program_kernel)}) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kDecodeSmem);
+        if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-    }
-    for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
-                           reinterpret_cast<const void*>(stack_program_kernel)}) {
         int nb = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kDecodeThreads, kDecodeSmem);
         if (e != cudaSuccess) return e;

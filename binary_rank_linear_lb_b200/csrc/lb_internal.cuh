@@ -24,13 +24,14 @@ constexpr int kCtasPerSm = 1;
 constexpr int kSliceElems = 512;             // columns covered by one lookup table
 constexpr int kSliceWords = kSliceElems / 32;
 constexpr int kRowBlock = 32;                // rows per warp work item (4 steps x 8 rows)
-constexpr int kLutBytes = 64 * 1024;         // 64 chunks x 256 entries x fp32
-constexpr int kVecPad = kSliceElems + kSliceElems / 32;   // staged slice, padded
-constexpr int kRingDepth = 3;                // rowblocks each warp has in flight
-constexpr int kRingSlots = kRingDepth + 1;
+constexpr int kLutBytes = 64 * 1024;         // one table: 64 chunks x 256 entries x fp32
+constexpr int kTables = 2;                   // tables resident at once (a batch of <= 2 tiles)
+// Tables sit at shared-window addresses kTableAddr0 + t * 64 KB, so the table
+// of a lookup is selected by bits 16-17 of the address (see lb_decode.cu).
+constexpr uint32_t kTableAddr0 = 64u * 1024u;
+constexpr int kVecPad = kSliceElems + kSliceElems / 16;   // staged slice, 4 floats of pad per 64
+constexpr int kDepth = 2;                    // rowblocks each warp has in flight (registers)
 constexpr int kRowBlockBytes = kRowBlock * kSliceWords * 4;   // 2 KB of signs
-constexpr int kRingSlotBytes = kRowBlockBytes + 128;          // + the lanes' row scales (128-aligned)
-constexpr int kRingBytes = kDecodeWarps * kRingSlots * kRingSlotBytes;   // 130 KB
 constexpr int kMaxLinearJobs = 16;           // per phase in a single-linear call
 constexpr int kMaxPhaseJobs = 16;            // jobs of one phase (stack phases use <= 6)
 constexpr int kMaxDecodeM = 8;               // rows of x the decode path takes at once
@@ -56,7 +57,7 @@ enum VecKind : int {
 };
 
 struct alignas(64) LbJob {
-    CUtensorMap tmap;         // 2-D TMA descriptor of P (32-row x 16-word boxes), if use_tma
+    CUtensorMap tmap;         // 2-D TMA descriptor of P (32-row x 16-word boxes) for L2 prefetch, if use_tma
     const uint32_t* P;        // packed rows [rows][ldw] (ldw = row pitch in words)
     const void* src;          // vector source
     const float* src2;        // second source (VK_SILU_MUL)
@@ -68,28 +69,39 @@ struct alignas(64) LbJob {
     float* resid_init;        // owner of a slice writes float(src) of the slice here
     int rows, cols, ldw, kind;
     int n_slices, n_rowblocks, unit_begin, norm_n;
-    int gqa_ghd, gqa_hd, use_tma, pad1;
+    int gqa_ghd, gqa_hd, use_tma;
+    int rg;                   // rowblocks per row group (units run group, slice, rowblock)
 };
 
-struct LbPhase {
+struct alignas(16) LbPhase {
     int job_begin, n_jobs, n_units, zero_n;
     float* zero_ptr;          // if set, the CTAs zero zero_n floats here during the phase
     int split_off;            // offset of this phase's split_g+1 unit boundaries in the split table
     int split_g;              // CTAs the split was made for (-1 or another grid: even split)
+    int next_job_begin;       // jobs of the following phase (0 / 0 for the last phase), so a
+    int next_n_jobs;          // CTA can fetch that phase's plan without reading its header first
+    int pad[2];
 };
+static_assert(sizeof(LbPhase) == 48, "LbPhase is copied in 16-byte pieces");
 
 // Stack plans are prepared once and reused with different x / y buffers, so
 // job pointers that mean "the call's x" or "the call's y" are stored as tags.
 #define LB_TAG_X ((const void*)1)
 #define LB_TAG_Y ((const void*)2)
 
-constexpr int kDecodeSmem = kLutBytes + kRingBytes + 4 * 4 * kVecPad + 4 * 32 + 64 + 64 +
-                            kMaxPhaseJobs * (int)sizeof(LbJob) + 8 * kDecodeWarps * kRingSlots;
+// Dynamic shared memory: everything below the first table (staged vectors,
+// reduction scratch, the phase plan) starts at the window's dynamic base
+// (1 KB on sm_100) and must end below kTableAddr0; the size requested covers
+// the tables for any base below that.
+constexpr int kMiscBytes = 4 * kTables * kVecPad + 4 * 32 + 64 +
+                           2 * (64 + kMaxPhaseJobs * (int)sizeof(LbJob));
+constexpr int kDecodeSmem = (int)kTableAddr0 + kTables * kLutBytes;
 static_assert(kDecodeSmem <= 227 * 1024, "decode kernel shared memory over the per-CTA limit");
+static_assert(kMiscBytes + 1024 <= (int)kTableAddr0, "decode plan cache overlaps the tables");
 
 // Plan of a single linear call, passed by value as a kernel parameter.
 constexpr int kMaxGrid = 256;                // CTAs a split table has room for
-constexpr int kTileCost = 40;                // vector stage + table build, in 1/16 warp iterations
+constexpr int kTileCost = 12;                // vector stage + table build, in 1/16 warp iterations
 
 struct LinearPlan {
     LbJob jobs[2 * kMaxLinearJobs];
@@ -111,6 +123,10 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {
 }
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" :: "l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
@@ -179,6 +195,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%3, %4}], [%2];"
         :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
 }
+// L2 prefetch of one box of a 2-D tensor map (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 :: "l"(map), "r"(x), "r"(y) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -187,8 +208,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 int device_sm_count();               // SMs of the current device (cached per device)
 bool device_is_sm100();
 cudaError_t decode_configure();      // one-time kernel attribute setup per device
-// 2-D TMA descriptor of a packed sign matrix (rows x ldw words, 16-byte pitch).
-bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw);
+// 2-D TMA descriptor of a packed sign matrix: rows x `words` words holding
+// signs, row pitch ldw words (a multiple of 4).
+bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw, int words);
 
 // Decode phase program launches (lb_decode.cu).
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,
@@ -197,6 +219,8 @@ cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const in
                               int n_phases, WsHeader* hdr, const void* x, float* y,
                               cudaStream_t s);
 int decode_grid();                   // CTAs of a decode launch on the current device
+// Row-group sizes of a phase's jobs for a grid of G CTAs.
+void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G);
 // Cost-balanced contiguous unit ranges for the G CTAs of a phase (out: G+1 boundaries).
 void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
 

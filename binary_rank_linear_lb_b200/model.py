@@ -2,8 +2,8 @@
 
 Each branch is generated from its own seeds (``synth``) and binarised on the GPU
 with ``lb_pack_signs``; the fp32 latents are dropped right after packing.  Rows
-are packed with a 16-byte pitch (``ld_words`` a multiple of 4, zero padding),
-which lets the decode kernels stream them with TMA.
+are packed with a 64-byte pitch (``ld_words`` a multiple of 16, zero padding),
+so the decode kernels stream aligned 64-byte row pieces.
 
 ``signs="bits"`` instead draws the packed words directly from a uniform bit
 source.  The signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so the
@@ -22,9 +22,14 @@ from .configs import Model, proj_shape
 
 
 def padded_words(k: int, pad: bool = True) -> int:
-    """Words per packed row of k signs: ceil(k/32), rounded up to a multiple of 4 if pad."""
+    """Words per packed row of k signs: ceil(k/32), rounded up to a multiple of 16 if pad.
+
+    A 64-byte pitch puts every 512-column slice of every row in one aligned
+    64-byte piece of memory, the DRAM access unit; the kernels never read the
+    padding, so the bytes streamed stay the packed signs themselves.
+    """
     w = (k + 31) // 32
-    return (w + 3) // 4 * 4 if pad else w
+    return (w + 15) // 16 * 16 if pad else w
 
 
 def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int, branch: int,
