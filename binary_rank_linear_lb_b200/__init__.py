@@ -38,10 +38,15 @@ class LbError(RuntimeError):
         super().__init__(f"{what} failed: {status_string(status)}")
 
 
+LB_LAYOUT_ROWS, LB_LAYOUT_SLICES = 0, 1
+LAYOUTS = {"rows": LB_LAYOUT_ROWS, "slices": LB_LAYOUT_SLICES}
+
+
 class lb_branch(ctypes.Structure):
     _fields_ = [("Vp", ctypes.c_void_p), ("Up", ctypes.c_void_p), ("h", ctypes.c_void_p),
                 ("g", ctypes.c_void_p), ("l", ctypes.c_void_p), ("ld_v", ctypes.c_int64),
-                ("ld_u", ctypes.c_int64)]
+                ("ld_u", ctypes.c_int64), ("layout", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class lb_stack_desc(ctypes.Structure):
@@ -55,7 +60,7 @@ EXPORTS = ("lb_status_string", "lb_version", "lb_pack_signs", "lb_linear_forward
            "lb_linear_workspace_size", "lb_linear_path", "lb_stack_workspace_size",
            "lb_stack_prepare", "lb_stack_forward", "lb_stack_forward_host",
            "lb_workspace_status", "lb_stack_output", "lb_linear_forward_noalloc",
-           "lb_noalloc_scratch_bytes")
+           "lb_noalloc_scratch_bytes", "lb_pack_signs_sliced", "lb_packed_words")
 
 _lib = None
 
@@ -74,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.lb_version.restype = ctypes.c_int
         L.lb_pack_signs.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, i64, vp]
         L.lb_pack_signs.restype = st
+        L.lb_pack_signs_sliced.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp]
+        L.lb_pack_signs_sliced.restype = st
+        L.lb_packed_words.argtypes = [i64, i64, ctypes.c_int, i64]
+        L.lb_packed_words.restype = sz
         L.lb_linear_forward.argtypes = [vp, st, i64, i64, i64, i64, vp, ctypes.c_int, vp, vp,
                                         sz, vp]
         L.lb_linear_forward.restype = st
@@ -121,37 +130,87 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 # ------------------------------------------------------------------ packing
+def packed_words(n: int, k: int, layout: int = LB_LAYOUT_ROWS, ld_words: int = 0) -> int:
+    """Words a packed matrix of n rows of k signs occupies (lb_packed_words)."""
+    return int(lib().lb_packed_words(n, k, int(layout), int(ld_words)))
+
+
 def pack_signs(latent: torch.Tensor, axis: int, ld_words: Optional[int] = None,
-               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               out: Optional[torch.Tensor] = None, stream=None,
+               layout: int = LB_LAYOUT_ROWS) -> torch.Tensor:
     """Packed sign words (int32 storage of uint32 words) of an fp32 latent.
 
-    axis=1: [rows][ceil(cols/32)] (U: out x r);  axis=0: [cols][ceil(rows/32)] (V: in x r).
+    axis=1: n = rows packed rows of k = cols signs (U: out x r); axis=0: n = cols
+    packed rows of k = rows signs (V: in x r).  LB_LAYOUT_ROWS gives [n][ld_words]
+    (default ceil(k/32)); LB_LAYOUT_SLICES gives the sliced layout as a flat tensor
+    of packed_words(n, k, LB_LAYOUT_SLICES) words.
     """
     rows, cols = latent.shape
     k = cols if axis == 1 else rows
     n = rows if axis == 1 else cols
-    ldw = (k + 31) // 32 if ld_words is None else int(ld_words)
-    if out is None:
-        out = torch.empty((n, ldw), dtype=torch.int32, device=latent.device)
     ld = latent.stride(0) if latent.dim() == 2 else cols
     if latent.stride(-1) != 1:
         raise ValueError("latent must have unit stride along its columns")
+    if layout == LB_LAYOUT_SLICES:
+        if out is None:
+            out = torch.empty(packed_words(n, k, LB_LAYOUT_SLICES), dtype=torch.int32,
+                              device=latent.device)
+        _check(lib().lb_pack_signs_sliced(_ptr(latent), rows, cols, ld, int(axis), _ptr(out),
+                                          _stream(stream)), "lb_pack_signs_sliced")
+        return out
+    ldw = (k + 31) // 32 if ld_words is None else int(ld_words)
+    if out is None:
+        out = torch.empty((n, ldw), dtype=torch.int32, device=latent.device)
     _check(lib().lb_pack_signs(_ptr(latent), rows, cols, ld, int(axis), _ptr(out), ldw,
                                _stream(stream)), "lb_pack_signs")
     return out
 
 
+def _slice_pitch(nw: int, s: int) -> int:
+    last = (nw - 1) // 16
+    return 16 if s < last else (nw - 16 * last + 3) // 4 * 4
+
+
+def slice_words(words: torch.Tensor, k: int) -> torch.Tensor:
+    """Row-major packed words [n][>= ceil(k/32)] regrouped into LB_LAYOUT_SLICES (flat)."""
+    n, nw = words.shape[0], (k + 31) // 32
+    blocks = []
+    for s in range((nw + 15) // 16):
+        w = words[:, 16 * s:min(16 * s + 16, nw)]
+        pitch = _slice_pitch(nw, s)
+        if w.shape[1] < pitch:
+            w = torch.cat([w, torch.zeros((n, pitch - w.shape[1]), dtype=w.dtype,
+                                          device=w.device)], dim=1)
+        blocks.append(w.reshape(-1))
+    return torch.cat(blocks).contiguous()
+
+
+def unslice_words(flat: torch.Tensor, n: int, k: int) -> torch.Tensor:
+    """Inverse of slice_words: [n][ceil(k/32)] row-major words of a sliced matrix."""
+    nw = (k + 31) // 32
+    cols, off = [], 0
+    for s in range((nw + 15) // 16):
+        pitch = _slice_pitch(nw, s)
+        block = flat[off:off + n * pitch].reshape(n, pitch)
+        cols.append(block[:, :min(16, nw - 16 * s)])
+        off += n * pitch
+    return torch.cat(cols, dim=1)
+
+
 # ------------------------------------------------------------------ one linear
 class Branch:
-    """Device tensors of one branch: packed signs and FP16 scales."""
+    """Device tensors of one branch: packed signs (in `layout`) and FP16 scales."""
 
     def __init__(self, Vp: torch.Tensor, Up: torch.Tensor, h: torch.Tensor, g: torch.Tensor,
-                 l: torch.Tensor):
+                 l: torch.Tensor, layout: int = LB_LAYOUT_ROWS):
         self.Vp, self.Up, self.h, self.g, self.l = Vp, Up, h, g, l
+        self.layout = layout
 
     def c_struct(self) -> lb_branch:
+        rows = self.layout == LB_LAYOUT_ROWS
         return lb_branch(_ptr(self.Vp), _ptr(self.Up), _ptr(self.h), _ptr(self.g), _ptr(self.l),
-                         self.Vp.shape[1], self.Up.shape[1])
+                         self.Vp.shape[1] if rows else 0, self.Up.shape[1] if rows else 0,
+                         self.layout, 0)
 
     @property
     def nbytes(self) -> int:

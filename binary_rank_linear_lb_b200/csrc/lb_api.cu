@@ -59,15 +59,16 @@ int vec_kind_for(lb_dtype t) {
 // Fill the size fields of a job whose matrix has `rows` packed rows of `cols`
 // signs with a pitch of `ld` words (0: unpadded), and its TMA descriptor when
 // the pitch allows one (16-byte rows).
-void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld) {
+void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld, int layout) {
     J.rows = (int)rows;
     J.cols = (int)cols;
-    J.ldw = (int)(ld ? ld : cdiv(cols, 32));
+    J.sliced = layout == LB_LAYOUT_SLICES ? 1 : 0;
+    J.ldw = J.sliced ? kSliceWords : (int)(ld ? ld : cdiv(cols, 32));
     J.n_slices = (int)cdiv(cols, kSliceElems);
     J.n_rowblocks = (int)cdiv(rows, kRowBlock);
     J.rg = J.n_rowblocks;
-    J.use_tma = 0;
-    if ((J.ldw & 3) == 0 && (reinterpret_cast<uintptr_t>(J.P) & 15) == 0)
+    J.use_tma = 0;   // sliced rows are contiguous per slice: plain bulk prefetches serve them
+    if (!J.sliced && (J.ldw & 3) == 0 && (reinterpret_cast<uintptr_t>(J.P) & 15) == 0)
         J.use_tma = make_sign_tmap(&J.tmap, J.P, J.rows, J.ldw, (int)cdiv(cols, 32)) ? 1 : 0;
 }
 
@@ -100,7 +101,9 @@ void add_job(LbPhase& ph, std::vector<LbJob>& jobs, LbJob J) {
 }
 
 bool branch_ok(const lb_branch& b) {
-    return b.Vp && b.Up && b.h && b.g && b.l && b.ld_v >= 0 && b.ld_u >= 0;
+    if (!(b.Vp && b.Up && b.h && b.g && b.l && b.ld_v >= 0 && b.ld_u >= 0)) return false;
+    if (b.layout == LB_LAYOUT_SLICES) return b.ld_v == 0 && b.ld_u == 0;
+    return b.layout == LB_LAYOUT_ROWS;
 }
 bool branch_aligned(const lb_branch& b) {
     return aligned(b.Vp, 16) && aligned(b.Up, 16) && aligned(b.h, 4) && aligned(b.g, 2) &&
@@ -278,7 +281,7 @@ void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
                     LbJob J = {};
                     if (ps.first) {
                         J.P = br(l, p, b).Vp;
-                        set_job_shape(J, r, in, br(l, p, b).ld_v);
+                        set_job_shape(J, r, in, br(l, p, b).ld_v, br(l, p, b).layout);
                         J.vscale = reinterpret_cast<const __half*>(br(l, p, b).g);
                         J.out = tptr(l, p, b);
                         if (p == LB_O) {
@@ -302,7 +305,7 @@ void build_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws,
                         if (first_job && norm) J.acc_sumsq = norm;
                     } else {
                         J.P = br(l, p, b).Up;
-                        set_job_shape(J, out, r, br(l, p, b).ld_u);
+                        set_job_shape(J, out, r, br(l, p, b).ld_u, br(l, p, b).layout);
                         J.kind = VK_T;
                         J.src = tptr(l, p, b);
                         J.vscale = reinterpret_cast<const __half*>(br(l, p, b).l);
@@ -375,7 +378,28 @@ lb_status lb_pack_signs(const float* latent, int64_t rows, int64_t cols, int64_t
     if (!aligned(latent, 4) || !aligned(packed, 4)) return LB_ERR_ALIGNMENT;
     const lb_status st = ensure_device();
     if (st != LB_OK) return st;
-    return launch_pack(latent, rows, cols, ld, axis, packed, ld_words,
+    return launch_pack(latent, rows, cols, ld, axis, packed, ld_words, false,
+                       static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? LB_OK
+               : LB_ERR_CUDA;
+}
+
+size_t lb_packed_words(int64_t n, int64_t k, int layout, int64_t ld_words) {
+    if (n <= 0 || k <= 0 || n > ((int64_t)1 << 40) || k > ((int64_t)1 << 40)) return 0;
+    const int64_t nw = cdiv(k, 32);
+    if (layout == LB_LAYOUT_SLICES) return (size_t)sliced_words(n, nw);
+    if (layout != LB_LAYOUT_ROWS || (ld_words != 0 && ld_words < nw)) return 0;
+    return (size_t)(n * (ld_words ? ld_words : nw));
+}
+
+lb_status lb_pack_signs_sliced(const float* latent, int64_t rows, int64_t cols, int64_t ld,
+                               int axis, uint32_t* packed, void* stream) {
+    if (!latent || !packed || rows <= 0 || cols <= 0 || ld < cols) return LB_ERR_INVALID_ARG;
+    if (axis != 0 && axis != 1) return LB_ERR_INVALID_ARG;
+    if (!aligned(latent, 4) || !aligned(packed, 16)) return LB_ERR_ALIGNMENT;
+    const lb_status st = ensure_device();
+    if (st != LB_OK) return st;
+    return launch_pack(latent, rows, cols, ld, axis, packed, 0, true,
                        static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? LB_OK
                : LB_ERR_CUDA;
@@ -421,8 +445,10 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
         // the tensor-core path reads g in 16-byte vectors and sign words in pairs
         bool ok = true;
         for (int b = 0; b < n_branches; ++b)
-            ok = ok && aligned(br[b].g, 16) && ((br[b].ld_v ? br[b].ld_v : cdiv(in, 32)) & 1) == 0 &&
-                 ((br[b].ld_u ? br[b].ld_u : cdiv(r, 32)) & 1) == 0;
+            ok = ok && aligned(br[b].g, 16) &&
+                 (br[b].layout == LB_LAYOUT_SLICES ||
+                  (((br[b].ld_v ? br[b].ld_v : cdiv(in, 32)) & 1) == 0 &&
+                   ((br[b].ld_u ? br[b].ld_u : cdiv(r, 32)) & 1) == 0));
         if (ok)
             return launch_prefill(x, vec_kind_for(x_dtype), M, in, out, r, br, n_branches, y,
                                   workspace, s) == cudaSuccess
@@ -444,7 +470,7 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
             for (int b = 0; b < n_branches; ++b) {
                 LbJob J = {};
                 J.P = br[b].Vp;
-                set_job_shape(J, r, in, br[b].ld_v);
+                set_job_shape(J, r, in, br[b].ld_v, br[b].layout);
                 J.kind = vec_kind_for(x_dtype);
                 J.src = static_cast<const char*>(x) + (size_t)(m0 + m) * (size_t)in * xsz;
                 J.vscale = reinterpret_cast<const __half*>(br[b].g);
@@ -459,7 +485,7 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
             for (int b = 0; b < n_branches; ++b) {
                 LbJob J = {};
                 J.P = br[b].Up;
-                set_job_shape(J, out, r, br[b].ld_u);
+                set_job_shape(J, out, r, br[b].ld_u, br[b].layout);
                 J.kind = VK_T;
                 J.src = t + ((size_t)m * n_branches + b) * (size_t)r;
                 J.vscale = reinterpret_cast<const __half*>(br[b].l);

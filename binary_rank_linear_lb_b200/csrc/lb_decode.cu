@@ -297,8 +297,9 @@ struct TileRt {
     int ldw, rows, wrem;     // row pitch, rows, words of the slice holding signs (<= 16)
     int rb0, nrb;
     uint32_t tb;             // table address bits (kTableAddr0 + t * 64 KB)
-    const CUtensorMap* tmap; // the job's tensor map (in the plan), or nullptr: no L2 prefetch
+    const CUtensorMap* tmap; // the job's tensor map (in the plan) for L2 prefetch, or nullptr
     int x;                   // the slice's first word (tensor-map coordinate)
+    int bulk;                // rows of the slice are contiguous: prefetch a rowblock as one range
 };
 
 // This CTA's place in a phase and the batch about to run.  sc[k] is this
@@ -444,6 +445,7 @@ __device__ __forceinline__ TileRt batch_tile(const Cursor& c, int n, int& rb) {
     T.tb = k ? c.rt[1].tb : c.rt[0].tb;
     T.tmap = k ? c.rt[1].tmap : c.rt[0].tmap;
     T.x = k ? c.rt[1].x : c.rt[0].x;
+    T.bulk = k ? c.rt[1].bulk : c.rt[0].bulk;
     rb = T.rb0 + (k ? n - c.rt[0].nrb : n);
     return T;
 }
@@ -454,7 +456,12 @@ __device__ __forceinline__ void prefetch_rb(const Cursor& c, int n) {
     if ((threadIdx.x & 31) == 0 && n < c.n_rb) {
         int rb;
         const TileRt T = batch_tile(c, n, rb);
-        if (T.tmap != nullptr) tma_prefetch_2d(T.tmap, T.x, rb * kRowBlock);
+        if (T.tmap != nullptr) {
+            tma_prefetch_2d(T.tmap, T.x, rb * kRowBlock);
+        } else if (T.bulk) {   // rows rb*32 .. of the slice block, 16-byte multiple
+            const int nrow = min(kRowBlock, T.rows - rb * kRowBlock);
+            bulk_prefetch_l2(T.P + (size_t)rb * kRowBlock * T.ldw, (uint32_t)(nrow * T.ldw * 4));
+        }
     }
 }
 
@@ -524,17 +531,24 @@ __device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args
             const Tile& t = c.t[k];
             const LbJob& J = sm.jobs[t.job];
             TileRt& T = c.rt[k];
-            T.P = J.P + (size_t)t.slice * kSliceWords;
+            const int nw = (J.cols + 31) / 32;
+            if (J.sliced) {   // the slice is a contiguous block of rows
+                T.P = J.P + (size_t)kSliceWords * (size_t)J.rows * (size_t)t.slice;
+                T.ldw = (int)sliced_pitch(nw, t.slice);
+            } else {
+                T.P = J.P + (size_t)t.slice * kSliceWords;
+                T.ldw = J.ldw;
+            }
             T.h = J.oscale;
             T.out = resolve(J.out, args);
-            T.ldw = J.ldw;
             T.rows = J.rows;
-            T.wrem = min(kSliceWords, (J.cols + 31) / 32 - t.slice * kSliceWords);
+            T.wrem = min(kSliceWords, nw - t.slice * kSliceWords);
             T.rb0 = t.rb0;
             T.nrb = t.nrb;
             T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
             T.tmap = J.use_tma ? &jobs_g[sm.phase->job_begin + t.job].tmap : nullptr;
             T.x = t.slice * kSliceWords;
+            T.bulk = J.sliced;
             c.n_rb += t.nrb;
             const int col = t.slice * kSliceElems + (int)threadIdx.x;
             if (col < J.cols) c.sc[k] = __ldg(reinterpret_cast<const unsigned short*>(J.vscale) + col);

@@ -71,6 +71,7 @@ struct alignas(64) LbJob {
     int n_slices, n_rowblocks, unit_begin, norm_n;
     int gqa_ghd, gqa_hd, use_tma;
     int rg;                   // rowblocks per row group (units run group, slice, rowblock)
+    int sliced;               // P is in the sliced layout (LB_LAYOUT_SLICES), ldw unused
 };
 
 struct alignas(16) LbPhase {
@@ -108,6 +109,25 @@ struct LinearPlan {
     LbPhase phases[2];
     int split[2 * (kMaxGrid + 1)];           // per-phase unit boundaries of the CTAs
 };
+
+// ------------------------------------------------------- sliced layout
+// LB_LAYOUT_SLICES (include/lb.h): a packed matrix of n rows with nw words
+// per row is stored slice by slice, slice s (words 16s .. 16s+15 of every row)
+// as a block of n rows; full slices have a pitch of 16 words, the last one the
+// words it holds rounded up to a multiple of 4.  Block s starts at word 16*n*s.
+__host__ __device__ __forceinline__ int64_t sliced_pitch(int64_t nw, int64_t s) {
+    const int64_t last = (nw - 1) >> 4;
+    return s < last ? 16 : ((nw - 16 * last) + 3) & ~(int64_t)3;
+}
+__host__ __device__ __forceinline__ int64_t sliced_offset(int64_t n, int64_t nw, int64_t row,
+                                                          int64_t w) {
+    const int64_t s = w >> 4;
+    return 16 * n * s + row * sliced_pitch(nw, s) + (w & 15);
+}
+__host__ __device__ __forceinline__ int64_t sliced_words(int64_t n, int64_t nw) {
+    const int64_t last = (nw - 1) >> 4;
+    return n * (16 * last + sliced_pitch(nw, last));
+}
 
 // ------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint4 ld_stream_v4(const uint32_t* p) {
@@ -233,8 +253,8 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
                            int64_t r, const lb_branch* br, int nb, float* y, void* workspace,
                            cudaStream_t s);
 
-// Packer (lb_pack.cu).
+// Packer (lb_pack.cu).  sliced: write the sliced layout (ld_words unused).
 cudaError_t launch_pack(const float* latent, int64_t rows, int64_t cols, int64_t ld, int axis,
-                        uint32_t* packed, int64_t ld_words, cudaStream_t s);
+                        uint32_t* packed, int64_t ld_words, bool sliced, cudaStream_t s);
 
 }  // namespace lb

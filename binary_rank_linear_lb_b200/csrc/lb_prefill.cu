@@ -145,7 +145,9 @@ struct PrefillGemm {
     int M, n_seg_rows, n_nseg, n_kseg, k_seg_len;   // N = n_nseg * n_seg_rows, K = n_kseg * k_seg_len
     int stage;                                       // 1 or 2
     const uint32_t* P[2];                            // packed signs per branch
-    int ldw[2];                                      // words per packed row, per branch
+    int ldw[2];                                      // words per packed row, per branch (rows layout)
+    int sliced[2];                                   // branch packed in LB_LAYOUT_SLICES
+    int nw;                                          // words holding the K = k_seg_len signs of a row
     const __half* bscale[2];                         // stage 1: g_b (per k); stage 2: h_b (per n)
     const __half* lscale[2];                         // stage 1: l_b (per output column)
     const float* row_sa;                             // [M] 2^a_m (stage 1 divides it out)
@@ -201,7 +203,11 @@ __device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int
 
 __device__ __forceinline__ uint2 load_bits(const PrefillGemm& g, int branch, int row, int kb) {
     if (row >= g.n_seg_rows) return make_uint2(0u, 0u);
-    return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + (size_t)row * g.ldw[branch] + kb * 2));
+    // a 64-sign K block is two words of one 16-word slice, so it is contiguous in both layouts
+    const size_t off = g.sliced[branch]
+                           ? (size_t)sliced_offset(g.n_seg_rows, g.nw, row, 2 * kb)
+                           : (size_t)row * g.ldw[branch] + kb * 2;
+    return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + off));
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -578,10 +584,12 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         PrefillGemm p = {};
         p.M = (int)M; p.n_seg_rows = (int)r; p.n_nseg = nb; p.n_kseg = 1; p.k_seg_len = (int)in;
         p.stage = 1;
+        p.nw = (int)((in + 31) / 32);
         for (int b = 0; b < 2; ++b) {
             const lb_branch& B = br[b < nb ? b : 0];
             p.P[b] = B.Vp;
             p.ldw[b] = (int)(B.ld_v ? B.ld_v : (in + 31) / 32);
+            p.sliced[b] = B.layout == LB_LAYOUT_SLICES ? 1 : 0;
             p.bscale[b] = reinterpret_cast<const __half*>(B.g);
             p.lscale[b] = reinterpret_cast<const __half*>(B.l);
         }
@@ -596,10 +604,12 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         PrefillGemm p = {};
         p.M = (int)M; p.n_seg_rows = (int)out; p.n_nseg = 1; p.n_kseg = nb; p.k_seg_len = (int)r;
         p.stage = 2;
+        p.nw = (int)((r + 31) / 32);
         for (int b = 0; b < 2; ++b) {
             const lb_branch& B = br[b < nb ? b : 0];
             p.P[b] = B.Up;
             p.ldw[b] = (int)(B.ld_u ? B.ld_u : (r + 31) / 32);
+            p.sliced[b] = B.layout == LB_LAYOUT_SLICES ? 1 : 0;
             p.bscale[b] = reinterpret_cast<const __half*>(B.h);
             p.lscale[b] = nullptr;
         }

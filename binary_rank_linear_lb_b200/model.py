@@ -1,9 +1,10 @@
 """Device-resident factorised linears and decoder stacks built from seeded inputs.
 
 Each branch is generated from its own seeds (``synth``) and binarised on the GPU
-with ``lb_pack_signs``; the fp32 latents are dropped right after packing.  Rows
-are packed with a 64-byte pitch (``ld_words`` a multiple of 16, zero padding),
-so the decode kernels stream aligned 64-byte row pieces.
+with ``lb_pack_signs_sliced`` (the default sliced layout, whose 512-sign slices
+are contiguous blocks of rows) or ``lb_pack_signs`` (row-major, with a 64-byte
+pitch: ``ld_words`` a multiple of 16, zero padding); the fp32 latents are
+dropped right after packing.
 
 ``signs="bits"`` instead draws the packed words directly from a uniform bit
 source.  The signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so the
@@ -17,7 +18,7 @@ from typing import List, Optional
 
 import torch
 
-from . import Branch, Stack, pack_signs, synth
+from . import LB_LAYOUT_ROWS, LB_LAYOUT_SLICES, Branch, Stack, pack_signs, slice_words, synth
 from .configs import Model, proj_shape
 
 
@@ -33,46 +34,50 @@ def padded_words(k: int, pad: bool = True) -> int:
 
 
 def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int, branch: int,
-                 device="cuda", signs: str = "latent", pad: bool = True) -> Branch:
+                 device="cuda", signs: str = "latent", pad: bool = True,
+                 layout: int = LB_LAYOUT_SLICES) -> Branch:
+    """One branch from its seeds.  layout: LB_LAYOUT_SLICES (the batch-1 fast
+    layout, the default) or LB_LAYOUT_ROWS (row-major, pitch padded_words(k, pad))."""
     s = lambda k: synth.tensor_seed(base, layer, proj, branch, k)
     h = synth.scale(out_f, s(synth.KIND_H), device)
     g = synth.scale(in_f, s(synth.KIND_G), device)
     l = synth.scale(r, s(synth.KIND_L), device)
     if signs == "latent":
         V = synth.latent(in_f, r, s(synth.KIND_V), device)
-        Vp = pack_signs(V, axis=0, ld_words=padded_words(in_f, pad))
+        Vp = pack_signs(V, axis=0, ld_words=padded_words(in_f, pad), layout=layout)
         del V
         U = synth.latent(out_f, r, s(synth.KIND_U), device)
-        Up = pack_signs(U, axis=1, ld_words=padded_words(r, pad))
+        Up = pack_signs(U, axis=1, ld_words=padded_words(r, pad), layout=layout)
         del U
     elif signs == "bits":
         def words(n_rows, k, seed):
             gen = torch.Generator(device=device)
             gen.manual_seed(seed)
             nw = (k + 31) // 32
-            w = torch.zeros((n_rows, padded_words(k, pad)), dtype=torch.int32, device=device)
+            ldw = padded_words(k, pad) if layout == LB_LAYOUT_ROWS else nw
+            w = torch.zeros((n_rows, ldw), dtype=torch.int32, device=device)
             w[:, :nw] = torch.randint(-2 ** 31, 2 ** 31, (n_rows, nw), generator=gen,
                                       device=device, dtype=torch.int64).to(torch.int32)
             if k % 32:
                 w[:, nw - 1] &= (1 << (k % 32)) - 1
-            return w
+            return w if layout == LB_LAYOUT_ROWS else slice_words(w, k)
         Vp = words(r, in_f, s(synth.KIND_V))
         Up = words(out_f, r, s(synth.KIND_U))
     else:
         raise ValueError(signs)
-    return Branch(Vp, Up, h, g, l)
+    return Branch(Vp, Up, h, g, l, layout)
 
 
 def build_linear(in_f: int, out_f: int, r: int, base: int = 0, layer: int = 0, proj: int = 0,
                  n_branches: int = 2, device="cuda", signs: str = "latent",
-                 pad: bool = True) -> List[Branch]:
-    return [build_branch(in_f, out_f, r, base, layer, proj, b, device, signs, pad)
+                 pad: bool = True, layout: int = LB_LAYOUT_SLICES) -> List[Branch]:
+    return [build_branch(in_f, out_f, r, base, layer, proj, b, device, signs, pad, layout)
             for b in range(n_branches)]
 
 
 def build_stack(model: Model, bpw: float, base: int = 0, n_layers: Optional[int] = None,
                 n_branches: int = 2, device="cuda", signs: str = "latent",
-                ranks: Optional[List[int]] = None) -> Stack:
+                ranks: Optional[List[int]] = None, layout: int = LB_LAYOUT_SLICES) -> Stack:
     nl = n_layers or model.n_layers
     rk = ranks or model.ranks(bpw)
     linears, all_ranks = [], []
@@ -80,7 +85,8 @@ def build_stack(model: Model, bpw: float, base: int = 0, n_layers: Optional[int]
         L = []
         for p in range(7):
             i, o = proj_shape(p, model.hidden, model.inter, model.kv_dim)
-            L.append(build_linear(i, o, rk[p], base, li, p, n_branches, device, signs))
+            L.append(build_linear(i, o, rk[p], base, li, p, n_branches, device, signs,
+                                  layout=layout))
         linears.append(L)
         all_ranks.append(list(rk))
     return Stack(linears, all_ranks, model.hidden, model.inter, model.n_heads, model.n_kv_heads,
@@ -89,10 +95,10 @@ def build_stack(model: Model, bpw: float, base: int = 0, n_layers: Optional[int]
 
 def build_mlp_block(model: Model, bpw: float, base: int = 0, n_branches: int = 2,
                     device="cuda", signs: str = "latent",
-                    ranks: Optional[List[int]] = None) -> Stack:
+                    ranks: Optional[List[int]] = None, layout: int = LB_LAYOUT_SLICES) -> Stack:
     rk = ranks or model.ranks(bpw)
     L: list = [None] * 7
     for p in (4, 5, 6):
         i, o = proj_shape(p, model.hidden, model.inter, model.kv_dim)
-        L[p] = build_linear(i, o, rk[p], base, 0, p, n_branches, device, signs)
+        L[p] = build_linear(i, o, rk[p], base, 0, p, n_branches, device, signs, layout=layout)
     return Stack([L], [list(rk)], model.hidden, model.inter, mlp_only=True, device=device)

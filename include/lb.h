@@ -81,19 +81,56 @@ int lb_version(void);
 lb_status lb_pack_signs(const float *latent, int64_t rows, int64_t cols, int64_t ld,
                         int axis, uint32_t *packed, int64_t ld_words, void *stream);
 
-/* One branch of a factorised layer (device pointers and row pitches).
- * ld_v / ld_u are the words per packed row of Vp / Up (0 means the unpadded
- * ceil(in/32) / ceil(r/32)).  Rows padded to a multiple of 4 words (16 bytes)
- * let the decode kernels stream them with the tensor-memory accelerator; other
- * pitches take a slower copy path.  Padding words are never read for results. */
+/*
+ * Layouts of a packed matrix of n rows of K signs (nw = ceil(K/32) words each).
+ *
+ *   LB_LAYOUT_ROWS   : row-major, [n][ld] words (ld >= nw), as written by
+ *                      lb_pack_signs.  The canonical layout.
+ *   LB_LAYOUT_SLICES : the same words regrouped by 512-sign slice, as written
+ *                      by lb_pack_signs_sliced.  Slice s (words 16s .. 16s+15
+ *                      of every row) is a block of n rows starting at word
+ *                      16*n*s; full slices have a pitch of 16 words (64 bytes),
+ *                      the last slice the words it holds rounded up to a
+ *                      multiple of 4.  Padding words are 0.
+ *
+ * Both hold the same bits.  The decode kernels read one 512-sign slice of many
+ * rows at a time: in the sliced layout that is one contiguous block, which
+ * DRAM streams at close to full bandwidth, whereas row-major rows give one
+ * 64-byte piece per row and DRAM about half of it.  Prefer LB_LAYOUT_SLICES
+ * for weights that are read by the batch-1 path.
+ */
+typedef enum { LB_LAYOUT_ROWS = 0, LB_LAYOUT_SLICES = 1 } lb_layout;
+
+/* Words a packed matrix of n rows of K signs occupies in `layout`
+ * (LB_LAYOUT_ROWS: n * max(ld_words, ceil(K/32))); 0 for bad arguments. */
+size_t lb_packed_words(int64_t n, int64_t k, int layout, int64_t ld_words);
+
+/*
+ * lb_pack_signs_sliced — lb_pack_signs writing LB_LAYOUT_SLICES: the packed
+ * matrix has n = rows (axis 1) or n = cols (axis 0) rows of K = cols (axis 1)
+ * or K = rows (axis 0) signs, and `packed` receives lb_packed_words(n, K,
+ * LB_LAYOUT_SLICES, 0) words.  Same errors as lb_pack_signs, and
+ * LB_ERR_ALIGNMENT unless packed is 16-byte aligned.
+ */
+lb_status lb_pack_signs_sliced(const float *latent, int64_t rows, int64_t cols, int64_t ld,
+                               int axis, uint32_t *packed, void *stream);
+
+/* One branch of a factorised layer (device pointers, row pitches, layout).
+ * ld_v / ld_u are the words per packed row of Vp / Up in LB_LAYOUT_ROWS (0
+ * means the unpadded ceil(in/32) / ceil(r/32)); with LB_LAYOUT_SLICES they
+ * must be 0.  In LB_LAYOUT_ROWS, a pitch that is a multiple of 16 words (64
+ * bytes) keeps every slice of every row one aligned DRAM piece.  Padding words
+ * are never read.  A zero-initialised `layout` means LB_LAYOUT_ROWS. */
 typedef struct {
-    const uint32_t *Vp;   /* [r][ld_v] signs of V_b packed along in          */
-    const uint32_t *Up;   /* [out][ld_u] signs of U_b packed along r         */
+    const uint32_t *Vp;   /* signs of V_b: r rows of in signs (packed along in)   */
+    const uint32_t *Up;   /* signs of U_b: out rows of r signs (packed along r)    */
     const uint16_t *h;    /* [out] FP16 row scale (IEEE binary16 bits), 4-byte aligned */
     const uint16_t *g;    /* [in]  FP16 column scale                         */
     const uint16_t *l;    /* [r]   FP16 latent scale                         */
     int64_t ld_v;         /* words per packed row of Vp, 0 or >= ceil(in/32) */
     int64_t ld_u;         /* words per packed row of Up, 0 or >= ceil(r/32)  */
+    int32_t layout;       /* lb_layout of Vp and Up                          */
+    int32_t reserved;     /* 0                                               */
 } lb_branch;
 
 /*

@@ -85,3 +85,25 @@ def test_stack_workspace_size_is_host_only(lb):
     assert L.lb_stack_workspace_size(ctypes.byref(bad)) == 0
     assert L.lb_stack_forward(ctypes.byref(bad), 256, size, 256, 256, None) == \
         lb.LB_ERR_INVALID_ARG
+
+
+def test_sliced_layout_sizes_and_argument_errors(lb):
+    L = lb.lib()
+    S, R = lb.LB_LAYOUT_SLICES, lb.LB_LAYOUT_ROWS
+    # n rows of k signs: full 16-word slices, then the last slice's words rounded up to 4
+    for n, k, words in ((1, 1, 4), (3, 512, 48), (2, 513, 2 * (16 + 4)), (5, 3136, 5 * (96 + 4)),
+                        (7, 1100, 7 * (32 + 4)), (4, 8192, 4 * 256)):
+        assert L.lb_packed_words(n, k, S, 0) == words
+    assert L.lb_packed_words(3, 100, R, 0) == 3 * 4
+    assert L.lb_packed_words(3, 100, R, 9) == 27
+    assert L.lb_packed_words(3, 100, R, 2) == 0          # pitch below ceil(k/32)
+    assert L.lb_packed_words(3, 100, 7, 0) == 0          # no such layout
+    assert L.lb_packed_words(0, 100, S, 0) == 0
+    assert L.lb_pack_signs_sliced(None, 4, 4, 4, 0, 16, None) == lb.LB_ERR_INVALID_ARG
+    assert L.lb_pack_signs_sliced(16, 4, 4, 4, 2, 16, None) == lb.LB_ERR_INVALID_ARG
+    assert L.lb_pack_signs_sliced(16, 4, 4, 4, 1, 24, None) == lb.LB_ERR_ALIGNMENT
+    # a sliced branch takes no row pitch, and the layout must be known
+    for ld_v, layout in ((4, S), (0, 9)):
+        br = (lb.lb_branch * 1)(lb.lb_branch(16, 16, 16, 16, 16, ld_v, 0, layout, 0))
+        assert L.lb_linear_forward(16, 0, 1, 64, 64, 32, ctypes.addressof(br), 1, 16, 16,
+                                   1 << 20, None) == lb.LB_ERR_INVALID_ARG

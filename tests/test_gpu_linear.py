@@ -17,8 +17,8 @@ from helpers import assert_close, oracle_linear, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def run_case(in_f, out_f, r, M, dtype, nb=2, base=0, rows=None):
-    brs = build_linear(in_f, out_f, r, base=base, n_branches=nb)
+def run_case(in_f, out_f, r, M, dtype, nb=2, base=0, rows=None, layout=lb.LB_LAYOUT_SLICES):
+    brs = build_linear(in_f, out_f, r, base=base, n_branches=nb, layout=layout)
     x = synth.activation((M, in_f), synth.tensor_seed(base, 0, 0, 0, synth.KIND_X), dtype, "cuda")
     y = lb.linear_forward(x, brs, in_f, out_f, r)
     torch.cuda.synchronize()
@@ -39,9 +39,21 @@ def test_single_linear_config():
 @pytest.mark.parametrize("shape", [(1, 1, 1), (32, 32, 32), (100, 33, 7), (1000, 300, 70),
                                    (1024, 1024, 1024), (1100, 2100, 1088), (300, 5000, 2100)])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
-def test_ragged_shapes(shape, dtype):
-    got, ref = run_case(*shape, M=1, dtype=dtype)
+@pytest.mark.parametrize("layout", [lb.LB_LAYOUT_SLICES, lb.LB_LAYOUT_ROWS])
+def test_ragged_shapes(shape, dtype, layout):
+    got, ref = run_case(*shape, M=1, dtype=dtype, layout=layout)
     assert_close(got, ref, what=str(shape))
+
+
+def test_rows_layout_unpadded_pitch():
+    """Row-major weights with the unpadded pitch ceil(k/32) (odd and 2-word pitches)."""
+    for in_f, out_f, r in ((1000, 300, 70), (640, 2100, 60), (96, 64, 33)):
+        brs = [b for b in build_linear(in_f, out_f, r, base=9, layout=lb.LB_LAYOUT_ROWS, pad=False)]
+        x = synth.activation((1, in_f), 90, torch.bfloat16, "cuda")
+        y = lb.linear_forward(x, brs, in_f, out_f, r)
+        torch.cuda.synchronize()
+        ref = oracle.forward(to_f64(x), oracle_linear(in_f, out_f, r, 9, 0, 0), in_f, out_f, r)
+        assert_close(y.cpu().numpy(), ref, what=f"unpadded {in_f, out_f, r}")
 
 
 @pytest.mark.parametrize("M", [2, 3, 8, 11])
@@ -91,10 +103,11 @@ def test_workspace_reports_ok_and_repeat_calls_agree():
 @pytest.mark.parametrize("shape", [(512, 256, 64), (640, 1000, 192), (1024, 1001, 128),
                                    (4096, 11008, 128)])
 @pytest.mark.parametrize("M", [16, 100, 256])
-def test_prefill_path_shapes(shape, M):
+@pytest.mark.parametrize("layout", [lb.LB_LAYOUT_SLICES, lb.LB_LAYOUT_ROWS])
+def test_prefill_path_shapes(shape, M, layout):
     in_f, out_f, r = shape
     assert lb.linear_path(M, in_f, out_f, r) == 1
-    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=3)
+    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=3, layout=layout)
     for m in (0, M // 2, M - 1):
         assert_close(got[m], ref[m], what=f"{shape} M={M} row {m}")
     assert_close(got, ref, what=f"{shape} M={M}")

@@ -1,4 +1,4 @@
-"""lb_pack_signs against the oracle's packer: bit-exact (GPU)."""
+"""lb_pack_signs / lb_pack_signs_sliced against the oracle's packer: bit-exact (GPU)."""
 import numpy as np
 import pytest
 import torch
@@ -60,3 +60,40 @@ def test_pack_full_size_70b_gate(which):
     w = lb.pack_signs(lat, axis)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), oracle.pack(lat.cpu().numpy(), axis))
+
+
+def spec_slices(words: np.ndarray, k: int) -> np.ndarray:
+    """The sliced layout as include/lb.h defines it, from row-major words [n][ceil(k/32)]."""
+    n, nw = words.shape[0], (k + 31) // 32
+    ns = (nw + 15) // 16
+    out = []
+    for s in range(ns):
+        width = min(16, nw - 16 * s)
+        pitch = 16 if s < ns - 1 else (width + 3) // 4 * 4
+        block = np.zeros((n, pitch), np.uint32)
+        block[:, :width] = words[:, 16 * s:16 * s + width]
+        out.append(block.reshape(-1))
+    return np.concatenate(out)
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (31, 33), (64, 512), (100, 513), (700, 1100),
+                                   (2000, 33), (1536, 96)])
+@pytest.mark.parametrize("axis", [0, 1])
+def test_pack_sliced_bit_exact(shape, axis):
+    rng = np.random.default_rng(shape[0] * 3 + shape[1] + 11 * axis)
+    lat = rng.standard_normal(shape).astype(np.float32)
+    lat.flat[rng.integers(0, lat.size, size=min(lat.size, 16))] = -0.0
+    t = torch.from_numpy(lat).cuda()
+    got = lb.pack_signs(t, axis, layout=lb.LB_LAYOUT_SLICES)
+    torch.cuda.synchronize()
+    k = shape[1] if axis == 1 else shape[0]
+    n = shape[0] if axis == 1 else shape[1]
+    ref = oracle.pack(lat, axis)
+    assert got.numel() == lb.packed_words(n, k, lb.LB_LAYOUT_SLICES)
+    np.testing.assert_array_equal(got.cpu().numpy().view(np.uint32), spec_slices(ref, k))
+    # and the binding's converters agree with the layout
+    back = lb.unslice_words(got, n, k).cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(back, ref)
+    np.testing.assert_array_equal(
+        lb.slice_words(torch.from_numpy(ref.view(np.int32)), k).numpy().view(np.uint32),
+        spec_slices(ref, k))

@@ -34,9 +34,9 @@ def ostack_names():
     return ("q", "k", "v", "o", "gate", "up", "down")
 
 
-def run_stack(model, bpw, n_layers, base, ranks=None):
+def run_stack(model, bpw, n_layers, base, ranks=None, layout=lb.LB_LAYOUT_SLICES):
     rk = ranks or model.ranks(bpw)
-    st = build_stack(model, bpw, base=base, n_layers=n_layers, ranks=rk)
+    st = build_stack(model, bpw, base=base, n_layers=n_layers, ranks=rk, layout=layout)
     x = synth.activation(model.hidden, synth.tensor_seed(base, 0, 0, 0, synth.KIND_X),
                          torch.bfloat16, "cuda")
     y = st.forward(x)
@@ -51,8 +51,10 @@ def run_stack(model, bpw, n_layers, base, ranks=None):
 SMALL = Model("small", hidden=256, inter=512, n_layers=3, n_heads=4, n_kv_heads=2, head_dim=64)
 
 
-def test_small_decoder_stack_and_intermediates():
-    st, x, y, h_ref, outs = run_stack(SMALL, 1.0, 3, base=3, ranks=[64, 32, 32, 64, 96, 96, 96])
+@pytest.mark.parametrize("layout", [lb.LB_LAYOUT_SLICES, lb.LB_LAYOUT_ROWS])
+def test_small_decoder_stack_and_intermediates(layout):
+    st, x, y, h_ref, outs = run_stack(SMALL, 1.0, 3, base=3, ranks=[64, 32, 32, 64, 96, 96, 96],
+                                      layout=layout)
     assert_close(y.cpu().numpy(), h_ref, what="small stack")
     for li in range(3):
         for p, name in ((0, "q"), (1, "k"), (2, "v"), (4, "gate"), (5, "up")):
