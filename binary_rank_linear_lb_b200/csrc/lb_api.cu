@@ -67,9 +67,6 @@ void set_job_shape(LbJob& J, int64_t rows, int64_t cols, int64_t ld, int layout)
     J.n_slices = (int)cdiv(cols, kSliceElems);
     J.n_rowblocks = (int)cdiv(rows, kRowBlock);
     J.rg = J.n_rowblocks;
-    J.use_tma = 0;   // sliced rows are contiguous per slice: plain bulk prefetches serve them
-    if (!J.sliced && (J.ldw & 3) == 0 && (reinterpret_cast<uintptr_t>(J.P) & 15) == 0)
-        J.use_tma = make_sign_tmap(&J.tmap, J.P, J.rows, J.ldw, (int)cdiv(cols, 32)) ? 1 : 0;
 }
 
 bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <= (1 << 26)); }

@@ -52,8 +52,6 @@ namespace {
 
 constexpr long long kSpinLimitCycles = 4000000000LL;   // ~2 s at 2 GHz
 constexpr int kMaxTiles = kTables;                      // tiles of one batch
-constexpr int kPrefetchDepth = 4;                       // rowblocks a warp has requested ahead (L2)
-constexpr int kEarlyPrefetch = 1;                       // of them, requested before a phase's wait
 
 struct Smem {
     float* vec;       // kTables staged slices; element j at j + 4*(j/64)
@@ -165,9 +163,9 @@ __device__ __forceinline__ T* resolve(T* p, const CallArgs& a) {
     return p;
 }
 
-// Grid-wide wait, split in two so a CTA can issue the next phase's loads and
-// prefetches between announcing that it is done (grid_arrive) and waiting for
-// everyone else (grid_wait).  The arrival is a release-add: every write of the
+// Grid-wide wait, split in two so a CTA can set up the next phase between
+// announcing that it is done (grid_arrive) and waiting for everyone else
+// (grid_wait).  The arrival is a release-add: every write of the
 // CTA made before it (ordered by the preceding __syncthreads) is visible to a
 // CTA whose acquire-load sees the count.  The wait gives up after
 // kSpinLimitCycles and records LB_ERR_TIMEOUT; it returns false if this CTA
@@ -233,6 +231,19 @@ __device__ __forceinline__ void load_src(const LbJob& J, const void* src, int j,
     }
 }
 
+// Entries m and m + 16 (m = kM .. 15) of one chunk; entry offsets are
+// immediates of the stores.
+template <int kM>
+__device__ __forceinline__ void store_entries(uint32_t base, const float (&p01)[4],
+                                              const float (&p23)[4], float c0, float c1) {
+    if constexpr (kM < 16) {
+        const float l4 = p01[kM & 3] + p23[kM >> 2];
+        sts_f32_off<kM * 256>(base, l4 + c0);
+        sts_f32_off<(kM + 16) * 256>(base, l4 + c1);
+        store_entries<kM + 1>(base, p01, p23, c0, c1);
+    }
+}
+
 // Build the table of one staged slice at shared address taddr.  Thread t owns
 // chunk c (slot i = t & 63: qb = i&3, wb1 = (i>>2)&1, gam = (i>>3)&3,
 // reg&1 = i>>5) and the 32 entries e = 32*(t>>6) + m, m = 0..31; a warp's 32
@@ -252,14 +263,7 @@ __device__ __forceinline__ void build_table(const float* vec, uint32_t taddr) {
     const float c0 = hk + hi.x, c1 = hk - hi.x;
     const uint32_t base = taddr + (uint32_t)k * (32u * 256u) + (uint32_t)w0 * 128u +
                           (uint32_t)(32 * gam + 16 * wb1 + 4 * qb);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        const float l4 = p01[m & 3] + p23[m >> 2];
-        asm volatile("st.shared.f32 [%0], %1;" :: "r"(base + (uint32_t)m * 256u), "f"(l4 + c0)
-                     : "memory");
-        asm volatile("st.shared.f32 [%0], %1;" :: "r"(base + (uint32_t)(m + 16) * 256u),
-                     "f"(l4 + c1) : "memory");
-    }
+    store_entries<0>(base, p01, p23, c0, c1);
 }
 
 // ---- tiles and batches ----------------------------------------------------
@@ -297,9 +301,6 @@ struct TileRt {
     int ldw, rows, wrem;     // row pitch, rows, words of the slice holding signs (<= 16)
     int rb0, nrb;
     uint32_t tb;             // table address bits (kTableAddr0 + t * 64 KB)
-    const CUtensorMap* tmap; // the job's tensor map (in the plan) for L2 prefetch, or nullptr
-    int x;                   // the slice's first word (tensor-map coordinate)
-    int bulk;                // rows of the slice are contiguous: prefetch a rowblock as one range
 };
 
 // This CTA's place in a phase and the batch about to run.  sc[k] is this
@@ -308,7 +309,6 @@ struct TileRt {
 struct Cursor {
     int u, u_end, j;
     int nt, n_rb;
-    int pf0;                 // rowblock steps of the batch already prefetched to L2
     Tile t[kMaxTiles];
     TileRt rt[kMaxTiles];
     unsigned short sc[kMaxTiles];   // fp16 bits
@@ -336,6 +336,12 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
     const int lane = threadIdx.x & 31;
     const int rho = lane >> 2, gam = lane & 3;
     const int w = 4 * gam;
+    if (T.wrem == kSliceWords && (T.ldw & 3) == 0 && rb * kRowBlock + kRowBlock <= T.rows) {
+        // the usual case: all 32 rows inside, full 16-word pieces
+        const uint32_t* p = T.P + (size_t)(rb * kRowBlock + 4 * rho) * (size_t)T.ldw + w;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) R.d[i] = ld_stream_v4(p + (size_t)i * T.ldw);
+    } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int row = rb * kRowBlock + 4 * rho + i;
@@ -359,6 +365,7 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
             }
         }
         R.d[i] = d;
+    }
     }
     R.h = 0x3C00u;   // 1.0
     if (T.h != nullptr) {
@@ -392,8 +399,9 @@ __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
         for (int r = 0; r < 4; ++r) {
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]) + (uint32_t)(r & 1) * 128u;
-                const float v = lds_f32(addr);
+                // odd registers sit in the upper half of each entry row: offset 128
+                const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]);
+                const float v = (r & 1) ? lds_f32_off<128>(addr) : lds_f32_off<0>(addr);
                 if (jj & 1) a1 += v; else a0 += v;
             }
         }
@@ -443,34 +451,8 @@ __device__ __forceinline__ TileRt batch_tile(const Cursor& c, int n, int& rb) {
     T.rb0 = k ? c.rt[1].rb0 : c.rt[0].rb0;
     T.nrb = k ? c.rt[1].nrb : c.rt[0].nrb;
     T.tb = k ? c.rt[1].tb : c.rt[0].tb;
-    T.tmap = k ? c.rt[1].tmap : c.rt[0].tmap;
-    T.x = k ? c.rt[1].x : c.rt[0].x;
-    T.bulk = k ? c.rt[1].bulk : c.rt[0].bulk;
     rb = T.rb0 + (k ? n - c.rt[0].nrb : n);
     return T;
-}
-
-// Lane 0 asks the TMA unit to bring rowblock n of the batch into L2 (no data
-// comes back to the SM; the register loads kDepth rowblocks later then hit L2).
-__device__ __forceinline__ void prefetch_rb(const Cursor& c, int n) {
-    if ((threadIdx.x & 31) == 0 && n < c.n_rb) {
-        int rb;
-        const TileRt T = batch_tile(c, n, rb);
-        if (T.tmap != nullptr) {
-            tma_prefetch_2d(T.tmap, T.x, rb * kRowBlock);
-        } else if (T.bulk) {   // rows rb*32 .. of the slice block, 16-byte multiple
-            const int nrow = min(kRowBlock, T.rows - rb * kRowBlock);
-            bulk_prefetch_l2(T.P + (size_t)rb * kRowBlock * T.ldw, (uint32_t)(nrow * T.ldw * 4));
-        }
-    }
-}
-
-// L2 prefetches for this warp's rowblocks d = from .. to-1 steps ahead
-// (n = wp + d * kDecodeWarps).  They never stall the warp: the TMA unit
-// takes them, and no data returns to the SM.
-__device__ __forceinline__ void batch_prefetch(const Cursor& c, int from, int to) {
-    const int wp = threadIdx.x >> 5;
-    for (int d = from; d < to; ++d) prefetch_rb(c, wp + d * kDecodeWarps);
 }
 
 // Issue this warp's first kDepth rowblocks of the batch into buf.  Register
@@ -503,7 +485,6 @@ __device__ __forceinline__ void batch_lookups(const Cursor& c, RB (&buf)[kDepth]
                 int rb;
                 const TileRt T = batch_tile(c, n, rb);
                 consume_rb(buf[d], T, rb, Bc, S);
-                prefetch_rb(c, n + kPrefetchDepth * kDecodeWarps);
                 const int nn = n + kDepth * kDecodeWarps;
                 if (nn < c.n_rb) {
                     int rb2;
@@ -517,11 +498,9 @@ __device__ __forceinline__ void batch_lookups(const Cursor& c, RB (&buf)[kDepth]
 
 // Collect the next batch at c.u and load this thread's scale elements.
 // Reads only plan data and weights.
-__device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args,
-                                            const LbJob* jobs_g, Cursor& c) {
+__device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args, Cursor& c) {
     c.nt = 0;
     c.n_rb = 0;
-    c.pf0 = 0;
 #pragma unroll
     for (int k = 0; k < kMaxTiles; ++k) {
         c.sc[k] = 0u;
@@ -546,9 +525,6 @@ __device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args
             T.rb0 = t.rb0;
             T.nrb = t.nrb;
             T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
-            T.tmap = J.use_tma ? &jobs_g[sm.phase->job_begin + t.job].tmap : nullptr;
-            T.x = t.slice * kSliceWords;
-            T.bulk = J.sliced;
             c.n_rb += t.nrb;
             const int col = t.slice * kSliceElems + (int)threadIdx.x;
             if (col < J.cols) c.sc[k] = __ldg(reinterpret_cast<const unsigned short*>(J.vscale) + col);
@@ -558,8 +534,7 @@ __device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args
 
 // Stage the batch's vector slices into shared memory (zero past cols): all
 // source loads are issued before any is used, so the batch costs one round
-// trip to L2, and L2 prefetches for this warp's first rowblocks of the batch
-// follow them.  The owner of a slice (the CTA holding its first rowblock) also
+// trip to L2.  The owner of a slice (the CTA holding its first rowblock) also
 // seeds the residual and adds the slice's sum of squares for RMSNorm; only
 // the first job of a phase carries acc_sumsq, so there is one sum per batch.
 // Ends with a CTA barrier.
@@ -579,8 +554,6 @@ __device__ __forceinline__ void stage_batch(const Smem& sm, const CallArgs& args
             if (J.kind == VK_T && J.norm_sumsq != nullptr) nrm[k] = __ldcg(J.norm_sumsq);
         }
     }
-    // the batch's first rowblocks head for L2 behind the (latency-critical) source loads
-    batch_prefetch(c, c.pf0, kPrefetchDepth);
     float sq = 0.0f;
     float* acc = nullptr;
 #pragma unroll
@@ -618,18 +591,17 @@ __device__ __forceinline__ void stage_batch(const Smem& sm, const CallArgs& args
 
 // The part of a phase that does not depend on earlier phases: this CTA's
 // unit range and its first batch.  sm.phase / sm.jobs must hold the phase.
-__device__ __forceinline__ void phase_begin(const Smem& sm, const CallArgs& args,
-                                            const LbJob* jobs_g, Cursor& c) {
+__device__ __forceinline__ void phase_begin(const Smem& sm, const CallArgs& args, Cursor& c) {
     unit_range(sm, c.u, c.u_end);
     c.j = 0;
     c.nt = 0;
     c.n_rb = 0;
-    if (c.u < c.u_end) batch_begin(sm, args, jobs_g, c);
+    if (c.u < c.u_end) batch_begin(sm, args, c);
 }
 
 // The rest of the phase, after the grid-wide wait.
-__device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, const LbJob* jobs_g,
-                                          Cursor& c, RB (&buf)[kDepth],
+__device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, Cursor& c,
+                                          RB (&buf)[kDepth],
                           const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
     const int G = gridDim.x, cta = blockIdx.x;
     float* zp = resolve(sm.phase->zero_ptr, args);
@@ -646,7 +618,7 @@ __device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, 
         __syncthreads();
         batch_lookups(c, buf, Bc, S);
         c.u += c.n_rb;
-        if (c.u < c.u_end) batch_begin(sm, args, jobs_g, c);
+        if (c.u < c.u_end) batch_begin(sm, args, c);
         __syncthreads();
     }
 }
@@ -682,9 +654,9 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
     __syncthreads();
     Cursor cur;
     RB buf[kDepth];
-    phase_begin(sm, args, jobs, cur);
+    phase_begin(sm, args, cur);
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args, jobs, cur, buf, Bc, S);
+        run_phase(sm, args, cur, buf, Bc, S);
         if (p + 1 < n_phases) {
             // Announce completion, then use the wait: switch to the next
             // phase's plan, load the scales of its first batch and fetch the
@@ -696,11 +668,7 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
             __syncthreads();
             const int nb = (p + 1) & 1;
             use_plan_buf(sm, nb);
-            phase_begin(sm, args, jobs, cur);
-            if (cur.u < cur.u_end) {   // a little of the next phase heads for L2 during the wait
-                batch_prefetch(cur, 0, kEarlyPrefetch);
-                cur.pf0 = kEarlyPrefetch;
-            }
+            phase_begin(sm, args, cur);
             if (kAsyncPlan && wp == kDecodeWarps - 1 && p + 2 < n_phases)
                 cache_plan_async(phases, p + 2, sm.phase->next_job_begin, sm.phase->next_n_jobs,
                                  jobs, splits, nb ^ 1);
@@ -756,36 +724,6 @@ cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
 }
 
 }  // namespace
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// 2-D tensor map of a packed sign matrix with 32-row x 16-word boxes (one
-// rowblock of one slice), used for L2 prefetches of whole rowblocks.
-bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw, int words) {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    if (!fn || rows <= 0 || ldw <= 0 || (ldw & 3) != 0 || words <= 0 || words > ldw) return false;
-    // the tensor's width is the words holding signs, so boxes stop before a padded pitch
-    const cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)ldw * 4};
-    const cuuint32_t box[2] = {(cuuint32_t)kSliceWords, (cuuint32_t)kRowBlock};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(P), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_64B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
 
 int decode_grid() { return device_sm_count() * kCtasPerSm; }
 

@@ -57,7 +57,6 @@ enum VecKind : int {
 };
 
 struct alignas(64) LbJob {
-    CUtensorMap tmap;         // 2-D TMA descriptor of P (32-row x 16-word boxes) for L2 prefetch, if use_tma
     const uint32_t* P;        // packed rows [rows][ldw] (ldw = row pitch in words)
     const void* src;          // vector source
     const float* src2;        // second source (VK_SILU_MUL)
@@ -69,7 +68,7 @@ struct alignas(64) LbJob {
     float* resid_init;        // owner of a slice writes float(src) of the slice here
     int rows, cols, ldw, kind;
     int n_slices, n_rowblocks, unit_begin, norm_n;
-    int gqa_ghd, gqa_hd, use_tma;
+    int gqa_ghd, gqa_hd;
     int rg;                   // rowblocks per row group (units run group, slice, rowblock)
     int sliced;               // P is in the sliced layout (LB_LAYOUT_SLICES), ldw unused
 };
@@ -148,28 +147,6 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float
     asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
                  :: "l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
-}
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-    asm volatile("prefetch.global.L1 [%0];" :: "l"(p));
-}
-// Exact-size L2 prefetch (16-byte aligned address, size a multiple of 16).
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
-}
-// Read-only sign words through L1 (rows are L1-prefetched a few steps ahead).
-__device__ __forceinline__ uint4 ld_sign_v4(const uint32_t* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint32_t ld_sign_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -183,10 +160,17 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
 }
-__device__ __forceinline__ float lds_f32(uint32_t saddr) {
+// Shared-memory load / store at a 32-bit shared-window address plus a
+// constant byte offset, which goes into the instruction instead of a register.
+template <int kOff>
+__device__ __forceinline__ float lds_f32_off(uint32_t saddr) {
     float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr));
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(saddr), "n"(kOff));
     return v;
+}
+template <int kOff>
+__device__ __forceinline__ void sts_f32_off(uint32_t saddr, float v) {
+    asm volatile("st.shared.f32 [%0+%1], %2;" :: "r"(saddr), "n"(kOff), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -215,22 +199,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%3, %4}], [%2];"
         :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
 }
-// L2 prefetch of one box of a 2-D tensor map (no shared memory involved).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 :: "l"(map), "r"(x), "r"(y) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // ------------------------------------------------------------ host helpers
 int device_sm_count();               // SMs of the current device (cached per device)
 bool device_is_sm100();
 cudaError_t decode_configure();      // one-time kernel attribute setup per device
-// 2-D TMA descriptor of a packed sign matrix: rows x `words` words holding
-// signs, row pitch ldw words (a multiple of 4).
-bool make_sign_tmap(CUtensorMap* map, const uint32_t* P, int rows, int ldw, int words);
 
 // Decode phase program launches (lb_decode.cu).
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,
