@@ -376,6 +376,36 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
 
 // Look up rowblock R against the table at address bits tb and add the row
 // sums (times the row scale) to out.
+// The 16 lookups of one 16-byte group (register R of the group, byte jj
+// chosen per lane by the selector), written out by template recursion so every
+// register and constant index is known at compile time.  Odd registers sit in
+// the upper half of each entry row: offset 128.
+template <int R, int JJ>
+__device__ __forceinline__ void group_lookups(const uint32_t (&w4)[4], const uint32_t (&B)[2][4],
+                                              const uint32_t (&S)[4], float& a0, float& a1) {
+    const uint32_t addr = prmt(w4[R], B[R >> 1][JJ], S[JJ]);
+    const float v = lds_f32_off<(R & 1) * 128>(addr);
+    if (JJ & 1) a1 += v; else a0 += v;
+    if constexpr (JJ < 3) group_lookups<R, JJ + 1>(w4, B, S, a0, a1);
+    else if constexpr (R < 3) group_lookups<R + 1, 0>(w4, B, S, a0, a1);
+}
+
+// Slice sums of the four row steps of a rowblock (lanes with rho >= 4 read the
+// halves of their group swapped).
+template <int I>
+__device__ __forceinline__ void step_sums(const RB& Rb, bool swap, const uint32_t (&B)[2][4],
+                                          const uint32_t (&S)[4], float (&acc)[4]) {
+    uint32_t w4[4];
+    w4[0] = swap ? Rb.d[I].z : Rb.d[I].x;
+    w4[1] = swap ? Rb.d[I].w : Rb.d[I].y;
+    w4[2] = swap ? Rb.d[I].x : Rb.d[I].z;
+    w4[3] = swap ? Rb.d[I].y : Rb.d[I].w;
+    float a0 = 0.0f, a1 = 0.0f;
+    group_lookups<0, 0>(w4, B, S, a0, a1);
+    acc[I] = a0 + a1;
+    if constexpr (I < 3) step_sums<I + 1>(Rb, swap, B, S, acc);
+}
+
 __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
                                            const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
     const int lane = threadIdx.x & 31;
@@ -387,26 +417,7 @@ __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) B[rh][jj] = Bc[rh][jj] + T.tb;
     float acc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t w4[4];
-        w4[0] = swap ? R.d[i].z : R.d[i].x;
-        w4[1] = swap ? R.d[i].w : R.d[i].y;
-        w4[2] = swap ? R.d[i].x : R.d[i].z;
-        w4[3] = swap ? R.d[i].y : R.d[i].w;
-        float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                // odd registers sit in the upper half of each entry row: offset 128
-                const uint32_t addr = prmt(w4[r], B[r >> 1][jj], S[jj]);
-                const float v = (r & 1) ? lds_f32_off<128>(addr) : lds_f32_off<0>(addr);
-                if (jj & 1) a1 += v; else a0 += v;
-            }
-        }
-        acc[i] = a0 + a1;
-    }
+    step_sums<0>(R, swap, B, S, acc);
     // Transpose-reduce over the 4 lanes of a row group (gam = lane bits 0-1):
     // afterwards lane gam of group rho holds the slice sum of row 4*rho + gam,
     // i.e. lane l holds row l of the rowblock.
