@@ -16,44 +16,56 @@
 // |T[m, .]| <= max_k |l_k| * sum_j |g_j x[m, j]|, so T never overflows fp16 and
 // keeps fp16's relative precision.  Stage 2 divides c_m out again.
 //
-// Kernel shape: one CTA per SM, persistent over 128 x 256 output tiles,
-// warp-specialised: warp 0 issues TMA loads of A, warp 1 allocates TMEM and
-// issues the MMAs (one thread), warps 4-7 drain the double-buffered TMEM
-// accumulator, warps 8-11 expand B.  Four pipeline stages of
-// (A 16 KB + B 32 KB) in shared memory, synchronised with mbarriers.
-// Every wait is bounded: on time-out the kernel records LB_ERR_TIMEOUT, lets
-// every role finish, frees its TMEM and returns.
+// Kernel shape: one CTA per SM, persistent over output tiles of MT x 128 rows
+// by 256 columns (MT = 1 or 2 M sub-tiles share each expanded B tile, so with
+// MT = 2 a B tile is expanded once per 256 output rows).  Warp-specialised:
+// warps 0-7 drain the TMEM accumulators, warp 8 issues the TMA loads of A,
+// warp 9 allocates TMEM and issues the MMAs (one thread), warps 10-17 expand
+// B.  TMEM holds 512 fp32 columns: two 256-column accumulators, used as a
+// double buffer (MT = 1) or as the two M sub-tiles of one tile (MT = 2).
+// Pipeline stages of (A MT x 16 KB + B 32 KB) in shared memory, synchronised
+// with mbarriers.  Every wait is bounded: on time-out the kernel records
+// LB_ERR_TIMEOUT, lets every role finish, frees its TMEM and returns.
 #include <cuda.h>
+
+#include <cstdlib>
 
 #include "lb_internal.cuh"
 
 namespace lb {
 namespace {
 
-constexpr int kTileM = 128;
+constexpr int kTileM = 128;                       // rows of one M sub-tile (one MMA)
 constexpr int kTileN = 256;
 constexpr int kBlockK = 64;                       // fp16 elements per stage (128 bytes)
-constexpr int kStages = 4;
-constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB
+constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB per M sub-tile
 constexpr int kBBytes = kTileN * kBlockK * 2;     // 32 KB
 constexpr int kGBytes = kBlockK * 2;              // g slice of the K block (stage 1)
-constexpr int kStageBytes = kABytes + kBBytes + 1024;   // keeps every tile 1024-aligned
-constexpr int kPrefillThreads = 512;              // 16 warps
-constexpr int kEpiWarp0 = 0;                      // warps 0..3 drain TMEM (lane quarter = warp)
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kExpandWarp0 = 8;                   // warps 8..15 expand B, one row per thread
-constexpr int kExpandThreads = 256;
+constexpr int kPrefillThreads = 576;              // 18 warps
+constexpr int kEpiWarps = 8;                      // warps 0..7 drain TMEM (lane quarter = warp & 3)
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kExpandWarp0 = 10;                  // warps 10..17 expand B, one row per thread
+constexpr int kExpandWarps = 8;
 constexpr int kTmemCols = 512;                    // two 256-column accumulators
 constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
-constexpr int kPrefillSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kMaxStages = 4;
+
+template <int MT>
+struct Shape {
+    static constexpr int kStageBytes = MT * kABytes + kBBytes + 1024;   // keeps tiles 1024-aligned
+    static constexpr int kStages = MT == 1 ? 4 : 3;
+    static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kBufs = 2 / MT;                                // accumulator buffers
+};
+static_assert(Shape<1>::kSmem <= 232448 && Shape<2>::kSmem <= 232448, "shared memory");
 
 // ------------------------------------------------------------------ PTX
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 struct Ctl {                 // shared control block
-    uint64_t full_a[kStages], full_b[kStages], empty[kStages];
+    uint64_t full_a[kMaxStages], full_b[kMaxStages], empty[kMaxStages];
     uint64_t acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
@@ -210,8 +222,11 @@ __device__ __forceinline__ uint2 load_bits(const PrefillGemm& g, int branch, int
     return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + off));
 }
 
+template <int MT>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ PrefillGemm g) {
+    using S = Shape<MT>;
+    constexpr int kStages = S::kStages, kStageBytes = S::kStageBytes;
     extern __shared__ __align__(1024) unsigned char dsm[];
     const uint32_t raw = smem_u32(dsm);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -220,19 +235,19 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
-    const int n_tiles = ((g.M + kTileM - 1) / kTileM) * g.n_nseg * nt_per_seg;
+    const int n_tiles = ((g.M + MT * kTileM - 1) / (MT * kTileM)) * g.n_nseg * nt_per_seg;
     const int kb_per_seg = g.k_seg_len / kBlockK;
     const int n_kb = g.n_kseg * kb_per_seg;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&ctl->full_a[s]), 1);
-            mbar_init(smem_u32(&ctl->full_b[s]), kExpandThreads);
+            mbar_init(smem_u32(&ctl->full_b[s]), kExpandWarps);
             mbar_init(smem_u32(&ctl->empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&ctl->acc_full[i]), 1);
-            mbar_init(smem_u32(&ctl->acc_empty[i]), 128);
+            mbar_init(smem_u32(&ctl->acc_empty[i]), kEpiWarps);
         }
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -262,14 +277,16 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                     const int kseg = kb / kb_per_seg;
                     const int kloc = (kb - kseg * kb_per_seg) * kBlockK;
                     const int kcol = kseg * g.k_seg_len + kloc;
+                    const uint32_t sa = base + s * kStageBytes;
                     if (g.stage == 1) {
-                        mbar_expect_tx(fb, kABytes + kGBytes);
-                        bulk_load(base + s * kStageBytes + kABytes + kBBytes,
-                                  g.bscale[nseg] + kloc, kGBytes, fb);
+                        mbar_expect_tx(fb, MT * kABytes + kGBytes);
+                        bulk_load(sa + MT * kABytes + kBBytes, g.bscale[nseg] + kloc, kGBytes, fb);
                     } else {
-                        mbar_expect_tx(fb, kABytes);
+                        mbar_expect_tx(fb, MT * kABytes);
                     }
-                    tma_load_2d(base + s * kStageBytes, &amap, fb, kcol, mb * kTileM);
+#pragma unroll
+                    for (int j = 0; j < MT; ++j)
+                        tma_load_2d(sa + j * kABytes, &amap, fb, kcol, (mb * MT + j) * kTileM);
                 }
             }
         }
@@ -278,10 +295,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         if (lane == 0) {
             int it = 0, tl = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x, ++tl) {
-                const int buf = tl & 1;
-                if (!wait_bar(ctl, &ctl->acc_empty[buf], ((tl >> 1) & 1) ^ 1, g.err)) break;
+                const int buf = tl % S::kBufs;
+                const uint32_t use = (uint32_t)(tl / S::kBufs);
+                if (!wait_bar(ctl, &ctl->acc_empty[buf], (use & 1) ^ 1, g.err)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(buf * kTileN);
+                const uint32_t d = tmem + (uint32_t)(buf * MT * kTileN);
                 bool ok = true;
                 for (int kb = 0; kb < n_kb; ++kb, ++it) {
                     const int s = it % kStages;
@@ -290,75 +308,94 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                         !wait_bar(ctl, &ctl->full_b[s], par, g.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_s = base + s * kStageBytes;
-                    const uint64_t ad = sw128_desc(a_s), bd = sw128_desc(a_s + kABytes);
+                    const uint64_t bd = sw128_desc(a_s + MT * kABytes);
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; ++kk)
-                        mma_f16(d, ad + 2ull * kk, bd + 2ull * kk, (kb | kk) != 0);
+#pragma unroll
+                        for (int j = 0; j < MT; ++j)
+                            mma_f16(d + (uint32_t)(j * kTileN), sw128_desc(a_s + j * kABytes) + 2ull * kk,
+                                    bd + 2ull * kk, (kb | kk) != 0);
                     mma_commit(smem_u32(&ctl->empty[s]));
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(&ctl->acc_full[buf]));
             }
         }
-    } else if (warp < kEpiWarp0 + 4) {
-        // ---------------- epilogue: TMEM -> registers -> global
-        const int q = warp - kEpiWarp0;              // TMEM lane quarter
+    } else if (warp < kEpiWarps) {
+        // ---------------- epilogue: TMEM -> registers -> global.  Warp w reads
+        // lane quarter w & 3; with MT = 2 the upper four warps drain the second
+        // M sub-tile, with MT = 1 they take the upper 128 columns.
+        const int q = warp & 3, hw = warp >> 2;
+        const int sub = MT == 2 ? hw : 0;
+        const int c_begin = MT == 2 ? 0 : hw * (kTileN / 2);
+        const int c_end = MT == 2 ? kTileN : c_begin + kTileN / 2;
         int tl = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
             int mb, nseg, nt;
             tile_coords(g, t, mb, nseg, nt);
-            const int buf = tl & 1;
-            if (!wait_bar(ctl, &ctl->acc_full[buf], (tl >> 1) & 1, g.err)) break;
+            const int buf = tl % S::kBufs;
+            // every lane waits; the warp stops together so the .sync.aligned loads stay converged
+            if (!__all_sync(0xffffffffu, wait_bar(ctl, &ctl->acc_full[buf],
+                                                  (uint32_t)(tl / S::kBufs) & 1, g.err)))
+                break;
             tc_fence_after();
-            const int m = mb * kTileM + q * 32 + lane;
+            const int m = (mb * MT + sub) * kTileM + q * 32 + lane;
             const bool mok = m < g.M;
             const float sa = mok ? __ldg(g.row_sa + m) : 1.0f;
             const float sc = mok ? __ldg(g.row_sc + m) : 1.0f;
-            for (int c0 = 0; c0 < kTileN; c0 += 32) {
+            const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * MT + sub) * kTileN);
+            for (int c0 = c_begin; c0 < c_end; c0 += 32) {
                 float v[32];
                 __syncwarp();
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTileN + c0), v);
+                tmem_ld32(tacc + (uint32_t)c0, v);
                 const int n0 = nt * kTileN + c0;       // row within the N segment
                 if (!mok || n0 >= g.n_seg_rows) continue;
+                const bool full = n0 + 32 <= g.n_seg_rows;
                 if (g.stage == 1) {
                     // T = l * t * 2^c with t = D / 2^a
                     const float f = sc / sa;
                     __half* dst = g.T + (size_t)m * (g.n_nseg * g.n_seg_rows) +
                                   (size_t)nseg * g.n_seg_rows + n0;
                     const __half* lb = g.lscale[nseg] + n0;
-                    if (n0 + 32 <= g.n_seg_rows) {
+                    if (full && (reinterpret_cast<uintptr_t>(lb) & 15) == 0) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 8) {
+                            const uint4 lv = __ldg(reinterpret_cast<const uint4*>(lb + i));
+                            const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
                             uint32_t w[4];
 #pragma unroll
                             for (int p = 0; p < 4; ++p) {
-                                const float a0 = v[i + 2 * p] * f * __half2float(__ldg(lb + i + 2 * p));
-                                const float a1 =
-                                    v[i + 2 * p + 1] * f * __half2float(__ldg(lb + i + 2 * p + 1));
-                                const __half2 h2 = __floats2half2_rn(a0, a1);
+                                const float2 l2 = __half22float2(*reinterpret_cast<const __half2*>(&lw[p]));
+                                const __half2 h2 = __floats2half2_rn(v[i + 2 * p] * f * l2.x,
+                                                                     v[i + 2 * p + 1] * f * l2.y);
                                 w[p] = *reinterpret_cast<const uint32_t*>(&h2);
                             }
                             *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     } else {
-                        for (int i = 0; i < 32 && n0 + i < g.n_seg_rows; ++i)
-                            dst[i] = __float2half_rn(v[i] * f * __half2float(__ldg(lb + i)));
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (n0 + i < g.n_seg_rows)
+                                dst[i] = __float2half_rn(v[i] * f * __half2float(__ldg(lb + i)));
                     }
                 } else {
                     const float f = 1.0f / sc;
                     float* dst = g.y + (size_t)m * g.n_seg_rows + n0;
-                    if (n0 + 32 <= g.n_seg_rows && (g.n_seg_rows & 3) == 0) {
+                    if (full && (g.n_seg_rows & 3) == 0) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
                             *reinterpret_cast<float4*>(dst + i) =
                                 make_float4(v[i] * f, v[i + 1] * f, v[i + 2] * f, v[i + 3] * f);
                     } else {
-                        for (int i = 0; i < 32 && n0 + i < g.n_seg_rows; ++i) dst[i] = v[i] * f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (n0 + i < g.n_seg_rows) dst[i] = v[i] * f;
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
         }
     } else if (warp >= kExpandWarp0) {
         // ---------------- B producers: packed signs -> fp16 tile, one row per thread
@@ -370,36 +407,36 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             tile_coords(g, t, mb, nseg, nt);
             const int row = nt * kTileN + e;
             const bool valid = row < g.n_seg_rows;
-            uint32_t hh[2] = {0u, 0u};
+            uint32_t hh0 = 0u, hh1 = 0u;             // h[row] of each branch in both fp16 halves
             if (g.stage == 2 && valid) {
-                for (int b = 0; b < g.n_kseg; ++b) {
-                    const uint32_t hb = __half_as_ushort(__ldg(g.bscale[b] + row));
-                    hh[b] = hb | (hb << 16);
+                const uint32_t h0 = __half_as_ushort(__ldg(g.bscale[0] + row));
+                hh0 = h0 | (h0 << 16);
+                if (g.n_kseg > 1) {
+                    const uint32_t h1 = __half_as_ushort(__ldg(g.bscale[1] + row));
+                    hh1 = h1 | (h1 << 16);
                 }
             }
-            const int br0 = g.stage == 1 ? nseg : 0;
-            uint2 nxt = load_bits(g, br0, row, 0);
+            // sign bits of K block kb, fetched two blocks ahead
+            auto bits_of = [&](int kb) {
+                const int ks = kb / kb_per_seg;
+                return load_bits(g, g.stage == 1 ? nseg : ks, row, kb - ks * kb_per_seg);
+            };
+            uint2 nx0 = bits_of(0);
+            uint2 nx1 = n_kb > 1 ? bits_of(1) : make_uint2(0u, 0u);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
                 const int s = it % kStages;
-                const int kseg = kb / kb_per_seg;
-                const int klocb = kb - kseg * kb_per_seg;
-                const int branch = g.stage == 1 ? nseg : kseg;
-                const uint2 cur = nxt;
-                if (kb + 1 < n_kb) {
-                    const int ks1 = (kb + 1) / kb_per_seg;
-                    nxt = load_bits(g, g.stage == 1 ? nseg : ks1, row, kb + 1 - ks1 * kb_per_seg);
-                }
-                if (!wait_bar(ctl, &ctl->empty[s], ((it / kStages) & 1) ^ 1, g.err)) { ok = false; break; }
-                if (g.stage == 1 && !wait_bar(ctl, &ctl->full_a[s], (it / kStages) & 1, g.err)) {
-                    ok = false;
-                    break;
-                }
-                (void)klocb;
-                const uint32_t sb = base + s * kStageBytes;
-                expand_row(sb + kABytes, sb + kABytes + kBBytes, e, cur, valid, g.stage == 1,
-                           hh[branch & 1]);
+                const int branch = g.stage == 1 ? nseg : kb / kb_per_seg;
+                const uint2 cur = nx0;
+                nx0 = nx1;
+                if (kb + 2 < n_kb) nx1 = bits_of(kb + 2);
+                bool w = wait_bar(ctl, &ctl->empty[s], ((it / kStages) & 1) ^ 1, g.err);
+                if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], (it / kStages) & 1, g.err);
+                if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+                const uint32_t sb = base + s * kStageBytes + MT * kABytes;
+                expand_row(sb, sb + kBBytes, e, cur, valid, g.stage == 1, (branch & 1) ? hh1 : hh0);
                 fence_async_smem();                  // make the stores visible to the tensor core
-                mbar_arrive(smem_u32(&ctl->full_b[s]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl->full_b[s]));
             }
         }
     }
@@ -535,8 +572,11 @@ bool make_amap(CUtensorMap* map, const __half* ptr, int rows, int cols) {
 }  // namespace
 
 cudaError_t prefill_configure() {
-    return cudaFuncSetAttribute(prefill_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kPrefillSmem);
+    cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<1>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Shape<1>::kSmem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(prefill_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Shape<2>::kSmem);
 }
 
 size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
@@ -548,6 +588,35 @@ size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
 bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
     return M >= 1 && in % kBlockK == 0 && r % kBlockK == 0 && out >= 1 && in <= (1 << 20) &&
            r <= (1 << 16) && out <= (1 << 24) && M <= (1 << 24);
+}
+
+// Sub-tiles per B tile: two halve the sign expansion per MMA but double the
+// tile, so on few tiles the coarser grain can cost a round of the persistent
+// grid.  Pick the shape with the smaller estimated time, a two-sub-tile tile
+// costing kTile2Cost one-sub-tile tiles.  LB_PREFILL_SUBTILES=1 or 2 in the
+// environment (read on every call) fixes the choice; both give the same result.
+static int pick_subtiles(const PrefillGemm& p, int grid) {
+    constexpr double kTile2Cost = 1.35;
+    if (const char* env = std::getenv("LB_PREFILL_SUBTILES")) {
+        if (env[0] == '1' && env[1] == 0) return 1;
+        if (env[0] == '2' && env[1] == 0) return 2;
+    }
+    if (p.M <= kTileM) return 1;
+    const long long nt = (long long)p.n_nseg * ((p.n_seg_rows + kTileN - 1) / kTileN);
+    const long long t1 = nt * ((p.M + kTileM - 1) / kTileM);
+    const long long t2 = nt * ((p.M + 2 * kTileM - 1) / (2 * kTileM));
+    const double c1 = (double)((t1 + grid - 1) / grid);
+    const double c2 = (double)((t2 + grid - 1) / grid) * kTile2Cost;
+    return c2 < c1 ? 2 : 1;
+}
+
+static cudaError_t launch_gemm(const CUtensorMap& amap, const PrefillGemm& p, int grid,
+                               cudaStream_t s) {
+    if (pick_subtiles(p, grid) == 2)
+        prefill_gemm_kernel<2><<<grid, kPrefillThreads, Shape<2>::kSmem, s>>>(amap, p);
+    else
+        prefill_gemm_kernel<1><<<grid, kPrefillThreads, Shape<1>::kSmem, s>>>(amap, p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int64_t out,
@@ -594,8 +663,7 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
             p.lscale[b] = reinterpret_cast<const __half*>(B.l);
         }
         p.row_sa = sa; p.row_sc = sc; p.T = T; p.y = nullptr; p.err = &hdr->error;
-        prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_gemm(amap, p, grid, s)) != cudaSuccess) return e;
     }
     // stage 2: y = (T) (h o sign U)^T over K = nb * r, epilogue divides 2^c out
     {
@@ -614,8 +682,7 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
             p.lscale[b] = nullptr;
         }
         p.row_sa = sa; p.row_sc = sc; p.T = nullptr; p.y = y; p.err = &hdr->error;
-        prefill_gemm_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(amap, p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_gemm(amap, p, grid, s)) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -113,6 +113,18 @@ def test_prefill_path_shapes(shape, M, layout):
     assert_close(got, ref, what=f"{shape} M={M}")
 
 
+@pytest.mark.parametrize("subtiles", ["1", "2"])
+@pytest.mark.parametrize("M", [129, 300, 520])
+@pytest.mark.parametrize("shape", [(640, 1000, 192), (1024, 1001, 128)])
+def test_prefill_subtile_shapes(shape, M, subtiles, monkeypatch):
+    """Both tile shapes of the tensor-core GEMMs (one or two 128-row M sub-tiles per
+    expanded sign tile), with M ragged inside the first or second sub-tile."""
+    monkeypatch.setenv("LB_PREFILL_SUBTILES", subtiles)
+    in_f, out_f, r = shape
+    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=7, layout=lb.LB_LAYOUT_SLICES)
+    assert_close(got, ref, what=f"{shape} M={M} sub-tiles={subtiles}")
+
+
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
 def test_prefill_path_dtypes_and_one_branch(dtype):
     got, ref = run_case(768, 512, 128, 64, dtype, nb=1, base=4)
