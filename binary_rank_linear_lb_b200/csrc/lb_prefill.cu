@@ -49,13 +49,24 @@ constexpr int kExpandWarp0 = 10;                  // warps 10..17 expand B, one 
 constexpr int kExpandWarps = 8;
 constexpr int kTmemCols = 512;                    // two 256-column accumulators
 constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
+constexpr uint32_t kSuspendNs = 20000;            // longest hardware suspension per try_wait
 constexpr int kMaxStages = 4;
 
+constexpr int kEpiBytes = 32 * 128;                // per-warp epilogue staging: 32 rows x 128 bytes
+constexpr int kPrefetchAhead = 6;                 // K blocks of A pulled into L2 ahead of the TMA loads
+constexpr int kBitsAhead = 4;                     // K blocks of sign bits held in registers ahead
+
+// Shared memory of one CTA, from the 1024-aligned base: the pipeline stages
+// (A sub-tiles then the B tile, each 1024-aligned), the epilogue staging
+// buffers, the g slices of the stages (stage 1), the control block.
 template <int MT>
 struct Shape {
-    static constexpr int kStageBytes = MT * kABytes + kBBytes + 1024;   // keeps tiles 1024-aligned
+    static constexpr int kStageBytes = MT * kABytes + kBBytes;
     static constexpr int kStages = MT == 1 ? 4 : 3;
-    static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kOffEpi = kStages * kStageBytes;
+    static constexpr int kOffG = kOffEpi + kEpiWarps * kEpiBytes;
+    static constexpr int kOffCtl = kOffG + kStages * kGBytes;
+    static constexpr int kSmem = kOffCtl + 256 /*barriers*/ + 1024 /*align*/;
     static constexpr int kBufs = 2 / MT;                                // accumulator buffers
 };
 static_assert(Shape<1>::kSmem <= 232448 && Shape<2>::kSmem <= 232448, "shared memory");
@@ -73,12 +84,24 @@ struct Ctl {                 // shared control block
 
 // Bounded wait on an mbarrier phase; on time-out raises the CTA abort flag
 // and the workspace error.  Returns false if the caller must stop.
+// try_wait that may suspend the thread in hardware for up to `ns` nanoseconds;
+// it resumes when the phase completes, so a waiting warp takes no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool wait_bar(Ctl* c, uint64_t* bar, uint32_t parity, int* err) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(a, parity)) return true;
+        if (mbar_try_wait_sleep(a, parity, kSuspendNs)) return true;
         if (*reinterpret_cast<volatile int*>(&c->abort)) return false;
         if (clock64() - t0 > kWaitLimit) {
             atomicExch(&c->abort, 1);
@@ -86,6 +109,12 @@ __device__ __forceinline__ bool wait_bar(Ctl* c, uint64_t* bar, uint32_t parity,
             return false;
         }
     }
+}
+
+// Pull one A box into L2 (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 :: "l"(map), "r"(x), "r"(y) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -183,20 +212,25 @@ __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb
 
 // Expand row n of one 256 x 64 B tile (K-major, 128-byte swizzle) from its 64
 // packed sign bits.  Element k is the scale with its sign bit flipped when the
-// bit is set: stage 1 scales per k (g slice staged in shared memory next to
-// the tile), stage 2 per row (hh = h[row] in both halves).  Bits of a byte are
-// spread to the top bit of each byte of a word by one multiply, and PRMT moves
-// two of them to bits 15 and 31 of the fp16 pair they sign.
+// bit is set: stage 1 scales per k (g slice staged in shared memory), stage 2
+// per row (hh = h[row] in both halves).  Per 16-byte piece (8 elements): one
+// multiply spreads four sign bits to the top bits of the four bytes of a word
+// (bit i to bit 8i + 7; the partial products never overlap, so nothing
+// carries); PRMT in sign-replicating mode copies the top bit of byte 2p and
+// 2p + 1 over bytes 0-1 and 2-3 of the fp16 pair p; one LOP3 keeps bits 15
+// and 31 of that and flips them into the scales.  Rows past the matrix are
+// expanded from whatever bits they get: only output columns that are never
+// stored read them.
 __device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int n, uint2 bits,
-                                           bool valid, bool per_k, uint32_t hh) {
-    const uint32_t rowoff = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 128u;
+                                           bool per_k, uint32_t hh) {
+    // 16-byte piece c of row n sits at slot c ^ (n & 7) of the row's 128 bytes
+    const uint32_t rowx = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 144u;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {                    // 16-byte chunk: k = 8c .. 8c+7
-        const uint32_t byte = ((c < 4 ? bits.x : bits.y) >> (8 * (c & 3))) & 0xFFu;
-        const uint32_t rlo = ((byte & 0xFu) * 0x10204080u) & 0x80808080u;
-        const uint32_t rhi = ((byte >> 4) * 0x10204080u) & 0x80808080u;
-        const uint32_t m0 = prmt(rlo, 0u, 0x1404u), m1 = prmt(rlo, 0u, 0x3424u);
-        const uint32_t m2 = prmt(rhi, 0u, 0x1404u), m3 = prmt(rhi, 0u, 0x3424u);
+    for (int c = 0; c < 8; ++c) {                    // k = 8c .. 8c+7
+        const uint32_t word = c < 4 ? bits.x : bits.y;
+        const uint32_t byte = c & 3 ? (word >> (8 * (c & 3))) & 0xFFu : word & 0xFFu;
+        const uint32_t slo = (byte & 0xFu) * 0x10204080u;
+        const uint32_t shi = (byte >> 4) * 0x10204080u;
         uint4 base;
         if (per_k) {
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -205,9 +239,11 @@ __device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int
         } else {
             base = make_uint4(hh, hh, hh, hh);
         }
-        const uint32_t o0 = valid ? base.x ^ m0 : 0u, o1 = valid ? base.y ^ m1 : 0u;
-        const uint32_t o2 = valid ? base.z ^ m2 : 0u, o3 = valid ? base.w ^ m3 : 0u;
-        const uint32_t addr = b_smem + rowoff + (uint32_t)((c ^ (n & 7)) * 16);
+        const uint32_t o0 = base.x ^ (prmt(slo, 0u, 0x9988u) & 0x80008000u);
+        const uint32_t o1 = base.y ^ (prmt(slo, 0u, 0xBBAAu) & 0x80008000u);
+        const uint32_t o2 = base.z ^ (prmt(shi, 0u, 0x9988u) & 0x80008000u);
+        const uint32_t o3 = base.w ^ (prmt(shi, 0u, 0xBBAAu) & 0x80008000u);
+        const uint32_t addr = b_smem + (rowx ^ (uint32_t)(c * 16));
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                      :: "r"(addr), "r"(o0), "r"(o1), "r"(o2), "r"(o3) : "memory");
     }
@@ -231,7 +267,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     const uint32_t raw = smem_u32(dsm);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* basep = dsm + (base - raw);
-    Ctl* ctl = reinterpret_cast<Ctl*>(basep + kStages * kStageBytes);
+    Ctl* ctl = reinterpret_cast<Ctl*>(basep + S::kOffCtl);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
@@ -263,24 +299,42 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp == kTmaWarp) {
-        // ---------------- TMA producer for A (and the g slice of stage 1)
+        // ---------------- TMA producer for A (and the g slice of stage 1).  A
+        // boxes kPrefetchAhead K blocks ahead (into the next tile at the end of
+        // one) are pulled into L2 first, so the loads find them there.
         if (lane == 0) {
+            auto acol = [&](int kb) {
+                const int ks = kb / kb_per_seg;
+                return ks * g.k_seg_len + (kb - ks * kb_per_seg) * kBlockK;
+            };
+            auto prefetch = [&](int t, int kb) {
+                int pb = kb + kPrefetchAhead;
+                if (pb >= n_kb) { t += gridDim.x; pb -= n_kb; }
+                if (t >= n_tiles || pb >= n_kb) return;
+                int mb, nseg, nt;
+                tile_coords(g, t, mb, nseg, nt);
+#pragma unroll
+                for (int j = 0; j < MT; ++j)
+                    if ((mb * MT + j) * kTileM < g.M) tma_prefetch_2d(&amap, acol(pb), (mb * MT + j) * kTileM);
+            };
+            if (blockIdx.x < n_tiles)
+                for (int kb = -kPrefetchAhead; kb < 0; ++kb) prefetch(blockIdx.x, kb);
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
                 int mb, nseg, nt;
                 tile_coords(g, t, mb, nseg, nt);
                 for (int kb = 0; kb < n_kb; ++kb, ++it) {
+                    prefetch(t, kb);
                     const int s = it % kStages;
                     const uint32_t par = ((it / kStages) & 1) ^ 1;
                     if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) break;
                     const uint32_t fb = smem_u32(&ctl->full_a[s]);
-                    const int kseg = kb / kb_per_seg;
-                    const int kloc = (kb - kseg * kb_per_seg) * kBlockK;
-                    const int kcol = kseg * g.k_seg_len + kloc;
+                    const int kcol = acol(kb);
                     const uint32_t sa = base + s * kStageBytes;
                     if (g.stage == 1) {
+                        const int kloc = kcol - (kb / kb_per_seg) * g.k_seg_len;
                         mbar_expect_tx(fb, MT * kABytes + kGBytes);
-                        bulk_load(sa + MT * kABytes + kBBytes, g.bscale[nseg] + kloc, kGBytes, fb);
+                        bulk_load(base + S::kOffG + s * kGBytes, g.bscale[nseg] + kloc, kGBytes, fb);
                     } else {
                         mbar_expect_tx(fb, MT * kABytes);
                     }
@@ -322,13 +376,20 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             }
         }
     } else if (warp < kEpiWarps) {
-        // ---------------- epilogue: TMEM -> registers -> global.  Warp w reads
-        // lane quarter w & 3; with MT = 2 the upper four warps drain the second
-        // M sub-tile, with MT = 1 they take the upper 128 columns.
+        // ---------------- epilogue: TMEM -> registers -> shared staging -> global.
+        // Warp w reads lane quarter w & 3; with MT = 2 the upper four warps drain
+        // the second M sub-tile, with MT = 1 they take the upper 128 columns.
+        // Each 32 x 32 chunk is scaled in registers (lane = row), written to
+        // the warp's staging buffer (16-byte piece c of row r at slot c ^ (r & 7),
+        // conflict-free both ways) and read back so that every store
+        // instruction writes whole row segments (128 bytes of y, 64 of T).
         const int q = warp & 3, hw = warp >> 2;
         const int sub = MT == 2 ? hw : 0;
         const int c_begin = MT == 2 ? 0 : hw * (kTileN / 2);
         const int c_end = MT == 2 ? kTileN : c_begin + kTileN / 2;
+        const uint32_t stg = base + S::kOffEpi + (uint32_t)warp * kEpiBytes;
+        const uint32_t my_row = stg + (uint32_t)lane * 128u;
+        const int ldt = g.n_nseg * g.n_seg_rows;          // T row pitch (stage 1)
         int tl = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
             int mb, nseg, nt;
@@ -339,59 +400,101 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                                                   (uint32_t)(tl / S::kBufs) & 1, g.err)))
                 break;
             tc_fence_after();
-            const int m = (mb * MT + sub) * kTileM + q * 32 + lane;
+            const int m0 = (mb * MT + sub) * kTileM + q * 32;     // first row of this warp
+            const int m = m0 + lane;
             const bool mok = m < g.M;
             const float sa = mok ? __ldg(g.row_sa + m) : 1.0f;
             const float sc = mok ? __ldg(g.row_sc + m) : 1.0f;
+            const float f = g.stage == 1 ? sc / sa : 1.0f / sc;
             const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * MT + sub) * kTileN);
             for (int c0 = c_begin; c0 < c_end; c0 += 32) {
                 float v[32];
                 __syncwarp();
                 tmem_ld32(tacc + (uint32_t)c0, v);
                 const int n0 = nt * kTileN + c0;       // row within the N segment
-                if (!mok || n0 >= g.n_seg_rows) continue;
-                const bool full = n0 + 32 <= g.n_seg_rows;
+                if (n0 >= g.n_seg_rows) continue;      // warp-uniform
                 if (g.stage == 1) {
-                    // T = l * t * 2^c with t = D / 2^a
-                    const float f = sc / sa;
-                    __half* dst = g.T + (size_t)m * (g.n_nseg * g.n_seg_rows) +
-                                  (size_t)nseg * g.n_seg_rows + n0;
+                    // T = l * t * 2^c with t = D / 2^a, fp16, 4 pieces of 16 bytes per row
                     const __half* lb = g.lscale[nseg] + n0;
-                    if (full && (reinterpret_cast<uintptr_t>(lb) & 15) == 0) {
+                    const bool lvec = n0 + 32 <= g.n_seg_rows && (reinterpret_cast<uintptr_t>(lb) & 15) == 0;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            const uint4 lv = __ldg(reinterpret_cast<const uint4*>(lb + i));
-                            const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-                            uint32_t w[4];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w[4];
+                        uint4 lv;
+                        if (lvec) {
+                            lv = __ldg(reinterpret_cast<const uint4*>(lb + 8 * c));
+                        } else {
+                            uint16_t e8[8];
 #pragma unroll
-                            for (int p = 0; p < 4; ++p) {
-                                const float2 l2 = __half22float2(*reinterpret_cast<const __half2*>(&lw[p]));
-                                const __half2 h2 = __floats2half2_rn(v[i + 2 * p] * f * l2.x,
-                                                                     v[i + 2 * p + 1] * f * l2.y);
-                                w[p] = *reinterpret_cast<const uint32_t*>(&h2);
-                            }
-                            *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                            for (int i = 0; i < 8; ++i)
+                                e8[i] = n0 + 8 * c + i < g.n_seg_rows ? __half_as_ushort(__ldg(lb + 8 * c + i)) : 0;
+                            lv = make_uint4(e8[0] | (uint32_t)e8[1] << 16, e8[2] | (uint32_t)e8[3] << 16,
+                                            e8[4] | (uint32_t)e8[5] << 16, e8[6] | (uint32_t)e8[7] << 16);
                         }
-                    } else {
+                        const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (n0 + i < g.n_seg_rows)
-                                dst[i] = __float2half_rn(v[i] * f * __half2float(__ldg(lb + i)));
+                        for (int p = 0; p < 4; ++p) {
+                            const float2 l2 = __half22float2(*reinterpret_cast<const __half2*>(&lw[p]));
+                            const __half2 h2 = __floats2half2_rn(v[8 * c + 2 * p] * f * l2.x,
+                                                                 v[8 * c + 2 * p + 1] * f * l2.y);
+                            w[p] = *reinterpret_cast<const uint32_t*>(&h2);
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(my_row + (uint32_t)((c ^ (lane & 7)) * 16)),
+                                        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+                    }
+                    __syncwarp();
+                    const int cc = lane & 3;
+                    const int col = n0 + 8 * cc;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {              // rows 8i .. 8i+7, 4 lanes per row
+                        const int rr = 8 * i + (lane >> 2);
+                        uint4 o;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+                                     : "r"(stg + (uint32_t)rr * 128u + (uint32_t)((cc ^ (rr & 7)) * 16)));
+                        if (m0 + rr < g.M && col < g.n_seg_rows) {
+                            __half* dst = g.T + (size_t)(m0 + rr) * ldt + (size_t)nseg * g.n_seg_rows + col;
+                            if (col + 8 <= g.n_seg_rows) {
+                                *reinterpret_cast<uint4*>(dst) = o;
+                            } else {
+                                const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+                                for (int e = 0; e < 8 && col + e < g.n_seg_rows; ++e)
+                                    reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(ow[e >> 1] >> (16 * (e & 1)));
+                            }
+                        }
                     }
                 } else {
-                    const float f = 1.0f / sc;
-                    float* dst = g.y + (size_t)m * g.n_seg_rows + n0;
-                    if (full && (g.n_seg_rows & 3) == 0) {
+                    // y = D / 2^c, fp32, 8 pieces of 16 bytes per row
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(dst + i) =
-                                make_float4(v[i] * f, v[i + 1] * f, v[i + 2] * f, v[i + 3] * f);
-                    } else {
+                    for (int c = 0; c < 8; ++c)
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(my_row + (uint32_t)((c ^ (lane & 7)) * 16)),
+                                        "f"(v[4 * c] * f), "f"(v[4 * c + 1] * f), "f"(v[4 * c + 2] * f),
+                                        "f"(v[4 * c + 3] * f) : "memory");
+                    __syncwarp();
+                    const int cc = lane & 7;
+                    const int col = n0 + 4 * cc;
+                    const bool vec = (g.n_seg_rows & 3) == 0;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (n0 + i < g.n_seg_rows) dst[i] = v[i] * f;
+                    for (int i = 0; i < 8; ++i) {              // rows 4i .. 4i+3, 8 lanes per row
+                        const int rr = 4 * i + (lane >> 3);
+                        float4 o;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(o.x), "=f"(o.y), "=f"(o.z), "=f"(o.w)
+                                     : "r"(stg + (uint32_t)rr * 128u + (uint32_t)((cc ^ (rr & 7)) * 16)));
+                        if (m0 + rr < g.M && col < g.n_seg_rows) {
+                            float* dst = g.y + (size_t)(m0 + rr) * g.n_seg_rows + col;
+                            if (vec) {
+                                *reinterpret_cast<float4*>(dst) = o;
+                            } else {
+                                const float ov[4] = {o.x, o.y, o.z, o.w};
+                                for (int e = 0; e < 4 && col + e < g.n_seg_rows; ++e) dst[e] = ov[e];
+                            }
+                        }
                     }
                 }
+                __syncwarp();                          // staging buffer free for the next chunk
             }
             tc_fence_before();
             __syncwarp();
@@ -400,15 +503,15 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     } else if (warp >= kExpandWarp0) {
         // ---------------- B producers: packed signs -> fp16 tile, one row per thread
         const int e = threadIdx.x - kExpandWarp0 * 32;
-        int it = 0;
+        int s = 0;                                   // pipeline slot of the current K block
+        uint32_t ph = 0;                             // and the parity of its current use
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             int mb, nseg, nt;
             tile_coords(g, t, mb, nseg, nt);
             const int row = nt * kTileN + e;
-            const bool valid = row < g.n_seg_rows;
             uint32_t hh0 = 0u, hh1 = 0u;             // h[row] of each branch in both fp16 halves
-            if (g.stage == 2 && valid) {
+            if (g.stage == 2 && row < g.n_seg_rows) {
                 const uint32_t h0 = __half_as_ushort(__ldg(g.bscale[0] + row));
                 hh0 = h0 | (h0 << 16);
                 if (g.n_kseg > 1) {
@@ -416,27 +519,37 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                     hh1 = h1 | (h1 << 16);
                 }
             }
-            // sign bits of K block kb, fetched two blocks ahead
-            auto bits_of = [&](int kb) {
-                const int ks = kb / kb_per_seg;
-                return load_bits(g, g.stage == 1 ? nseg : ks, row, kb - ks * kb_per_seg);
+            // sign bits, fetched kBitsAhead K blocks ahead into a register ring;
+            // (fs, fk) = K segment and block within it of the next fetch
+            int fs = 0, fk = 0;
+            auto fetch = [&]() {
+                const uint2 v = load_bits(g, g.stage == 1 ? nseg : fs, row, fk);
+                if (++fk == kb_per_seg) { fk = 0; ++fs; }
+                return v;
             };
-            uint2 nx0 = bits_of(0);
-            uint2 nx1 = n_kb > 1 ? bits_of(1) : make_uint2(0u, 0u);
-            for (int kb = 0; kb < n_kb; ++kb, ++it) {
-                const int s = it % kStages;
-                const int branch = g.stage == 1 ? nseg : kb / kb_per_seg;
-                const uint2 cur = nx0;
-                nx0 = nx1;
-                if (kb + 2 < n_kb) nx1 = bits_of(kb + 2);
-                bool w = wait_bar(ctl, &ctl->empty[s], ((it / kStages) & 1) ^ 1, g.err);
-                if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], (it / kStages) & 1, g.err);
-                if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-                const uint32_t sb = base + s * kStageBytes + MT * kABytes;
-                expand_row(sb, sb + kBBytes, e, cur, valid, g.stage == 1, (branch & 1) ? hh1 : hh0);
-                fence_async_smem();                  // make the stores visible to the tensor core
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl->full_b[s]));
+            uint2 nx[kBitsAhead];
+#pragma unroll
+            for (int j = 0; j < kBitsAhead; ++j) nx[j] = j < n_kb ? fetch() : make_uint2(0u, 0u);
+            int seg = 0, kin = 0;                    // K segment of the current block, block within it
+            for (int kb0 = 0; kb0 < n_kb && ok; kb0 += kBitsAhead) {
+#pragma unroll
+                for (int j = 0; j < kBitsAhead; ++j) {
+                    const int kb = kb0 + j;
+                    if (kb >= n_kb) break;
+                    const uint2 cur = nx[j];
+                    if (kb + kBitsAhead < n_kb) nx[j] = fetch();
+                    bool w = wait_bar(ctl, &ctl->empty[s], ph ^ 1, g.err);
+                    if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, g.err);
+                    if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+                    const uint32_t sb = base + s * kStageBytes + MT * kABytes;
+                    expand_row(sb, base + S::kOffG + s * kGBytes, e, cur, g.stage == 1,
+                               (seg & 1) ? hh1 : hh0);
+                    fence_async_smem();              // make the stores visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&ctl->full_b[s]));
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                    if (++kin == kb_per_seg) { kin = 0; ++seg; }
+                }
             }
         }
     }
