@@ -19,7 +19,9 @@
 // (two slices or two matrices) as one stream.
 //
 // Lane mapping of the lookups.  Lane l = 4*rho + gam (rho = 0..7 picks one of 8
-// rows of a step, gam = 0..3 one of four 16-byte word groups of the row).  At
+// rows of a step -- row 8*step + rho of the rowblock, so that a step's 8 rows
+// are contiguous in the sliced layout -- and gam = 0..3 one of four 16-byte
+// word groups of the row).  At
 // step (r, jj) the lane reads register r of its group (with the two halves of
 // the group swapped when rho >= 4) and byte (jj + rho) % 4 of that word, so
 // the 32 lanes touch 32 chunks in 32 different banks.  A single PRMT merges the
@@ -315,8 +317,9 @@ struct Cursor {
 };
 
 // One rowblock (32 rows x 16 words of a slice) as this lane holds it: row
-// step i covers rows 4*rho + i, the lane's words 4*gam .. 4*gam+3; h is the
-// row scale of the lane's output row (row `lane` of the rowblock).
+// step i covers row 8*i + rho, the lane's words 4*gam .. 4*gam+3, so with a
+// 16-word pitch one load instruction of the warp reads 512 contiguous bytes;
+// h is the row scale of the lane's output row (row 8*gam + rho).
 struct RB {
     uint4 d[4];
     unsigned short h;   // fp16 bits, converted at use so the load does not stall the warp
@@ -338,13 +341,13 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
     const int w = 4 * gam;
     if (T.wrem == kSliceWords && (T.ldw & 3) == 0 && rb * kRowBlock + kRowBlock <= T.rows) {
         // the usual case: all 32 rows inside, full 16-word pieces
-        const uint32_t* p = T.P + (size_t)(rb * kRowBlock + 4 * rho) * (size_t)T.ldw + w;
+        const uint32_t* p = T.P + (size_t)(rb * kRowBlock + rho) * (size_t)T.ldw + w;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) R.d[i] = ld_stream_v4(p + (size_t)i * T.ldw);
+        for (int i = 0; i < 4; ++i) R.d[i] = ld_stream_v4(p + (size_t)(8 * i) * T.ldw);
     } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int row = rb * kRowBlock + 4 * rho + i;
+        const int row = rb * kRowBlock + 8 * i + rho;
         uint4 d = make_uint4(0u, 0u, 0u, 0u);
         if (row < T.rows && w < T.wrem) {
             const uint32_t* p = T.P + (size_t)row * (size_t)T.ldw + w;
@@ -369,7 +372,7 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
     }
     R.h = 0x3C00u;   // 1.0
     if (T.h != nullptr) {
-        const int orow = rb * kRowBlock + lane;
+        const int orow = rb * kRowBlock + 8 * gam + rho;
         R.h = orow < T.rows ? __ldg(reinterpret_cast<const unsigned short*>(T.h) + orow) : 0u;
     }
 }
@@ -419,8 +422,8 @@ __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
     float acc[4];
     step_sums<0>(R, swap, B, S, acc);
     // Transpose-reduce over the 4 lanes of a row group (gam = lane bits 0-1):
-    // afterwards lane gam of group rho holds the slice sum of row 4*rho + gam,
-    // i.e. lane l holds row l of the rowblock.
+    // afterwards lane gam of group rho holds the slice sum of row step gam,
+    // i.e. of row 8*gam + rho of the rowblock.
     const bool up2 = (gam & 2) != 0, up1 = (gam & 1) != 0;
     float n2[2];
 #pragma unroll
@@ -433,18 +436,20 @@ __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
     const float keep1 = up1 ? n2[1] : n2[0];
     const float tot = (keep1 + __shfl_xor_sync(0xffffffffu, send1, 1)) *
                       __half2float(__ushort_as_half(R.h));
-    // Lane 4q adds rows 4q..4q+3 with one vector reduction (the L2 takes a
-    // 16-byte reduction at the rate of a 4-byte one); partial or unaligned
-    // groups fall back to one reduction per row.
-    const float t1 = __shfl_down_sync(0xffffffffu, tot, 1);
-    const float t2 = __shfl_down_sync(0xffffffffu, tot, 2);
-    const float t3 = __shfl_down_sync(0xffffffffu, tot, 3);
-    const int g0 = rb * kRowBlock + 4 * rho;             // first row of the lane's group
+    // Rows 8*gam + 4k .. +3 sit in lanes 16k + gam + 4j (j = 0..3): the lane
+    // with j = 0 adds them with one vector reduction (the L2 takes a 16-byte
+    // reduction at the rate of a 4-byte one); partial or unaligned groups fall
+    // back to one reduction per row.
+    const float t1 = __shfl_down_sync(0xffffffffu, tot, 4);
+    const float t2 = __shfl_down_sync(0xffffffffu, tot, 8);
+    const float t3 = __shfl_down_sync(0xffffffffu, tot, 12);
+    const int row = rb * kRowBlock + 8 * gam + rho;       // the row this lane holds
+    const int g0 = row - (rho & 3);                       // first row of its group of 4
     float* og = T.out + g0;
     if (g0 + 4 <= T.rows && (reinterpret_cast<uintptr_t>(og) & 15u) == 0) {
-        if (gam == 0) red_add_v4_f32(og, tot, t1, t2, t3);
-    } else if (g0 + gam < T.rows) {
-        red_add_f32(og + gam, tot);
+        if ((rho & 3) == 0) red_add_v4_f32(og, tot, t1, t2, t3);
+    } else if (row < T.rows) {
+        red_add_f32(T.out + row, tot);
     }
 }
 
