@@ -80,6 +80,7 @@ void plan_splits(LbPhase* phases, int n_phases, LbJob* jobs, int G, int* split) 
         phases[p].next_n_jobs = p + 1 < n_phases ? phases[p + 1].n_jobs : 0;
         phases[p].split_off = p * (kMaxGrid + 1);
         phases[p].split_g = -1;
+        phases[p].starts_g = -1;   // no start table unless plan_starts makes one
         plan_row_groups(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units,
                         std::max(G, 1));
         if (G < 1 || G > kMaxGrid) continue;
@@ -122,6 +123,7 @@ struct StackLayout {
     size_t acc_end;                  // end of the accumulator area
     size_t x_dev, y_dev;             // staging for lb_stack_forward_host
     size_t phases, jobs, splits;     // plan
+    size_t starts;                   // [phase][kMaxGrid] first batches of the CTAs
     int n_phases, n_jobs;
     size_t total;
 };
@@ -242,6 +244,8 @@ StackLayout stack_layout(const lb_stack_desc* d) {
     off = round_up(off + sizeof(LbJob) * (size_t)L.n_jobs, 256);
     L.splits = off;
     off = round_up(off + sizeof(int) * (size_t)(kMaxGrid + 1) * (size_t)L.n_phases, 256);
+    L.starts = off;
+    off = round_up(off + sizeof(LbStart) * (size_t)kMaxGrid * (size_t)L.n_phases, 256);
     L.total = off;
     return L;
 }
@@ -528,7 +532,10 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
     build_stack_plan(d, L, static_cast<char*>(workspace), phases, jobs);
     if ((int)phases.size() != L.n_phases || (int)jobs.size() != L.n_jobs) return LB_ERR_CUDA;
     std::vector<int> split((size_t)(kMaxGrid + 1) * L.n_phases, 0);
-    plan_splits(phases.data(), L.n_phases, jobs.data(), decode_grid(), split.data());
+    const int G = decode_grid();
+    plan_splits(phases.data(), L.n_phases, jobs.data(), G, split.data());
+    std::vector<LbStart> starts((size_t)kMaxGrid * L.n_phases, LbStart{});
+    plan_starts(phases.data(), L.n_phases, jobs.data(), split.data(), G, starts.data());
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
@@ -539,6 +546,9 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
     if (cudaMemcpyAsync(ws + L.splits, split.data(), sizeof(int) * split.size(),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return LB_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + L.starts, starts.data(), sizeof(LbStart) * starts.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
@@ -557,7 +567,8 @@ lb_status lb_stack_forward(const lb_stack_desc* d, void* workspace, size_t ws_by
     char* ws = static_cast<char*>(workspace);
     if (launch_stack_plan(reinterpret_cast<const LbPhase*>(ws + L.phases),
                           reinterpret_cast<const LbJob*>(ws + L.jobs),
-                          reinterpret_cast<const int*>(ws + L.splits), L.n_phases,
+                          reinterpret_cast<const int*>(ws + L.splits),
+                          reinterpret_cast<const LbStart*>(ws + L.starts), L.n_phases,
                           reinterpret_cast<WsHeader*>(ws), x, y, s) != cudaSuccess)
         return LB_ERR_CUDA;
     return LB_OK;

@@ -61,13 +61,14 @@ struct Smem {
     int* flag;        // one int
     LbPhase* phase;   // the current phase, copied from the plan
     int* range;       // this CTA's unit range in it (from the split table)
+    LbStart* start;   // this CTA's first batch of it (when the plan has a start table)
     LbJob* jobs;      // its jobs (at most kMaxPhaseJobs), copied from the plan
 };
 
-// Two plan buffers (phase header, unit range, jobs): the current phase's and
-// the next one's, which is copied in while the current phase runs.
+// Two plan buffers (phase header, unit range, first batch, jobs): the current
+// phase's and the next one's, which is copied in while the current phase runs.
 constexpr int kOffPlan = 4 * kTables * kVecPad + 4 * 32 + 64;
-constexpr int kPlanBufBytes = 64 + kMaxPhaseJobs * (int)sizeof(LbJob);
+constexpr int kPlanBufBytes = 128 + kMaxPhaseJobs * (int)sizeof(LbJob);
 static_assert(kOffPlan % 64 == 0, "plan buffers must be 64-byte aligned");
 static_assert(kOffPlan + 2 * kPlanBufBytes == kMiscBytes, "shared layout out of step");
 
@@ -80,7 +81,8 @@ __device__ __forceinline__ void use_plan_buf(Smem& s, int b) {
     unsigned char* base = dyn_smem() + kOffPlan + b * kPlanBufBytes;
     s.phase = reinterpret_cast<LbPhase*>(base);
     s.range = reinterpret_cast<int*>(base + sizeof(LbPhase));
-    s.jobs = reinterpret_cast<LbJob*>(base + 64);
+    s.start = reinterpret_cast<LbStart*>(base + 64);
+    s.jobs = reinterpret_cast<LbJob*>(base + 128);
 }
 
 __device__ __forceinline__ Smem smem_layout() {
@@ -104,13 +106,16 @@ __device__ __forceinline__ int split_index(int q) {
 // Copy phase q, its jobs and this CTA's unit range into plan buffer b, with
 // every thread of the CTA (plan data never changes during a call).
 __device__ void cache_plan(const LbPhase* phases, int q, const LbJob* jobs, const int* splits,
-                           int b) {
+                           const LbStart* starts, int b) {
     Smem s;
     use_plan_buf(s, b);
     const LbPhase ph = phases[q];
     if (threadIdx.x == 0) *s.phase = ph;
     const int si = split_index(q);
     if (threadIdx.x < 2) s.range[threadIdx.x] = si >= 0 ? splits[si + threadIdx.x] : 0;
+    if (starts != nullptr && ph.starts_g == (int)gridDim.x && threadIdx.x < 16)
+        reinterpret_cast<int*>(s.start)[threadIdx.x] =
+            reinterpret_cast<const int*>(starts + (size_t)q * kMaxGrid + blockIdx.x)[threadIdx.x];
     const int n_words = ph.n_jobs * (int)(sizeof(LbJob) / 4);
     const uint32_t* src = reinterpret_cast<const uint32_t*>(jobs + ph.job_begin);
     uint32_t* dst = reinterpret_cast<uint32_t*>(s.jobs);
@@ -129,7 +134,8 @@ __device__ __forceinline__ void cp_async(void* dst, const void* src, int bytes) 
 // memory); the job range comes from the previous phase's header.  Completed
 // by plan_wait in the same warp before a CTA barrier.
 __device__ void cache_plan_async(const LbPhase* phases, int q, int job_begin, int n_jobs,
-                                 const LbJob* jobs, const int* splits, int b) {
+                                 const LbJob* jobs, const int* splits, const LbStart* starts,
+                                 int b) {
     Smem s;
     use_plan_buf(s, b);
     const int lane = threadIdx.x & 31;
@@ -146,6 +152,11 @@ __device__ void cache_plan_async(const LbPhase* phases, int q, int job_begin, in
     }
     const int si = split_index(q);
     if (lane < 2 && si >= 0) cp_async(s.range + lane, splits + si + lane, 4);
+    // the start record (used only if the phase header says the table was made for this grid)
+    if (starts != nullptr && si >= 0 && lane >= 4 && lane < 8)
+        cp_async(reinterpret_cast<uint4*>(s.start) + (lane - 4),
+                 reinterpret_cast<const uint4*>(starts + (size_t)q * kMaxGrid + blockIdx.x) +
+                     (lane - 4), 16);
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
@@ -269,32 +280,6 @@ __device__ __forceinline__ void build_table(const float* vec, uint32_t taddr) {
 }
 
 // ---- tiles and batches ----------------------------------------------------
-__device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int u) {
-    while (j + 1 < j_end && jobs[j + 1].unit_begin <= u) ++j;
-    return j;
-}
-
-struct Tile {
-    int job, slice, rb0, nrb;
-};
-
-// The tile of this CTA's unit range that starts at unit u (u < u_end).  A
-// job's units run row group by row group, slice by slice inside a group, so
-// the CTAs holding the slices of one group stream the same rows together and
-// each DRAM page is read while it is open.
-__device__ __forceinline__ Tile next_tile(const LbJob* jobs, int n_jobs, int& j, int u, int u_end) {
-    j = find_job(jobs, j, n_jobs, u);
-    const LbJob& J = jobs[j];
-    const int local = u - J.unit_begin;
-    const int per_group = J.rg * J.n_slices;
-    const int g = local / per_group;
-    const int off = local - g * per_group;
-    const int rows_g = min(J.rg, J.n_rowblocks - g * J.rg);
-    const int s = off / rows_g;
-    const int rbi = off - s * rows_g;
-    return Tile{j, s, g * J.rg + rbi, min(rows_g - rbi, u_end - u)};
-}
-
 // What the lookup loop needs of one tile of the current batch.
 struct TileRt {
     const uint32_t* P;       // first word of the slice in row 0
@@ -311,7 +296,7 @@ struct TileRt {
 struct Cursor {
     int u, u_end, j;
     int nt, n_rb;
-    Tile t[kMaxTiles];
+    LbTile t[kMaxTiles];
     TileRt rt[kMaxTiles];
     unsigned short sc[kMaxTiles];   // fp16 bits
 };
@@ -512,8 +497,32 @@ __device__ __forceinline__ void batch_lookups(const Cursor& c, RB (&buf)[kDepth]
     }
 }
 
+// Tile k of the batch (c.t[k] set): what the lookup loop needs of it, and
+// this thread's element of its vector scale.  Reads only plan data and weights.
+__device__ __forceinline__ void tile_setup(const Smem& sm, const CallArgs& args, Cursor& c, int k) {
+    const LbTile& t = c.t[k];
+    const LbJob& J = sm.jobs[t.job];
+    TileRt& T = c.rt[k];
+    const int nw = (J.cols + 31) / 32;
+    if (J.sliced) {   // the slice is a contiguous block of rows
+        T.P = J.P + (size_t)kSliceWords * (size_t)J.rows * (size_t)t.slice;
+        T.ldw = (int)sliced_pitch(nw, t.slice);
+    } else {
+        T.P = J.P + (size_t)t.slice * kSliceWords;
+        T.ldw = J.ldw;
+    }
+    T.h = J.oscale;
+    T.out = resolve(J.out, args);
+    T.rows = J.rows;
+    T.wrem = min(kSliceWords, nw - t.slice * kSliceWords);
+    T.rb0 = t.rb0;
+    T.nrb = t.nrb;
+    T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
+    const int col = t.slice * kSliceElems + (int)threadIdx.x;
+    if (col < J.cols) c.sc[k] = __ldg(reinterpret_cast<const unsigned short*>(J.vscale) + col);
+}
+
 // Collect the next batch at c.u and load this thread's scale elements.
-// Reads only plan data and weights.
 __device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args, Cursor& c) {
     c.nt = 0;
     c.n_rb = 0;
@@ -523,27 +532,8 @@ __device__ __forceinline__ void batch_begin(const Smem& sm, const CallArgs& args
         if (c.u + c.n_rb < c.u_end) {
             c.t[k] = next_tile(sm.jobs, sm.phase->n_jobs, c.j, c.u + c.n_rb, c.u_end);
             c.nt = k + 1;
-            const Tile& t = c.t[k];
-            const LbJob& J = sm.jobs[t.job];
-            TileRt& T = c.rt[k];
-            const int nw = (J.cols + 31) / 32;
-            if (J.sliced) {   // the slice is a contiguous block of rows
-                T.P = J.P + (size_t)kSliceWords * (size_t)J.rows * (size_t)t.slice;
-                T.ldw = (int)sliced_pitch(nw, t.slice);
-            } else {
-                T.P = J.P + (size_t)t.slice * kSliceWords;
-                T.ldw = J.ldw;
-            }
-            T.h = J.oscale;
-            T.out = resolve(J.out, args);
-            T.rows = J.rows;
-            T.wrem = min(kSliceWords, nw - t.slice * kSliceWords);
-            T.rb0 = t.rb0;
-            T.nrb = t.nrb;
-            T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
-            c.n_rb += t.nrb;
-            const int col = t.slice * kSliceElems + (int)threadIdx.x;
-            if (col < J.cols) c.sc[k] = __ldg(reinterpret_cast<const unsigned short*>(J.vscale) + col);
+            c.n_rb += c.t[k].nrb;
+            tile_setup(sm, args, c, k);
         }
     }
 }
@@ -607,7 +597,26 @@ __device__ __forceinline__ void stage_batch(const Smem& sm, const CallArgs& args
 
 // The part of a phase that does not depend on earlier phases: this CTA's
 // unit range and its first batch.  sm.phase / sm.jobs must hold the phase.
+// The first batch comes from the plan's start table when it was made for this
+// grid (the same tiles batch_begin would find), else from batch_begin.
 __device__ __forceinline__ void phase_begin(const Smem& sm, const CallArgs& args, Cursor& c) {
+    if (sm.phase->starts_g == (int)gridDim.x) {
+        const LbStart& S = *sm.start;
+        c.u = S.u;
+        c.u_end = S.u_end;
+        c.j = S.j;
+        c.nt = S.nt;
+        c.n_rb = S.n_rb;
+#pragma unroll
+        for (int k = 0; k < kMaxTiles; ++k) {
+            c.sc[k] = 0u;
+            if (k < c.nt) {
+                c.t[k] = S.t[k];
+                tile_setup(sm, args, c, k);
+            }
+        }
+        return;
+    }
     unit_range(sm, c.u, c.u_end);
     c.j = 0;
     c.nt = 0;
@@ -641,8 +650,8 @@ __device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, 
 
 template <bool kAsyncPlan>
 __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases, const LbJob* jobs,
-                                            const int* splits, WsHeader* hdr,
-                                            const CallArgs& args) {
+                                            const int* splits, const LbStart* starts,
+                                            WsHeader* hdr, const CallArgs& args) {
     Smem sm = smem_layout();
     const unsigned G = gridDim.x;
     if (*reinterpret_cast<volatile int*>(&hdr->error) != 0) return;   // sticky after a timeout
@@ -665,8 +674,8 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
     }
     // The first two phases' plans are copied in by the whole CTA; each later
     // one is fetched asynchronously by the last warp one phase ahead.
-    cache_plan(phases, 0, jobs, splits, 0);
-    if (n_phases > 1) cache_plan(phases, 1, jobs, splits, 1);
+    cache_plan(phases, 0, jobs, splits, starts, 0);
+    if (n_phases > 1) cache_plan(phases, 1, jobs, splits, starts, 1);
     __syncthreads();
     Cursor cur;
     RB buf[kDepth];
@@ -687,10 +696,10 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
             phase_begin(sm, args, cur);
             if (kAsyncPlan && wp == kDecodeWarps - 1 && p + 2 < n_phases)
                 cache_plan_async(phases, p + 2, sm.phase->next_job_begin, sm.phase->next_n_jobs,
-                                 jobs, splits, nb ^ 1);
+                                 jobs, splits, starts, nb ^ 1);
             if (!kAsyncPlan && p + 2 < n_phases) {   // (not reached: such plans have two phases)
                 __syncthreads();
-                cache_plan(phases, p + 2, jobs, splits, nb ^ 1);
+                cache_plan(phases, p + 2, jobs, splits, starts, nb ^ 1);
             }
             if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) {
                 if (wp == kDecodeWarps - 1) plan_wait();
@@ -714,15 +723,15 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 linear_program_kernel(const __grid_constant__ LinearPlan plan, int n_phases, WsHeader* hdr) {
     const CallArgs args = {nullptr, nullptr};
-    run_program<false>(plan.phases, n_phases, plan.jobs, plan.split, hdr, args);
+    run_program<false>(plan.phases, n_phases, plan.jobs, plan.split, nullptr, hdr, args);
 }
 
 __global__ void __launch_bounds__(kDecodeThreads, kCtasPerSm)
 stack_program_kernel(const LbPhase* __restrict__ phases, const LbJob* __restrict__ jobs,
-                     const int* __restrict__ splits, int n_phases, WsHeader* hdr, const void* x,
-                     float* y) {
+                     const int* __restrict__ splits, const LbStart* __restrict__ starts,
+                     int n_phases, WsHeader* hdr, const void* x, float* y) {
     const CallArgs args = {x, y};
-    run_program<true>(phases, n_phases, jobs, splits, hdr, args);
+    run_program<true>(phases, n_phases, jobs, splits, starts, hdr, args);
 }
 
 cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
@@ -830,6 +839,31 @@ void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out)
     for (int c = used; c <= G; ++c) out[c] = n_units;
 }
 
+void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* split, int G,
+                 LbStart* out) {
+    for (int q = 0; q < n_phases; ++q) {
+        LbPhase& ph = phases[q];
+        ph.starts_g = -1;
+        if (G > kMaxGrid || ph.split_g != G) continue;
+        const LbJob* pj = jobs + ph.job_begin;
+        const int* sp = split + ph.split_off;
+        for (int c = 0; c < G; ++c) {
+            LbStart S = {};
+            S.u = sp[c];
+            S.u_end = sp[c + 1];
+            // the tiles of the first batch, as the kernel's batch_begin takes them
+            for (int k = 0; k < kTables; ++k) {
+                if (S.u + S.n_rb >= S.u_end) break;
+                S.t[k] = next_tile(pj, ph.n_jobs, S.j, S.u + S.n_rb, S.u_end);
+                S.nt = k + 1;
+                S.n_rb += S.t[k].nrb;
+            }
+            out[(size_t)q * kMaxGrid + c] = S;
+        }
+        ph.starts_g = G;
+    }
+}
+
 cudaError_t decode_configure() {
     for (const void* fn : {reinterpret_cast<const void*>(linear_program_kernel),
                            reinterpret_cast<const void*>(stack_program_kernel)}) {
@@ -854,9 +888,9 @@ cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phas
 }
 
 cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const int* splits,
-                              int n_phases, WsHeader* hdr, const void* x, float* y,
-                              cudaStream_t s) {
-    void* args[] = {&phases, &jobs, &splits, &n_phases, &hdr, &x, &y};
+                              const LbStart* starts, int n_phases, WsHeader* hdr, const void* x,
+                              float* y, cudaStream_t s) {
+    void* args[] = {&phases, &jobs, &splits, &starts, &n_phases, &hdr, &x, &y};
     return launch_coop(reinterpret_cast<const void*>(stack_program_kernel), args, s);
 }
 

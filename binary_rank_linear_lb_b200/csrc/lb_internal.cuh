@@ -80,9 +80,49 @@ struct alignas(16) LbPhase {
     int split_g;              // CTAs the split was made for (-1 or another grid: even split)
     int next_job_begin;       // jobs of the following phase (0 / 0 for the last phase), so a
     int next_n_jobs;          // CTA can fetch that phase's plan without reading its header first
-    int pad[2];
+    int starts_g;             // CTAs the start table was made for (-1: no table, compute on device)
+    int pad;
 };
 static_assert(sizeof(LbPhase) == 48, "LbPhase is copied in 16-byte pieces");
+
+// A tile: the units of one slice of one job that a CTA runs in one go.
+struct LbTile {
+    int job, slice, rb0, nrb;
+};
+
+// A CTA's first batch of a phase (its unit range and the tiles of the range
+// that the first batch takes), computed on the host when the plan is made so
+// the CTA does not search for them between two phases.
+struct alignas(16) LbStart {
+    int u, u_end, j, nt, n_rb, pad[3];
+    LbTile t[2];
+};
+static_assert(sizeof(LbStart) == 64, "LbStart is copied in 16-byte pieces");
+
+__host__ __device__ __forceinline__ int find_job(const LbJob* jobs, int j, int j_end, int u) {
+    while (j + 1 < j_end && jobs[j + 1].unit_begin <= u) ++j;
+    return j;
+}
+
+// The tile of a unit range that starts at unit u (u < u_end).  A job's units
+// run row group by row group, slice by slice inside a group, so the CTAs
+// holding the slices of one group stream the same rows together and each DRAM
+// page is read while it is open.
+__host__ __device__ __forceinline__ LbTile next_tile(const LbJob* jobs, int n_jobs, int& j, int u,
+                                                     int u_end) {
+    j = find_job(jobs, j, n_jobs, u);
+    const LbJob& J = jobs[j];
+    const int local = u - J.unit_begin;
+    const int per_group = J.rg * J.n_slices;
+    const int g = local / per_group;
+    const int off = local - g * per_group;
+    const int left = J.n_rowblocks - g * J.rg;
+    const int rows_g = J.rg < left ? J.rg : left;
+    const int s = off / rows_g;
+    const int rbi = off - s * rows_g;
+    const int rest = u_end - u;
+    return LbTile{j, s, g * J.rg + rbi, rows_g - rbi < rest ? rows_g - rbi : rest};
+}
 
 // Stack plans are prepared once and reused with different x / y buffers, so
 // job pointers that mean "the call's x" or "the call's y" are stored as tags.
@@ -94,7 +134,7 @@ static_assert(sizeof(LbPhase) == 48, "LbPhase is copied in 16-byte pieces");
 // (1 KB on sm_100) and must end below kTableAddr0; the size requested covers
 // the tables for any base below that.
 constexpr int kMiscBytes = 4 * kTables * kVecPad + 4 * 32 + 64 +
-                           2 * (64 + kMaxPhaseJobs * (int)sizeof(LbJob));
+                           2 * (128 + kMaxPhaseJobs * (int)sizeof(LbJob));
 constexpr int kDecodeSmem = (int)kTableAddr0 + kTables * kLutBytes;
 static_assert(kDecodeSmem <= 227 * 1024, "decode kernel shared memory over the per-CTA limit");
 static_assert(kMiscBytes + 1024 <= (int)kTableAddr0, "decode plan cache overlaps the tables");
@@ -209,13 +249,17 @@ cudaError_t decode_configure();      // one-time kernel attribute setup per devi
 cudaError_t launch_linear_plan(const LinearPlan& plan, WsHeader* hdr, int n_phases,
                                cudaStream_t s);
 cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const int* splits,
-                              int n_phases, WsHeader* hdr, const void* x, float* y,
-                              cudaStream_t s);
+                              const LbStart* starts, int n_phases, WsHeader* hdr, const void* x,
+                              float* y, cudaStream_t s);
 int decode_grid();                   // CTAs of a decode launch on the current device
 // Row-group sizes of a phase's jobs for a grid of G CTAs.
 void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G);
 // Cost-balanced contiguous unit ranges for the G CTAs of a phase (out: G+1 boundaries).
 void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
+// The first batch of each CTA of each phase from the split table (G <= kMaxGrid);
+// out holds n_phases * kMaxGrid records, phase q's at q * kMaxGrid.  Sets starts_g.
+void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* split, int G,
+                 LbStart* out);
 
 // Tensor-core prefill path (lb_prefill.cu).
 constexpr int kPrefillMinM = 16;             // lb_linear_forward uses it from this many rows
