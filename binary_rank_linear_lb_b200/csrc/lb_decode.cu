@@ -324,11 +324,14 @@ __device__ __forceinline__ void load_rb(const TileRt& T, int rb, RB& R) {
     const int lane = threadIdx.x & 31;
     const int rho = lane >> 2, gam = lane & 3;
     const int w = 4 * gam;
-    if (T.wrem == kSliceWords && (T.ldw & 3) == 0 && rb * kRowBlock + kRowBlock <= T.rows) {
-        // the usual case: all 32 rows inside, full 16-word pieces
+    if (((T.wrem | T.ldw) & 3) == 0 && rb * kRowBlock + kRowBlock <= T.rows) {
+        // the usual case: all 32 rows inside, whole 16-byte groups (lanes past
+        // the slice's words hold zeros)
         const uint32_t* p = T.P + (size_t)(rb * kRowBlock + rho) * (size_t)T.ldw + w;
+        const bool in = w < T.wrem;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) R.d[i] = ld_stream_v4(p + (size_t)(8 * i) * T.ldw);
+        for (int i = 0; i < 4; ++i)
+            R.d[i] = in ? ld_stream_v4(p + (size_t)(8 * i) * T.ldw) : make_uint4(0u, 0u, 0u, 0u);
     } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -514,7 +517,9 @@ __device__ __forceinline__ void tile_setup(const Smem& sm, const CallArgs& args,
     T.h = J.oscale;
     T.out = resolve(J.out, args);
     T.rows = J.rows;
-    T.wrem = min(kSliceWords, nw - t.slice * kSliceWords);
+    // words of the slice a lane may read: in the sliced layout the whole pitch
+    // (padding words hold bits of columns whose vector elements are zero)
+    T.wrem = J.sliced ? T.ldw : min(kSliceWords, nw - t.slice * kSliceWords);
     T.rb0 = t.rb0;
     T.nrb = t.nrb;
     T.tb = kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes;
