@@ -462,10 +462,11 @@ __device__ __forceinline__ TileRt batch_tile(const Cursor& c, int n, int& rb) {
 // Issue this warp's first kDepth rowblocks of the batch into buf.  Register
 // loads can stall a warp at issue once the SM's outstanding misses fill up,
 // so they are issued only after the batch's tables are built.
-__device__ __forceinline__ void batch_loads(const Cursor& c, RB (&buf)[kDepth]) {
+__device__ __forceinline__ void batch_loads(const Cursor& c, RB (&buf)[kDepth], int d0 = 0) {
     const int wp = threadIdx.x >> 5;
 #pragma unroll
     for (int d = 0; d < kDepth; ++d) {
+        if (d < d0) continue;
         const int n = wp + d * kDecodeWarps;
         if (n < c.n_rb) {
             int rb;
@@ -641,10 +642,20 @@ __device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, 
             zp[i] = 0.0f;
     }
     while (c.u < c.u_end) {
+        // each warp's first rowblock is requested before the vector is staged
+        // (32 KB per CTA), its second after the tables are built
+        {
+            const int n = (int)(threadIdx.x >> 5);
+            if (n < c.n_rb) {
+                int rb;
+                const TileRt T = batch_tile(c, n, rb);
+                load_rb(T, rb, buf[0]);
+            }
+        }
         stage_batch(sm, args, c);
         for (int k = 0; k < c.nt; ++k)
             build_table(sm.vec + k * kVecPad, kTableAddr0 + (uint32_t)k * (uint32_t)kLutBytes);
-        batch_loads(c, buf);
+        batch_loads(c, buf, 1);
         __syncthreads();
         batch_lookups(c, buf, Bc, S);
         c.u += c.n_rb;
