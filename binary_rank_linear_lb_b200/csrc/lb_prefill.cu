@@ -198,6 +198,20 @@ struct PrefillGemm {
     int* err;
 };
 
+// Both GEMMs of a call as one persistent launch: the tile list is stage 1's
+// tiles, then stage 2's, dealt round-robin to the CTAs.  A stage-2 tile reads
+// the rows of T of its M block, so before loading them its TMA thread waits
+// until every epilogue warp of the block's stage-1 tiles has published its
+// rows (done[mb] reaching done_target).  Every CTA reaches all its stage-1
+// tiles before any stage-2 tile, and the other roles never wait for the TMA
+// thread, so a stage-1 tile is never held up behind a waiting stage-2 tile.
+struct PrefillPlan {
+    PrefillGemm g[2];
+    int n_tiles[2];
+    int* done;           // [M blocks] stage-1 epilogue warps finished, zeroed per call
+    int done_target;     // kEpiWarps * (stage-1 tiles of one M block)
+};
+
 namespace {
 
 __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb, int& nseg,
@@ -258,9 +272,36 @@ __device__ __forceinline__ uint2 load_bits(const PrefillGemm& g, int branch, int
     return __ldg(reinterpret_cast<const uint2*>(g.P[branch] + off));
 }
 
+__device__ __forceinline__ int ld_acquire_s32(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// The GEMM, tensor map and index within its GEMM of global tile t.
+struct TileRef {
+    const PrefillGemm* g;
+    const CUtensorMap* map;
+    int stage2, t, mb, nseg, nt, kb_per_seg, n_kb;
+};
+__device__ __forceinline__ TileRef tile_ref(const PrefillPlan& plan, const CUtensorMap* amap1,
+                                            const CUtensorMap* amap2, int t) {
+    TileRef r;
+    r.stage2 = t >= plan.n_tiles[0] ? 1 : 0;
+    r.g = r.stage2 ? &plan.g[1] : &plan.g[0];
+    r.map = r.stage2 ? amap2 : amap1;
+    r.t = t - (r.stage2 ? plan.n_tiles[0] : 0);
+    tile_coords(*r.g, r.t, r.mb, r.nseg, r.nt);
+    r.kb_per_seg = r.g->k_seg_len / kBlockK;
+    r.n_kb = r.g->n_kseg * r.kb_per_seg;
+    return r;
+}
+
 template <int MT>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
-prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ PrefillGemm g) {
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
+                    const __grid_constant__ CUtensorMap amap2,
+                    const __grid_constant__ PrefillPlan plan) {
     using S = Shape<MT>;
     constexpr int kStages = S::kStages, kStageBytes = S::kStageBytes;
     extern __shared__ __align__(1024) unsigned char dsm[];
@@ -270,10 +311,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     Ctl* ctl = reinterpret_cast<Ctl*>(basep + S::kOffCtl);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
-    const int n_tiles = ((g.M + MT * kTileM - 1) / (MT * kTileM)) * g.n_nseg * nt_per_seg;
-    const int kb_per_seg = g.k_seg_len / kBlockK;
-    const int n_kb = g.n_kseg * kb_per_seg;
+    const int n_tiles = plan.n_tiles[0] + plan.n_tiles[1];
+    int* const err = plan.g[0].err;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -301,46 +340,75 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     if (warp == kTmaWarp) {
         // ---------------- TMA producer for A (and the g slice of stage 1).  A
         // boxes kPrefetchAhead K blocks ahead (into the next tile at the end of
-        // one) are pulled into L2 first, so the loads find them there.
+        // one) are pulled into L2 first, so the loads find them there; a
+        // stage-2 tile's boxes only once its rows of T are complete.
         if (lane == 0) {
-            auto acol = [&](int kb) {
-                const int ks = kb / kb_per_seg;
-                return ks * g.k_seg_len + (kb - ks * kb_per_seg) * kBlockK;
+            auto acol = [](const TileRef& r, int kb) {
+                const int ks = kb / r.kb_per_seg;
+                return ks * r.g->k_seg_len + (kb - ks * r.kb_per_seg) * kBlockK;
             };
-            auto prefetch = [&](int t, int kb) {
+            auto ready = [&](const TileRef& r) {
+                return !r.stage2 ||
+                       *reinterpret_cast<volatile const int*>(plan.done + r.mb) >= plan.done_target;
+            };
+            auto prefetch = [&](const TileRef& cur, int t, int kb) {
                 int pb = kb + kPrefetchAhead;
-                if (pb >= n_kb) { t += gridDim.x; pb -= n_kb; }
-                if (t >= n_tiles || pb >= n_kb) return;
-                int mb, nseg, nt;
-                tile_coords(g, t, mb, nseg, nt);
+                TileRef r = cur;
+                if (pb >= cur.n_kb) {
+                    t += gridDim.x;
+                    if (t >= n_tiles) return;
+                    pb -= cur.n_kb;
+                    r = tile_ref(plan, &amap1, &amap2, t);
+                    if (pb >= r.n_kb || !ready(r)) return;
+                }
 #pragma unroll
                 for (int j = 0; j < MT; ++j)
-                    if ((mb * MT + j) * kTileM < g.M) tma_prefetch_2d(&amap, acol(pb), (mb * MT + j) * kTileM);
+                    if ((r.mb * MT + j) * kTileM < r.g->M)
+                        tma_prefetch_2d(r.map, acol(r, pb), (r.mb * MT + j) * kTileM);
             };
-            if (blockIdx.x < n_tiles)
-                for (int kb = -kPrefetchAhead; kb < 0; ++kb) prefetch(blockIdx.x, kb);
+            if (blockIdx.x < n_tiles) {
+                const TileRef r0 = tile_ref(plan, &amap1, &amap2, blockIdx.x);
+                if (ready(r0))
+                    for (int kb = 0; kb < kPrefetchAhead && kb < r0.n_kb; ++kb) prefetch(r0, blockIdx.x, kb - kPrefetchAhead);
+            }
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
-                int mb, nseg, nt;
-                tile_coords(g, t, mb, nseg, nt);
-                for (int kb = 0; kb < n_kb; ++kb, ++it) {
-                    prefetch(t, kb);
+                const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+                const PrefillGemm& g = *r.g;
+                if (r.stage2) {
+                    // wait (bounded) for the M block's rows of T, then order the TMA
+                    // reads after the generic-proxy writes that produced them
+                    const long long t0 = clock64();
+                    while (ld_acquire_s32(plan.done + r.mb) < plan.done_target) {
+                        if (*reinterpret_cast<volatile int*>(&ctl->abort)) break;
+                        if (clock64() - t0 > kWaitLimit) {
+                            atomicExch(&ctl->abort, 1);
+                            atomicExch(err, (int)LB_ERR_TIMEOUT);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    if (ctl->abort) break;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
+                for (int kb = 0; kb < r.n_kb; ++kb, ++it) {
+                    prefetch(r, t, kb);
                     const int s = it % kStages;
                     const uint32_t par = ((it / kStages) & 1) ^ 1;
-                    if (!wait_bar(ctl, &ctl->empty[s], par, g.err)) break;
+                    if (!wait_bar(ctl, &ctl->empty[s], par, err)) break;
                     const uint32_t fb = smem_u32(&ctl->full_a[s]);
-                    const int kcol = acol(kb);
+                    const int kcol = acol(r, kb);
                     const uint32_t sa = base + s * kStageBytes;
-                    if (g.stage == 1) {
-                        const int kloc = kcol - (kb / kb_per_seg) * g.k_seg_len;
+                    if (!r.stage2) {
+                        const int kloc = kcol - (kb / r.kb_per_seg) * g.k_seg_len;
                         mbar_expect_tx(fb, MT * kABytes + kGBytes);
-                        bulk_load(base + S::kOffG + s * kGBytes, g.bscale[nseg] + kloc, kGBytes, fb);
+                        bulk_load(base + S::kOffG + s * kGBytes, g.bscale[r.nseg] + kloc, kGBytes, fb);
                     } else {
                         mbar_expect_tx(fb, MT * kABytes);
                     }
 #pragma unroll
                     for (int j = 0; j < MT; ++j)
-                        tma_load_2d(sa + j * kABytes, &amap, fb, kcol, (mb * MT + j) * kTileM);
+                        tma_load_2d(sa + j * kABytes, r.map, fb, kcol, (r.mb * MT + j) * kTileM);
                 }
             }
         }
@@ -351,15 +419,16 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x, ++tl) {
                 const int buf = tl % S::kBufs;
                 const uint32_t use = (uint32_t)(tl / S::kBufs);
-                if (!wait_bar(ctl, &ctl->acc_empty[buf], (use & 1) ^ 1, g.err)) break;
+                if (!wait_bar(ctl, &ctl->acc_empty[buf], (use & 1) ^ 1, err)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * MT * kTileN);
+                const int n_kb = tile_ref(plan, &amap1, &amap2, t).n_kb;
                 bool ok = true;
                 for (int kb = 0; kb < n_kb; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t par = (it / kStages) & 1;
-                    if (!wait_bar(ctl, &ctl->full_a[s], par, g.err) ||
-                        !wait_bar(ctl, &ctl->full_b[s], par, g.err)) { ok = false; break; }
+                    if (!wait_bar(ctl, &ctl->full_a[s], par, err) ||
+                        !wait_bar(ctl, &ctl->full_b[s], par, err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_s = base + s * kStageBytes;
                     const uint64_t bd = sw128_desc(a_s + MT * kABytes);
@@ -389,15 +458,16 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         const int c_end = MT == 2 ? kTileN : c_begin + kTileN / 2;
         const uint32_t stg = base + S::kOffEpi + (uint32_t)warp * kEpiBytes;
         const uint32_t my_row = stg + (uint32_t)lane * 128u;
-        const int ldt = g.n_nseg * g.n_seg_rows;          // T row pitch (stage 1)
         int tl = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-            int mb, nseg, nt;
-            tile_coords(g, t, mb, nseg, nt);
+            const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+            const PrefillGemm& g = *r.g;
+            const int mb = r.mb, nseg = r.nseg, nt = r.nt;
+            const int ldt = g.n_nseg * g.n_seg_rows;      // T row pitch (stage 1)
             const int buf = tl % S::kBufs;
             // every lane waits; the warp stops together so the .sync.aligned loads stay converged
             if (!__all_sync(0xffffffffu, wait_bar(ctl, &ctl->acc_full[buf],
-                                                  (uint32_t)(tl / S::kBufs) & 1, g.err)))
+                                                  (uint32_t)(tl / S::kBufs) & 1, err)))
                 break;
             tc_fence_after();
             const int m0 = (mb * MT + sub) * kTileM + q * 32;     // first row of this warp
@@ -498,7 +568,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
+                // stage 1: this warp's rows of T are written; publish them to the
+                // stage-2 tiles of the M block (release orders the warp's stores)
+                if (!r.stage2)
+                    asm volatile("red.release.gpu.global.add.s32 [%0], 1;"
+                                 :: "l"(plan.done + mb) : "memory");
+            }
         }
     } else if (warp >= kExpandWarp0) {
         // ---------------- B producers: packed signs -> fp16 tile, one row per thread
@@ -507,8 +584,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         uint32_t ph = 0;                             // and the parity of its current use
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            int mb, nseg, nt;
-            tile_coords(g, t, mb, nseg, nt);
+            const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+            const PrefillGemm& g = *r.g;
+            const int nseg = r.nseg, nt = r.nt, kb_per_seg = r.kb_per_seg, n_kb = r.n_kb;
             const int row = nt * kTileN + e;
             uint32_t hh0 = 0u, hh1 = 0u;             // h[row] of each branch in both fp16 halves
             if (g.stage == 2 && row < g.n_seg_rows) {
@@ -538,8 +616,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                     if (kb >= n_kb) break;
                     const uint2 cur = nx[j];
                     if (kb + kBitsAhead < n_kb) nx[j] = fetch();
-                    bool w = wait_bar(ctl, &ctl->empty[s], ph ^ 1, g.err);
-                    if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, g.err);
+                    bool w = wait_bar(ctl, &ctl->empty[s], ph ^ 1, err);
+                    if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, err);
                     if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
                     const uint32_t sb = base + s * kStageBytes + MT * kABytes;
                     expand_row(sb, base + S::kOffG + s * kGBytes, e, cur, g.stage == 1,
@@ -695,7 +773,7 @@ cudaError_t prefill_configure() {
 size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     return up(sizeof(WsHeader)) + up(2 * (size_t)M * in) + up(2 * (size_t)M * 2 * r) +
-           up(8 * (size_t)M) + 256;
+           up(8 * (size_t)M) + 256 + up(4 * (size_t)((M + kTileM - 1) / kTileM));
 }
 
 bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
@@ -708,27 +786,43 @@ bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
 // grid.  Pick the shape with the smaller estimated time, a two-sub-tile tile
 // costing kTile2Cost one-sub-tile tiles.  LB_PREFILL_SUBTILES=1 or 2 in the
 // environment (read on every call) fixes the choice; both give the same result.
-static int pick_subtiles(const PrefillGemm& p, int grid) {
+static long long gemm_tiles(const PrefillGemm& p, int mt) {
+    return (long long)p.n_nseg * ((p.n_seg_rows + kTileN - 1) / kTileN) *
+           ((p.M + mt * kTileM - 1) / (mt * kTileM));
+}
+
+static int pick_subtiles(const PrefillGemm* p, int grid) {
     constexpr double kTile2Cost = 1.35;
     if (const char* env = std::getenv("LB_PREFILL_SUBTILES")) {
         if (env[0] == '1' && env[1] == 0) return 1;
         if (env[0] == '2' && env[1] == 0) return 2;
     }
-    if (p.M <= kTileM) return 1;
-    const long long nt = (long long)p.n_nseg * ((p.n_seg_rows + kTileN - 1) / kTileN);
-    const long long t1 = nt * ((p.M + kTileM - 1) / kTileM);
-    const long long t2 = nt * ((p.M + 2 * kTileM - 1) / (2 * kTileM));
-    const double c1 = (double)((t1 + grid - 1) / grid);
-    const double c2 = (double)((t2 + grid - 1) / grid) * kTile2Cost;
-    return c2 < c1 ? 2 : 1;
+    if (p[0].M <= kTileM) return 1;
+    // makespan estimate: the K blocks of all tiles spread over the grid, plus
+    // one tile of imbalance (tiles are dealt round-robin)
+    double c[3] = {0.0, 0.0, 0.0};
+    for (int mt = 1; mt <= 2; ++mt) {
+        const double cost = mt == 2 ? kTile2Cost : 1.0;
+        double work = 0.0, lump = 0.0;
+        for (int i = 0; i < 2; ++i) {
+            const double n_kb = (double)p[i].n_kseg * (double)(p[i].k_seg_len / kBlockK);
+            work += (double)gemm_tiles(p[i], mt) * n_kb * cost;
+            lump = n_kb * cost > lump ? n_kb * cost : lump;
+        }
+        c[mt] = work / (double)grid + lump;
+    }
+    return c[2] < c[1] ? 2 : 1;
 }
 
-static cudaError_t launch_gemm(const CUtensorMap& amap, const PrefillGemm& p, int grid,
-                               cudaStream_t s) {
-    if (pick_subtiles(p, grid) == 2)
-        prefill_gemm_kernel<2><<<grid, kPrefillThreads, Shape<2>::kSmem, s>>>(amap, p);
-    else
-        prefill_gemm_kernel<1><<<grid, kPrefillThreads, Shape<1>::kSmem, s>>>(amap, p);
+template <int MT>
+static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const CUtensorMap& m2,
+                                int grid, cudaStream_t s) {
+    for (int i = 0; i < 2; ++i) plan.n_tiles[i] = (int)gemm_tiles(plan.g[i], MT);
+    plan.done_target = kEpiWarps * plan.g[0].n_nseg * ((plan.g[0].n_seg_rows + kTileN - 1) / kTileN);
+    const int blocks = (plan.g[0].M + MT * kTileM - 1) / (MT * kTileM);
+    cudaError_t e = cudaMemsetAsync(plan.done, 0, sizeof(int) * (size_t)blocks, s);
+    if (e != cudaSuccess) return e;
+    prefill_gemm_kernel<MT><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
     return cudaGetLastError();
 }
 
@@ -747,6 +841,8 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     float* sc = sa + M;
     off += up(8 * (size_t)M);
     float* lmax = reinterpret_cast<float*>(ws + off);
+    off += 256;
+    int* done = reinterpret_cast<int*>(ws + off);   // per M block, stage-1 tiles finished
 
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
     if (e != cudaSuccess) return e;
@@ -758,12 +854,13 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         sa, sc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    const int grid = device_sm_count();
+    PrefillPlan plan = {};
+    plan.done = done;
     // stage 1: T = (x 2^a) (g o sign V)^T, epilogue applies l, 2^-a, 2^c
+    CUtensorMap amap1, amap2;
+    if (!make_amap(&amap1, X16, (int)M, (int)in)) return cudaErrorInvalidValue;
     {
-        CUtensorMap amap;
-        if (!make_amap(&amap, X16, (int)M, (int)in)) return cudaErrorInvalidValue;
-        PrefillGemm p = {};
+        PrefillGemm& p = plan.g[0];
         p.M = (int)M; p.n_seg_rows = (int)r; p.n_nseg = nb; p.n_kseg = 1; p.k_seg_len = (int)in;
         p.stage = 1;
         p.nw = (int)((in + 31) / 32);
@@ -776,13 +873,11 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
             p.lscale[b] = reinterpret_cast<const __half*>(B.l);
         }
         p.row_sa = sa; p.row_sc = sc; p.T = T; p.y = nullptr; p.err = &hdr->error;
-        if ((e = launch_gemm(amap, p, grid, s)) != cudaSuccess) return e;
     }
     // stage 2: y = (T) (h o sign U)^T over K = nb * r, epilogue divides 2^c out
+    if (!make_amap(&amap2, T, (int)M, (int)(nb * r))) return cudaErrorInvalidValue;
     {
-        CUtensorMap amap;
-        if (!make_amap(&amap, T, (int)M, (int)(nb * r))) return cudaErrorInvalidValue;
-        PrefillGemm p = {};
+        PrefillGemm& p = plan.g[1];
         p.M = (int)M; p.n_seg_rows = (int)out; p.n_nseg = 1; p.n_kseg = nb; p.k_seg_len = (int)r;
         p.stage = 2;
         p.nw = (int)((r + 31) / 32);
@@ -795,9 +890,10 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
             p.lscale[b] = nullptr;
         }
         p.row_sa = sa; p.row_sc = sc; p.T = nullptr; p.y = y; p.err = &hdr->error;
-        if ((e = launch_gemm(amap, p, grid, s)) != cudaSuccess) return e;
     }
-    return cudaSuccess;
+    const int grid = device_sm_count();
+    return pick_subtiles(plan.g, grid) == 2 ? launch_gemms<2>(plan, amap1, amap2, grid, s)
+                                            : launch_gemms<1>(plan, amap1, amap2, grid, s);
 }
 
 }  // namespace lb
