@@ -297,6 +297,23 @@ __device__ __forceinline__ TileRef tile_ref(const PrefillPlan& plan, const CUten
     return r;
 }
 
+// Piece p (8 fp16 values, l[n0 + 8p .. n0 + 8p + 7]) of segment nseg's l,
+// zero past the segment.
+__device__ __forceinline__ uint4 load_l8(const PrefillGemm& g, int nseg, int n0, int p) {
+    const __half* lb = g.lscale[nseg] + n0 + 8 * p;
+    if (n0 + 8 * p + 8 <= g.n_seg_rows && (reinterpret_cast<uintptr_t>(lb) & 15) == 0)
+        return __ldg(reinterpret_cast<const uint4*>(lb));
+    uint32_t e2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int n = n0 + 8 * p + 2 * i;
+        const uint32_t lo = n < g.n_seg_rows ? __half_as_ushort(__ldg(lb + 2 * i)) : 0u;
+        const uint32_t hi = n + 1 < g.n_seg_rows ? __half_as_ushort(__ldg(lb + 2 * i + 1)) : 0u;
+        e2[i] = lo | (hi << 16);
+    }
+    return make_uint4(e2[0], e2[1], e2[2], e2[3]);
+}
+
 template <int MT>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
@@ -465,16 +482,22 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             const int mb = r.mb, nseg = r.nseg, nt = r.nt;
             const int ldt = g.n_nseg * g.n_seg_rows;      // T row pitch (stage 1)
             const int buf = tl % S::kBufs;
-            // every lane waits; the warp stops together so the .sync.aligned loads stay converged
-            if (!__all_sync(0xffffffffu, wait_bar(ctl, &ctl->acc_full[buf],
-                                                  (uint32_t)(tl / S::kBufs) & 1, err)))
-                break;
-            tc_fence_after();
+            // per-tile loads go out before the wait: the row scales, and (stage 1)
+            // l of the first chunk; l of chunk c+1 is loaded while chunk c is stored
             const int m0 = (mb * MT + sub) * kTileM + q * 32;     // first row of this warp
             const int m = m0 + lane;
             const bool mok = m < g.M;
             const float sa = mok ? __ldg(g.row_sa + m) : 1.0f;
             const float sc = mok ? __ldg(g.row_sc + m) : 1.0f;
+            // (stage 1) lane p < 4 holds piece p of the next chunk's l
+            uint4 lnext = make_uint4(0u, 0u, 0u, 0u);
+            if (g.stage == 1 && lane < 4 && nt * kTileN + c_begin < g.n_seg_rows)
+                lnext = load_l8(g, nseg, nt * kTileN + c_begin, lane);
+            // every lane waits; the warp stops together so the .sync.aligned loads stay converged
+            if (!__all_sync(0xffffffffu, wait_bar(ctl, &ctl->acc_full[buf],
+                                                  (uint32_t)(tl / S::kBufs) & 1, err)))
+                break;
+            tc_fence_after();
             const float f = g.stage == 1 ? sc / sa : 1.0f / sc;
             const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * MT + sub) * kTileN);
             for (int c0 = c_begin; c0 < c_end; c0 += 32) {
@@ -484,23 +507,26 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 const int n0 = nt * kTileN + c0;       // row within the N segment
                 if (n0 >= g.n_seg_rows) continue;      // warp-uniform
                 if (g.stage == 1) {
-                    // T = l * t * 2^c with t = D / 2^a, fp16, 4 pieces of 16 bytes per row
-                    const __half* lb = g.lscale[nseg] + n0;
-                    const bool lvec = n0 + 32 <= g.n_seg_rows && (reinterpret_cast<uintptr_t>(lb) & 15) == 0;
+                    // T = l * t * 2^c with t = D / 2^a, fp16, 4 pieces of 16 bytes per row.
+                    // This chunk's l goes to the half of row 0 of the staging buffer
+                    // that the chunk leaves unused (slots 4-7); the next chunk's l is
+                    // requested meanwhile.
+                    const uint32_t lbuf = stg + 64u;
+                    if (lane < 4) {
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(lbuf + 16u * (uint32_t)lane), "r"(lnext.x), "r"(lnext.y),
+                                        "r"(lnext.z), "r"(lnext.w) : "memory");
+                        if (c0 + 32 < c_end && n0 + 32 < g.n_seg_rows)
+                            lnext = load_l8(g, nseg, n0 + 32, lane);
+                    }
+                    __syncwarp();
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t w[4];
                         uint4 lv;
-                        if (lvec) {
-                            lv = __ldg(reinterpret_cast<const uint4*>(lb + 8 * c));
-                        } else {
-                            uint16_t e8[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                e8[i] = n0 + 8 * c + i < g.n_seg_rows ? __half_as_ushort(__ldg(lb + 8 * c + i)) : 0;
-                            lv = make_uint4(e8[0] | (uint32_t)e8[1] << 16, e8[2] | (uint32_t)e8[3] << 16,
-                                            e8[4] | (uint32_t)e8[5] << 16, e8[6] | (uint32_t)e8[7] << 16);
-                        }
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(lv.x), "=r"(lv.y), "=r"(lv.z), "=r"(lv.w)
+                                     : "r"(lbuf + 16u * (uint32_t)c));
                         const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
