@@ -51,6 +51,9 @@ constexpr int kTmemCols = 512;                    // two 256-column accumulators
 constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
 constexpr uint32_t kSuspendNs = 20000;            // longest hardware suspension per try_wait
 constexpr int kMaxStages = 4;
+constexpr int kPartFloats = 8 * 32 * 32;          // one epilogue warp's share of a tile (8 chunks)
+constexpr int kSplitMaxParts = 160;               // stage-1 tile parts the split buffer holds
+constexpr int kSplitMax = 3;                      // K parts of one stage-1 tile (the last one folds the others)
 
 constexpr int kEpiBytes = 32 * 128;                // per-warp epilogue staging: 32 rows x 128 bytes
 constexpr int kPrefetchAhead = 6;                 // K blocks of A pulled into L2 ahead of the TMA loads
@@ -176,6 +179,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 16 columns of fp32 from / to TMEM (one row per lane).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+           "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+           "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+           "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+           "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+           "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ problem
@@ -205,11 +235,19 @@ struct PrefillGemm {
 // rows (done[mb] reaching done_target).  Every CTA reaches all its stage-1
 // tiles before any stage-2 tile, and the other roles never wait for the TMA
 // thread, so a stage-1 tile is never held up behind a waiting stage-2 tile.
+// With few stage-1 tiles (small M, low rank) stage 1 is split along K into
+// `split` parts, adjacent in the tile list.  For each of its chunks an
+// epilogue warp writes its fp32 partial sums to `partial` and takes a ticket
+// for its region of the tile; the warp that draws the last ticket adds the
+// other parts' partials to its own accumulator and finishes the region into T.
 struct PrefillPlan {
     PrefillGemm g[2];
-    int n_tiles[2];
+    int n_tiles[2];      // tiles of each GEMM (stage 1: tiles x split)
     int* done;           // [M blocks] stage-1 epilogue warps finished, zeroed per call
     int done_target;     // kEpiWarps * (stage-1 tiles of one M block)
+    int split;           // K parts of a stage-1 tile (1: no split)
+    float* partial;      // [tile][part][epilogue warp][kPartFloats] fp32 partial sums
+    int* tickets;        // [tile][epilogue warp], zeroed per call
 };
 
 namespace {
@@ -278,22 +316,29 @@ __device__ __forceinline__ int ld_acquire_s32(const int* p) {
     return v;
 }
 
-// The GEMM, tensor map and index within its GEMM of global tile t.
+// The GEMM, tensor map, tile within its GEMM, K part and K-block range
+// [kb0, kb1) of global tile t.
 struct TileRef {
     const PrefillGemm* g;
     const CUtensorMap* map;
-    int stage2, t, mb, nseg, nt, kb_per_seg, n_kb;
+    int stage2, t, part, mb, nseg, nt, kb_per_seg, kb0, kb1;
 };
+template <bool SPLIT>
 __device__ __forceinline__ TileRef tile_ref(const PrefillPlan& plan, const CUtensorMap* amap1,
                                             const CUtensorMap* amap2, int t) {
     TileRef r;
     r.stage2 = t >= plan.n_tiles[0] ? 1 : 0;
     r.g = r.stage2 ? &plan.g[1] : &plan.g[0];
     r.map = r.stage2 ? amap2 : amap1;
-    r.t = t - (r.stage2 ? plan.n_tiles[0] : 0);
+    const int parts = (SPLIT && !r.stage2) ? plan.split : 1;
+    const int tl = t - (r.stage2 ? plan.n_tiles[0] : 0);
+    r.t = tl / parts;
+    r.part = tl - r.t * parts;
     tile_coords(*r.g, r.t, r.mb, r.nseg, r.nt);
     r.kb_per_seg = r.g->k_seg_len / kBlockK;
-    r.n_kb = r.g->n_kseg * r.kb_per_seg;
+    const int n_kb = r.g->n_kseg * r.kb_per_seg;
+    r.kb0 = (int)((long long)n_kb * r.part / parts);
+    r.kb1 = (int)((long long)n_kb * (r.part + 1) / parts);
     return r;
 }
 
@@ -314,7 +359,7 @@ __device__ __forceinline__ uint4 load_l8(const PrefillGemm& g, int nseg, int n0,
     return make_uint4(e2[0], e2[1], e2[2], e2[3]);
 }
 
-template <int MT>
+template <int MT, bool SPLIT>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const __grid_constant__ CUtensorMap amap2,
@@ -371,12 +416,12 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             auto prefetch = [&](const TileRef& cur, int t, int kb) {
                 int pb = kb + kPrefetchAhead;
                 TileRef r = cur;
-                if (pb >= cur.n_kb) {
+                if (pb >= cur.kb1) {
                     t += gridDim.x;
                     if (t >= n_tiles) return;
-                    pb -= cur.n_kb;
-                    r = tile_ref(plan, &amap1, &amap2, t);
-                    if (pb >= r.n_kb || !ready(r)) return;
+                    r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+                    pb = r.kb0 + (pb - cur.kb1);
+                    if (pb >= r.kb1 || !ready(r)) return;
                 }
 #pragma unroll
                 for (int j = 0; j < MT; ++j)
@@ -384,13 +429,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         tma_prefetch_2d(r.map, acol(r, pb), (r.mb * MT + j) * kTileM);
             };
             if (blockIdx.x < n_tiles) {
-                const TileRef r0 = tile_ref(plan, &amap1, &amap2, blockIdx.x);
+                const TileRef r0 = tile_ref<SPLIT>(plan, &amap1, &amap2, blockIdx.x);
                 if (ready(r0))
-                    for (int kb = 0; kb < kPrefetchAhead && kb < r0.n_kb; ++kb) prefetch(r0, blockIdx.x, kb - kPrefetchAhead);
+                    for (int kb = r0.kb0; kb < r0.kb0 + kPrefetchAhead && kb < r0.kb1; ++kb)
+                        prefetch(r0, blockIdx.x, kb - kPrefetchAhead);
             }
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
-                const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+                const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
                 const PrefillGemm& g = *r.g;
                 if (r.stage2) {
                     // wait (bounded) for the M block's rows of T, then order the TMA
@@ -408,7 +454,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     if (ctl->abort) break;
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                 }
-                for (int kb = 0; kb < r.n_kb; ++kb, ++it) {
+                for (int kb = r.kb0; kb < r.kb1; ++kb, ++it) {
                     prefetch(r, t, kb);
                     const int s = it % kStages;
                     const uint32_t par = ((it / kStages) & 1) ^ 1;
@@ -439,9 +485,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 if (!wait_bar(ctl, &ctl->acc_empty[buf], (use & 1) ^ 1, err)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * MT * kTileN);
-                const int n_kb = tile_ref(plan, &amap1, &amap2, t).n_kb;
+                const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
                 bool ok = true;
-                for (int kb = 0; kb < n_kb; ++kb, ++it) {
+                for (int kb = r.kb0; kb < r.kb1; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t par = (it / kStages) & 1;
                     if (!wait_bar(ctl, &ctl->full_a[s], par, err) ||
@@ -454,7 +500,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
 #pragma unroll
                         for (int j = 0; j < MT; ++j)
                             mma_f16(d + (uint32_t)(j * kTileN), sw128_desc(a_s + j * kABytes) + 2ull * kk,
-                                    bd + 2ull * kk, (kb | kk) != 0);
+                                    bd + 2ull * kk, (kb != r.kb0) || (kk != 0));
                     mma_commit(smem_u32(&ctl->empty[s]));
                 }
                 if (!ok) break;
@@ -477,7 +523,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
         const uint32_t my_row = stg + (uint32_t)lane * 128u;
         int tl = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-            const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+            const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
             const PrefillGemm& g = *r.g;
             const int mb = r.mb, nseg = r.nseg, nt = r.nt;
             const int ldt = g.n_nseg * g.n_seg_rows;      // T row pitch (stage 1)
@@ -500,7 +546,57 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             tc_fence_after();
             const float f = g.stage == 1 ? sc / sa : 1.0f / sc;
             const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((buf * MT + sub) * kTileN);
-            for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+            // K split of stage 1: write this warp's partial sums (lane-interleaved
+            // 16-byte pieces, so every access of the warp is 512 contiguous bytes),
+            // then take a ticket; the last of the parts finishes the region
+            const bool split = SPLIT && !r.stage2 && plan.split > 1;
+            bool finish = true;
+            if constexpr (SPLIT) if (split) {
+                float* pw = plan.partial +
+                            ((size_t)(r.t * plan.split + r.part) * kEpiWarps + warp) * kPartFloats;
+                for (int c0 = c_begin, ci = 0; c0 < c_end; c0 += 32, ++ci) {
+                    float v[32];
+                    __syncwarp();
+                    tmem_ld32(tacc + (uint32_t)c0, v);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        __stcg(reinterpret_cast<float4*>(pw + ci * 1024 + (i * 32 + lane) * 4),
+                               make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+                }
+                __syncwarp();
+                int ticket = 0;
+                if (lane == 0)
+                    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                                 : "=r"(ticket) : "l"(plan.tickets + r.t * kEpiWarps + warp) : "memory");
+                finish = __shfl_sync(0xffffffffu, ticket, 0) == plan.split - 1;
+                __syncwarp();
+                if (finish) {
+                    // fold the other parts' sums into this warp's accumulator in TMEM,
+                    // half a chunk (16 columns) at a time
+                    const float* p0 = plan.partial + (size_t)r.t * plan.split * kEpiWarps * kPartFloats +
+                                      (size_t)warp * kPartFloats;
+                    for (int h = 0; h < (c_end - c_begin) / 16; ++h) {
+                        float v[16];
+                        __syncwarp();
+                        tmem_ld16(tacc + (uint32_t)(c_begin + 16 * h), v);
+                        for (int p = 0; p < plan.split; ++p) {
+                            if (p == r.part) continue;
+                            const float* pc = p0 + (size_t)p * kEpiWarps * kPartFloats + h * 512;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 o = __ldcg(reinterpret_cast<const float4*>(pc + (i * 32 + lane) * 4));
+                                v[4 * i] += o.x;
+                                v[4 * i + 1] += o.y;
+                                v[4 * i + 2] += o.z;
+                                v[4 * i + 3] += o.w;
+                            }
+                        }
+                        tmem_st16(tacc + (uint32_t)(c_begin + 16 * h), v);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                }
+            }
+            for (int c0 = c_begin; finish && c0 < c_end; c0 += 32) {
                 float v[32];
                 __syncwarp();
                 tmem_ld32(tacc + (uint32_t)c0, v);
@@ -598,7 +694,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 mbar_arrive(smem_u32(&ctl->acc_empty[buf]));
                 // stage 1: this warp's rows of T are written; publish them to the
                 // stage-2 tiles of the M block (release orders the warp's stores)
-                if (!r.stage2)
+                if (!r.stage2 && finish)
                     asm volatile("red.release.gpu.global.add.s32 [%0], 1;"
                                  :: "l"(plan.done + mb) : "memory");
             }
@@ -610,9 +706,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
         uint32_t ph = 0;                             // and the parity of its current use
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            const TileRef r = tile_ref(plan, &amap1, &amap2, t);
+            const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
             const PrefillGemm& g = *r.g;
-            const int nseg = r.nseg, nt = r.nt, kb_per_seg = r.kb_per_seg, n_kb = r.n_kb;
+            const int nseg = r.nseg, nt = r.nt, kb_per_seg = r.kb_per_seg;
+            const int n_kb = r.kb1 - r.kb0;          // K blocks of this tile (its part of K)
             const int row = nt * kTileN + e;
             uint32_t hh0 = 0u, hh1 = 0u;             // h[row] of each branch in both fp16 halves
             if (g.stage == 2 && row < g.n_seg_rows) {
@@ -625,7 +722,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             }
             // sign bits, fetched kBitsAhead K blocks ahead into a register ring;
             // (fs, fk) = K segment and block within it of the next fetch
-            int fs = 0, fk = 0;
+            const int seg0 = r.kb0 / kb_per_seg, kin0 = r.kb0 - seg0 * kb_per_seg;
+            int fs = seg0, fk = kin0;
             auto fetch = [&]() {
                 const uint2 v = load_bits(g, g.stage == 1 ? nseg : fs, row, fk);
                 if (++fk == kb_per_seg) { fk = 0; ++fs; }
@@ -634,7 +732,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             uint2 nx[kBitsAhead];
 #pragma unroll
             for (int j = 0; j < kBitsAhead; ++j) nx[j] = j < n_kb ? fetch() : make_uint2(0u, 0u);
-            int seg = 0, kin = 0;                    // K segment of the current block, block within it
+            int seg = seg0, kin = kin0;              // K segment of the current block, block within it
             for (int kb0 = 0; kb0 < n_kb && ok; kb0 += kBitsAhead) {
 #pragma unroll
                 for (int j = 0; j < kBitsAhead; ++j) {
@@ -789,17 +887,36 @@ bool make_amap(CUtensorMap* map, const __half* ptr, int rows, int cols) {
 }  // namespace
 
 cudaError_t prefill_configure() {
-    cudaError_t e = cudaFuncSetAttribute(prefill_gemm_kernel<1>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Shape<1>::kSmem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(prefill_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Shape<2>::kSmem);
+    const void* fns[4] = {(const void*)prefill_gemm_kernel<1, false>, (const void*)prefill_gemm_kernel<1, true>,
+                          (const void*)prefill_gemm_kernel<2, false>, (const void*)prefill_gemm_kernel<2, true>};
+    const int smem[4] = {Shape<1>::kSmem, Shape<1>::kSmem, Shape<2>::kSmem, Shape<2>::kSmem};
+    for (int i = 0; i < 4; ++i) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// Stage 1 may be split along K only when it has fewer tiles than the split
+// buffer has parts even with one sub-tile and two branches; the buffer is
+// reserved for exactly those shapes.
+static bool split_possible(int64_t M, int64_t r) {
+    const int64_t tiles = ((M + kTileM - 1) / kTileM) * 2 * ((r + kTileN - 1) / kTileN);
+    return tiles < kSplitMaxParts;
+}
+
+static size_t split_bytes(int64_t M, int64_t r) {
+    if (!split_possible(M, r)) return 0;
+    return (size_t)kSplitMaxParts * kEpiWarps * kPartFloats * sizeof(float) +
+           (size_t)kSplitMaxParts * kEpiWarps * sizeof(int);
 }
 
 size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     return up(sizeof(WsHeader)) + up(2 * (size_t)M * in) + up(2 * (size_t)M * 2 * r) +
-           up(8 * (size_t)M) + 256 + up(4 * (size_t)((M + kTileM - 1) / kTileM));
+           up(8 * (size_t)M) + 256 + up(4 * (size_t)((M + kTileM - 1) / kTileM)) +
+           up(split_bytes(M, r));
 }
 
 bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
@@ -843,12 +960,30 @@ static int pick_subtiles(const PrefillGemm* p, int grid) {
 template <int MT>
 static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const CUtensorMap& m2,
                                 int grid, cudaStream_t s) {
-    for (int i = 0; i < 2; ++i) plan.n_tiles[i] = (int)gemm_tiles(plan.g[i], MT);
+    const int tiles1 = (int)gemm_tiles(plan.g[0], MT);
+    // split stage 1 along K while it would leave SMs idle: up to 8 parts of at
+    // least 8 K blocks each, at most kSplitMaxParts parts in all
+    int split = 1;
+    if (plan.partial != nullptr) {
+        const int n_kb = plan.g[0].n_kseg * (plan.g[0].k_seg_len / kBlockK);
+        while (split < kSplitMax && tiles1 * (split + 1) <= grid && tiles1 * (split + 1) <= kSplitMaxParts &&
+               n_kb / (split + 1) >= 8)
+            ++split;
+    }
+    plan.split = split;
+    plan.n_tiles[0] = tiles1 * split;
+    plan.n_tiles[1] = (int)gemm_tiles(plan.g[1], MT);
     plan.done_target = kEpiWarps * plan.g[0].n_nseg * ((plan.g[0].n_seg_rows + kTileN - 1) / kTileN);
     const int blocks = (plan.g[0].M + MT * kTileM - 1) / (MT * kTileM);
     cudaError_t e = cudaMemsetAsync(plan.done, 0, sizeof(int) * (size_t)blocks, s);
     if (e != cudaSuccess) return e;
-    prefill_gemm_kernel<MT><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+    if (split > 1 &&
+        (e = cudaMemsetAsync(plan.tickets, 0, sizeof(int) * (size_t)tiles1 * kEpiWarps, s)) != cudaSuccess)
+        return e;
+    if (split > 1)
+        prefill_gemm_kernel<MT, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+    else
+        prefill_gemm_kernel<MT, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
     return cudaGetLastError();
 }
 
@@ -869,6 +1004,13 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     float* lmax = reinterpret_cast<float*>(ws + off);
     off += 256;
     int* done = reinterpret_cast<int*>(ws + off);   // per M block, stage-1 tiles finished
+    off += up(4 * (size_t)((M + kTileM - 1) / kTileM));
+    float* partial = nullptr;                       // stage-1 K split: partial sums, tickets
+    int* tickets = nullptr;
+    if (split_possible(M, r)) {
+        partial = reinterpret_cast<float*>(ws + off);
+        tickets = reinterpret_cast<int*>(ws + off + (size_t)kSplitMaxParts * kEpiWarps * kPartFloats * sizeof(float));
+    }
 
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
     if (e != cudaSuccess) return e;
@@ -882,6 +1024,8 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
 
     PrefillPlan plan = {};
     plan.done = done;
+    plan.partial = partial;
+    plan.tickets = tickets;
     // stage 1: T = (x 2^a) (g o sign V)^T, epilogue applies l, 2^-a, 2^c
     CUtensorMap amap1, amap2;
     if (!make_amap(&amap1, X16, (int)M, (int)in)) return cudaErrorInvalidValue;
