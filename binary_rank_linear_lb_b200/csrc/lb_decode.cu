@@ -424,21 +424,10 @@ __device__ __forceinline__ void consume_rb(const RB& R, const TileRt& T, int rb,
     const float keep1 = up1 ? n2[1] : n2[0];
     const float tot = (keep1 + __shfl_xor_sync(0xffffffffu, send1, 1)) *
                       __half2float(__ushort_as_half(R.h));
-    // Rows 8*gam + 4k .. +3 sit in lanes 16k + gam + 4j (j = 0..3): the lane
-    // with j = 0 adds them with one vector reduction (the L2 takes a 16-byte
-    // reduction at the rate of a 4-byte one); partial or unaligned groups fall
-    // back to one reduction per row.
-    const float t1 = __shfl_down_sync(0xffffffffu, tot, 4);
-    const float t2 = __shfl_down_sync(0xffffffffu, tot, 8);
-    const float t3 = __shfl_down_sync(0xffffffffu, tot, 12);
+    // The 32 lanes hold the rowblock's 32 rows, so one reduction per lane is
+    // a single coalesced 128-byte reduction for the warp.
     const int row = rb * kRowBlock + 8 * gam + rho;       // the row this lane holds
-    const int g0 = row - (rho & 3);                       // first row of its group of 4
-    float* og = T.out + g0;
-    if (g0 + 4 <= T.rows && (reinterpret_cast<uintptr_t>(og) & 15u) == 0) {
-        if ((rho & 3) == 0) red_add_v4_f32(og, tot, t1, t2, t3);
-    } else if (row < T.rows) {
-        red_add_f32(T.out + row, tot);
-    }
+    if (row < T.rows) red_add_f32(T.out + row, tot);
 }
 
 // Rowblock n of a batch (n < n_rb): its tile (selected field by field, so
