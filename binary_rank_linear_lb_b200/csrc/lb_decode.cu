@@ -759,11 +759,10 @@ int decode_grid() { return device_sm_count() * kCtasPerSm; }
 
 // Contiguous unit ranges for G CTAs with the smallest largest cost.  A CTA
 // takes its tiles in batches of up to kTables; a batch costs kTileCost per
-// tile (vector stage + table build, in 1/kDecodeWarps warp iterations) plus
-// ceil(rowblocks / kDecodeWarps) warp iterations, since its warps take the
-// batch's rowblocks kDecodeWarps at a time.  Units run job by job, slice-major
-// inside a job, so a phase is a list of tiles of n_rowblocks units each; a
-// greedy fill is optimal for a given bound, which a bisection minimises.
+// tile (vector stage + table build, in rowblock times) plus one per rowblock.
+// Units run job by job, slice-major inside a job, so a phase is a list of
+// tiles of n_rowblocks units each; a greedy fill is optimal for a given bound,
+// which a bisection minimises.
 namespace {
 template <class F>
 void for_each_tile(const LbJob* jobs, int n_jobs, F f) {
@@ -772,7 +771,10 @@ void for_each_tile(const LbJob* jobs, int n_jobs, F f) {
             for (int s = 0; s < jobs[j].n_slices; ++s)
                 f(std::min(jobs[j].rg, jobs[j].n_rowblocks - g0));
 }
-long long ceil_warps(long long k) { return (k + kDecodeWarps - 1) / kDecodeWarps * kDecodeWarps; }
+// A batch's rowblocks cost in proportion to their number: the lookups are
+// bound by the shared-memory pipe of the SM, so a round in which only some of
+// the 16 warps have a rowblock takes proportionally less time.
+long long rb_cost(long long k) { return k; }
 struct Fill {
     long long closed;   // cost of the CTA's finished batches
     int tiles;          // tiles in its open batch
@@ -782,13 +784,13 @@ struct Fill {
 long long join(const Fill& f, long long take, Fill& g) {
     g = f;
     if (g.tiles == kTables) {
-        g.closed += g.tiles * kTileCost + ceil_warps(g.rb);
+        g.closed += g.tiles * kTileCost + rb_cost(g.rb);
         g.tiles = 0;
         g.rb = 0;
     }
     g.tiles += 1;
     g.rb += take;
-    return g.closed + g.tiles * kTileCost + ceil_warps(g.rb);
+    return g.closed + g.tiles * kTileCost + rb_cost(g.rb);
 }
 // CTAs a greedy fill under cost bound T needs; boundaries go to `out` if set.
 int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
@@ -803,8 +805,7 @@ int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
                 f = Fill{0, 0, 0};
             }
             join(f, 0, g);
-            const long long room =
-                (T - g.closed - g.tiles * kTileCost) / kDecodeWarps * kDecodeWarps - g.rb;
+            const long long room = T - g.closed - g.tiles * kTileCost - g.rb;
             const int take = (int)std::max<long long>(1, std::min<long long>(n, room));
             join(f, take, f);
             n -= take;
