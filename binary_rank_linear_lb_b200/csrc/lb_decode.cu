@@ -771,10 +771,21 @@ void for_each_tile(const LbJob* jobs, int n_jobs, F f) {
             for (int s = 0; s < jobs[j].n_slices; ++s)
                 f(std::min(jobs[j].rg, jobs[j].n_rowblocks - g0));
 }
-// A batch's rowblocks cost in proportion to their number: the lookups are
-// bound by the shared-memory pipe of the SM, so a round in which only some of
-// the 16 warps have a rowblock takes proportionally less time.
-long long rb_cost(long long k) { return k; }
+// A batch's rowblocks cost one each in the rounds where all 16 warps have one
+// (the lookups are bound by the SM's shared-memory pipe); a last, partial
+// round costs in proportion to its rowblocks, but at least kPartialRound,
+// since each of its warps still waits out a rowblock's latency.
+constexpr long long kPartialRound = 8;
+long long rb_cost(long long k) {
+    const long long full = k / kDecodeWarps * kDecodeWarps, rest = k - full;
+    return full + (rest > 0 ? std::max(rest, kPartialRound) : 0);
+}
+// The most rowblocks whose cost fits in `avail`.
+long long rb_room(long long avail) {
+    if (avail <= 0) return 0;
+    const long long full = avail / kDecodeWarps * kDecodeWarps, rest = avail - full;
+    return full + (rest >= kPartialRound ? rest : 0);
+}
 struct Fill {
     long long closed;   // cost of the CTA's finished batches
     int tiles;          // tiles in its open batch
@@ -805,7 +816,7 @@ int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
                 f = Fill{0, 0, 0};
             }
             join(f, 0, g);
-            const long long room = T - g.closed - g.tiles * kTileCost - g.rb;
+            const long long room = rb_room(T - g.closed - g.tiles * kTileCost) - g.rb;
             const int take = (int)std::max<long long>(1, std::min<long long>(n, room));
             join(f, take, f);
             n -= take;
