@@ -18,6 +18,7 @@ timed as the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -46,6 +47,41 @@ WORKLOADS = {
 }
 METRIC = "batch-1 layer-stack tokens/s"
 L2_BYTES = 126 * 1024 * 1024
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# a workload's dominant kernel, from the ncu captures summarised in profiles/.
+# A figure is reported only while the kernel's sources hash to the value it
+# was captured with (otherwise the line carries null).  Stack figures come
+# from a capture of a shorter stack of the same layers and are scaled by the
+# layer count: every layer reads its own weights once, so traffic grows in
+# proportion.  workload: (sources hash, bytes per captured launch, layers
+# captured, or 0 for a single linear).
+MEASURED_TRAFFIC = {
+    "stack70b-1.0": ("b8f7d12833ad983c", 215009024 + 5149184, 2),
+    "prefill-gate7b-1.0-M4096": ("33f9624454cfb4d2", 53061120 + 143990784, 0),
+}
+KERNEL_SOURCES = {
+    "stack_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),
+    "linear_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),
+    "prefill_gemm_kernel": ("lb_prefill.cu", "lb_internal.cuh"),
+}
+
+
+def kernel_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "binary_rank_linear_lb_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, kernel: str, n_layers: int):
+    rec = MEASURED_TRAFFIC.get(workload)
+    if rec is None or rec[0] != kernel_hash(kernel):
+        return None
+    src, nbytes, layers = rec
+    return nbytes * n_layers / layers if layers else float(nbytes)
 
 
 def describe(name: str, n_layers: int = 0) -> str:
@@ -480,6 +516,8 @@ def main():
             launches = 4 * args.steps
         else:
             roof["kernel"] = "linear_program_kernel"
+    roof["traffic"] = measured_traffic(args.workload, roof["kernel"],
+                                       getattr(st, "n_layers", 0))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
