@@ -7,10 +7,10 @@ pitch: ``ld_words`` a multiple of 16, zero padding); the fp32 latents are
 dropped right after packing.
 
 ``signs="bits"`` instead draws the packed words directly from a uniform bit
-source.  The signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so the
-packed matrices have the same distribution; this only shortens the set-up of
-the largest stacks (whose latents would be hundreds of GB of fp32) and is never
-used where a result is compared with the oracle.
+source (``synth.sign_words``).  The signs of i.i.d. N(0, 1) latents are i.i.d.
+fair coins, so the packed matrices have the same distribution; this shortens
+the set-up of the largest stacks (whose latents would be hundreds of GB of
+fp32).  The oracle side of a test draws the same words from the same seeds.
 """
 from __future__ import annotations
 
@@ -51,16 +51,13 @@ def build_branch(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int
         del U
     elif signs == "bits":
         def words(n_rows, k, seed):
-            gen = torch.Generator(device=device)
-            gen.manual_seed(seed)
-            nw = (k + 31) // 32
-            ldw = padded_words(k, pad) if layout == LB_LAYOUT_ROWS else nw
-            w = torch.zeros((n_rows, ldw), dtype=torch.int32, device=device)
-            w[:, :nw] = torch.randint(-2 ** 31, 2 ** 31, (n_rows, nw), generator=gen,
-                                      device=device, dtype=torch.int64).to(torch.int32)
-            if k % 32:
-                w[:, nw - 1] &= (1 << (k % 32)) - 1
-            return w if layout == LB_LAYOUT_ROWS else slice_words(w, k)
+            w = synth.sign_words(n_rows, k, seed, device)
+            if layout != LB_LAYOUT_ROWS:
+                return slice_words(w, k)
+            ldw = padded_words(k, pad)
+            out = torch.zeros((n_rows, ldw), dtype=torch.int32, device=device)
+            out[:, :w.shape[1]] = w
+            return out
         Vp = words(r, in_f, s(synth.KIND_V))
         Up = words(out_f, r, s(synth.KIND_U))
     else:

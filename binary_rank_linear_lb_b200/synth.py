@@ -6,7 +6,9 @@ Every tensor has its own seed derived from (base seed, layer, projection,
 branch, kind), so any single tensor can be regenerated on its own.
 
 Distributions: latents N(0, 1) fp32; scales |N(1, 0.1)| rounded to fp16;
-activations N(0, 1) in the requested dtype.
+activations N(0, 1) in the requested dtype; sign words uniform random bits
+(the signs of i.i.d. N(0, 1) latents are i.i.d. fair coins, so packed words
+drawn directly have the distribution of packed latents).
 """
 from __future__ import annotations
 
@@ -43,6 +45,17 @@ def activation(shape, seed: int, dtype=torch.bfloat16, device="cpu") -> torch.Te
         shape = (shape,)
     z = torch.randn(tuple(shape), generator=_gen(seed, device), device=device, dtype=torch.float32)
     return z.to(dtype)
+
+
+def sign_words(n_rows: int, k: int, seed: int, device="cpu") -> torch.Tensor:
+    """Uniform random packed signs: int32 words [n_rows][ceil(k/32)], bit j of
+    word w of a row standing for element 32*w + j; the bits past k are zero."""
+    nw = (k + 31) // 32
+    w = torch.randint(-2 ** 31, 2 ** 31, (n_rows, nw), generator=_gen(seed, device),
+                      device=device, dtype=torch.int64).to(torch.int32)
+    if k % 32:
+        w[:, nw - 1] &= (1 << (k % 32)) - 1
+    return w
 
 
 def branch_tensors(in_f: int, out_f: int, r: int, base: int, layer: int, proj: int, branch: int,

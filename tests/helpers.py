@@ -19,6 +19,15 @@ def oracle_branch(in_f, out_f, r, base, layer, proj, b, device="cuda"):
                                       host(g).astype(np.float64), host(l).astype(np.float64))
 
 
+def oracle_branch_bits(in_f, out_f, r, base, layer, proj, b, device="cuda"):
+    """A branch whose packed signs are drawn directly as words (model's signs="bits")."""
+    s = lambda k: synth.tensor_seed(base, layer, proj, b, k)
+    words = lambda n, k, kind: synth.sign_words(n, k, s(kind), device).cpu().numpy().view(np.uint32)
+    sc = lambda n, kind: synth.scale(n, s(kind), device).float().cpu().numpy().astype(np.float64)
+    return oracle.Branch(words(r, in_f, synth.KIND_V), words(out_f, r, synth.KIND_U),
+                         sc(out_f, synth.KIND_H), sc(in_f, synth.KIND_G), sc(r, synth.KIND_L))
+
+
 def oracle_linear(in_f, out_f, r, base, layer, proj, nb=2, device="cuda"):
     return [oracle_branch(in_f, out_f, r, base, layer, proj, b, device) for b in range(nb)]
 

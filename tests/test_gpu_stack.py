@@ -14,7 +14,7 @@ from binary_rank_linear_lb_b200 import synth
 from binary_rank_linear_lb_b200.configs import LLAMA2_13B, LLAMA2_7B, LLAMA2_70B, Model
 from binary_rank_linear_lb_b200.model import build_mlp_block, build_stack
 
-from helpers import assert_close, oracle_linear, to_f64
+from helpers import assert_close, oracle_branch_bits, oracle_linear, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -88,6 +88,31 @@ def test_13b_stack_full_depth_0p1():
 def test_70b_stack_two_layers_full_width():
     _, _, y, h_ref, _ = run_stack(LLAMA2_70B, 0.55, 2, base=7)
     assert_close(y.cpu().numpy(), h_ref, what="70B x2 @ 0.55")
+
+
+@pytest.mark.slow
+def test_70b_stack_full_depth_bench_workload():
+    """bench.py's default workload as it times it: all 80 layers of the 70B-shaped stack at
+    1.0 bits/weight, two branches, sign words drawn directly, the sliced layout, one
+    cooperative launch; the oracle runs the same seeded layers one at a time."""
+    model, base = LLAMA2_70B, 0
+    st = build_stack(model, 1.0, base=base, signs="bits")
+    x = synth.activation(model.hidden, 1234, torch.bfloat16, "cuda")
+    y = st.forward(x).cpu().numpy()
+    torch.cuda.synchronize()
+    assert st.status() == lb.LB_OK
+    del st
+    torch.cuda.empty_cache()
+    rk = model.ranks(1.0)
+    h = to_f64(x)
+    for li in range(model.n_layers):
+        L = {}
+        for p, name in enumerate(ostack_names()):
+            i, o = model.shapes()[p]
+            L[name] = ostack.Linear([oracle_branch_bits(i, o, rk[p], base, li, p, b)
+                                     for b in range(2)], i, o, rk[p])
+        h = ostack.decoder_stack(h, [L], model.n_heads, model.n_kv_heads, model.head_dim)
+    assert_close(y, h, what="70B x80 @ 1.0, bench workload")
 
 
 @pytest.mark.parametrize("bpw", [1.0, 0.55, 0.3, 0.1])
