@@ -52,6 +52,7 @@ constexpr long long kWaitLimit = 4000000000LL;    // cycles (~2 s)
 constexpr uint32_t kSuspendNs = 20000;            // longest hardware suspension per try_wait
 constexpr int kMaxStages = 4;
 constexpr int kPartFloats = 8 * 32 * 32;          // one epilogue warp's share of a tile (8 chunks)
+constexpr int kSplit2Max = 4;                      // K parts of a stage-2 tile at most
 constexpr int kSplitMaxParts = 160;               // stage-1 tile parts the split buffer holds
 constexpr int kSplitMax = 3;                      // K parts of one stage-1 tile (the last one folds the others)
 
@@ -240,6 +241,8 @@ struct PrefillGemm {
 // epilogue warp writes its fp32 partial sums to `partial` and takes a ticket
 // for its region of the tile; the warp that draws the last ticket adds the
 // other parts' partials to its own accumulator and finishes the region into T.
+// With few stage-2 tiles, stage 2 is split along K too (`split2` parts); its
+// parts add their sums into y, which the host zeroes first.
 struct PrefillPlan {
     PrefillGemm g[2];
     int n_tiles[2];      // tiles of each GEMM (stage 1: tiles x split)
@@ -248,6 +251,8 @@ struct PrefillPlan {
     int split;           // K parts of a stage-1 tile (1: no split)
     float* partial;      // [tile][part][epilogue warp][kPartFloats] fp32 partial sums
     int* tickets;        // [tile][epilogue warp], zeroed per call
+    int split2;          // K parts of a stage-2 tile (1: no split; else y, zeroed first,
+                         // takes each part's sums by reduction)
 };
 
 namespace {
@@ -323,14 +328,14 @@ struct TileRef {
     const CUtensorMap* map;
     int stage2, t, part, mb, nseg, nt, kb_per_seg, kb0, kb1;
 };
-template <bool SPLIT>
+template <bool SPLIT, bool SPLIT2>
 __device__ __forceinline__ TileRef tile_ref(const PrefillPlan& plan, const CUtensorMap* amap1,
                                             const CUtensorMap* amap2, int t) {
     TileRef r;
     r.stage2 = t >= plan.n_tiles[0] ? 1 : 0;
     r.g = r.stage2 ? &plan.g[1] : &plan.g[0];
     r.map = r.stage2 ? amap2 : amap1;
-    const int parts = (SPLIT && !r.stage2) ? plan.split : 1;
+    const int parts = r.stage2 ? (SPLIT2 ? plan.split2 : 1) : (SPLIT ? plan.split : 1);
     const int tl = t - (r.stage2 ? plan.n_tiles[0] : 0);
     r.t = tl / parts;
     r.part = tl - r.t * parts;
@@ -359,7 +364,7 @@ __device__ __forceinline__ uint4 load_l8(const PrefillGemm& g, int nseg, int n0,
     return make_uint4(e2[0], e2[1], e2[2], e2[3]);
 }
 
-template <int MT, bool SPLIT>
+template <int MT, bool SPLIT, bool SPLIT2>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const __grid_constant__ CUtensorMap amap2,
@@ -419,7 +424,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 if (pb >= cur.kb1) {
                     t += gridDim.x;
                     if (t >= n_tiles) return;
-                    r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+                    r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
                     pb = r.kb0 + (pb - cur.kb1);
                     if (pb >= r.kb1 || !ready(r)) return;
                 }
@@ -429,14 +434,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         tma_prefetch_2d(r.map, acol(r, pb), (r.mb * MT + j) * kTileM);
             };
             if (blockIdx.x < n_tiles) {
-                const TileRef r0 = tile_ref<SPLIT>(plan, &amap1, &amap2, blockIdx.x);
+                const TileRef r0 = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, blockIdx.x);
                 if (ready(r0))
                     for (int kb = r0.kb0; kb < r0.kb0 + kPrefetchAhead && kb < r0.kb1; ++kb)
                         prefetch(r0, blockIdx.x, kb - kPrefetchAhead);
             }
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
-                const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+                const TileRef r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
                 const PrefillGemm& g = *r.g;
                 if (r.stage2) {
                     // wait (bounded) for the M block's rows of T, then order the TMA
@@ -485,7 +490,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 if (!wait_bar(ctl, &ctl->acc_empty[buf], (use & 1) ^ 1, err)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * MT * kTileN);
-                const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+                const TileRef r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
                 bool ok = true;
                 for (int kb = r.kb0; kb < r.kb1; ++kb, ++it) {
                     const int s = it % kStages;
@@ -523,7 +528,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
         const uint32_t my_row = stg + (uint32_t)lane * 128u;
         int tl = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
-            const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+            const TileRef r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
             const PrefillGemm& g = *r.g;
             const int mb = r.mb, nseg = r.nseg, nt = r.nt;
             const int ldt = g.n_nseg * g.n_seg_rows;      // T row pitch (stage 1)
@@ -668,6 +673,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const int cc = lane & 7;
                     const int col = n0 + 4 * cc;
                     const bool vec = (g.n_seg_rows & 3) == 0;
+                    const bool add = SPLIT2 && plan.split2 > 1;   // K parts reduce into y
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {              // rows 4i .. 4i+3, 8 lanes per row
                         const int rr = 4 * i + (lane >> 3);
@@ -678,10 +684,18 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         if (m0 + rr < g.M && col < g.n_seg_rows) {
                             float* dst = g.y + (size_t)(m0 + rr) * g.n_seg_rows + col;
                             if (vec) {
-                                *reinterpret_cast<float4*>(dst) = o;
+                                if (add)
+                                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                                                 :: "l"(dst), "f"(o.x), "f"(o.y), "f"(o.z), "f"(o.w)
+                                                 : "memory");
+                                else
+                                    *reinterpret_cast<float4*>(dst) = o;
                             } else {
                                 const float ov[4] = {o.x, o.y, o.z, o.w};
-                                for (int e = 0; e < 4 && col + e < g.n_seg_rows; ++e) dst[e] = ov[e];
+                                for (int e = 0; e < 4 && col + e < g.n_seg_rows; ++e) {
+                                    if (add) atomicAdd(dst + e, ov[e]);
+                                    else dst[e] = ov[e];
+                                }
                             }
                         }
                     }
@@ -706,7 +720,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
         uint32_t ph = 0;                             // and the parity of its current use
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            const TileRef r = tile_ref<SPLIT>(plan, &amap1, &amap2, t);
+            const TileRef r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
             const PrefillGemm& g = *r.g;
             const int nseg = r.nseg, nt = r.nt, kb_per_seg = r.kb_per_seg;
             const int n_kb = r.kb1 - r.kb0;          // K blocks of this tile (its part of K)
@@ -887,10 +901,15 @@ bool make_amap(CUtensorMap* map, const __half* ptr, int rows, int cols) {
 }  // namespace
 
 cudaError_t prefill_configure() {
-    const void* fns[4] = {(const void*)prefill_gemm_kernel<1, false>, (const void*)prefill_gemm_kernel<1, true>,
-                          (const void*)prefill_gemm_kernel<2, false>, (const void*)prefill_gemm_kernel<2, true>};
-    const int smem[4] = {Shape<1>::kSmem, Shape<1>::kSmem, Shape<2>::kSmem, Shape<2>::kSmem};
-    for (int i = 0; i < 4; ++i) {
+    const void* fns[6] = {(const void*)prefill_gemm_kernel<1, false, false>,
+                          (const void*)prefill_gemm_kernel<1, true, false>,
+                          (const void*)prefill_gemm_kernel<1, true, true>,
+                          (const void*)prefill_gemm_kernel<2, false, false>,
+                          (const void*)prefill_gemm_kernel<2, true, false>,
+                          (const void*)prefill_gemm_kernel<2, true, true>};
+    const int smem[6] = {Shape<1>::kSmem, Shape<1>::kSmem, Shape<1>::kSmem,
+                         Shape<2>::kSmem, Shape<2>::kSmem, Shape<2>::kSmem};
+    for (int i = 0; i < 6; ++i) {
         const cudaError_t e =
             cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
         if (e != cudaSuccess) return e;
@@ -972,7 +991,20 @@ static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const 
     }
     plan.split = split;
     plan.n_tiles[0] = tiles1 * split;
-    plan.n_tiles[1] = (int)gemm_tiles(plan.g[1], MT);
+    // and stage 2 the same way (its parts reduce into y, zeroed below)
+    const int tiles2 = (int)gemm_tiles(plan.g[1], MT);
+    const int n_kb2 = plan.g[1].n_kseg * (plan.g[1].k_seg_len / kBlockK);
+    int split2 = 1;
+    while (split2 < kSplit2Max && tiles2 * (split2 + 1) <= grid && n_kb2 / (split2 + 1) >= 8)
+        ++split2;
+    // LB_PREFILL_SPLIT2=1..4 in the environment (read on every call) fixes the
+    // split, at most one part per K block so that no part is empty
+    if (const char* env = std::getenv("LB_PREFILL_SPLIT2")) {
+        const int v = std::atoi(env);
+        if (v >= 1 && v <= kSplit2Max) split2 = v < n_kb2 ? v : n_kb2;
+    }
+    plan.split2 = split2;
+    plan.n_tiles[1] = tiles2 * split2;
     plan.done_target = kEpiWarps * plan.g[0].n_nseg * ((plan.g[0].n_seg_rows + kTileN - 1) / kTileN);
     const int blocks = (plan.g[0].M + MT * kTileM - 1) / (MT * kTileM);
     cudaError_t e = cudaMemsetAsync(plan.done, 0, sizeof(int) * (size_t)blocks, s);
@@ -980,10 +1012,18 @@ static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const 
     if (split > 1 &&
         (e = cudaMemsetAsync(plan.tickets, 0, sizeof(int) * (size_t)tiles1 * kEpiWarps, s)) != cudaSuccess)
         return e;
-    if (split > 1)
-        prefill_gemm_kernel<MT, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+    if (split2 > 1 &&
+        (e = cudaMemsetAsync(plan.g[1].y, 0,
+                             sizeof(float) * (size_t)plan.g[1].M * (size_t)plan.g[1].n_seg_rows, s)) !=
+            cudaSuccess)
+        return e;
+    // the split instantiations cost registers, so shapes that split nothing run without them
+    if (split2 > 1)
+        prefill_gemm_kernel<MT, true, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+    else if (split > 1)
+        prefill_gemm_kernel<MT, true, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
     else
-        prefill_gemm_kernel<MT, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+        prefill_gemm_kernel<MT, false, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
     return cudaGetLastError();
 }
 

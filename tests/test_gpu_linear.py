@@ -125,6 +125,20 @@ def test_prefill_subtile_shapes(shape, M, subtiles, monkeypatch):
     assert_close(got, ref, what=f"{shape} M={M} sub-tiles={subtiles}")
 
 
+@pytest.mark.parametrize("split2", ["1", "2", "3", "4"])
+@pytest.mark.parametrize("subtiles", ["1", "2"])
+@pytest.mark.parametrize("M,shape", [(64, (640, 1000, 192)), (300, (1024, 1001, 128)),
+                                     (100, (512, 256, 64))])
+def test_prefill_stage2_k_split(M, shape, subtiles, split2, monkeypatch):
+    """The second GEMM split along K into 1-4 parts that add into y (vector and scalar
+    reductions: out = 1001 is not a multiple of 4), with both tile shapes."""
+    monkeypatch.setenv("LB_PREFILL_SUBTILES", subtiles)
+    monkeypatch.setenv("LB_PREFILL_SPLIT2", split2)
+    in_f, out_f, r = shape
+    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=9, layout=lb.LB_LAYOUT_SLICES)
+    assert_close(got, ref, what=f"{shape} M={M} sub-tiles={subtiles} split2={split2}")
+
+
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
 def test_prefill_path_dtypes_and_one_branch(dtype):
     got, ref = run_case(768, 512, 128, 64, dtype, nb=1, base=4)
