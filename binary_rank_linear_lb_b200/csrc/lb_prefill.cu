@@ -54,7 +54,7 @@ constexpr int kMaxStages = 4;
 constexpr int kPartFloats = 8 * 32 * 32;          // one epilogue warp's share of a tile (8 chunks)
 constexpr int kSplit2Max = 4;                      // K parts of a stage-2 tile at most
 constexpr int kSplitMaxParts = 160;               // stage-1 tile parts the split buffer holds
-constexpr int kSplitMax = 3;                      // K parts of one stage-1 tile (the last one folds the others)
+constexpr int kSplitMax = 4;                      // K parts of one stage-1 tile (the last one folds the others)
 
 constexpr int kEpiBytes = 32 * 128;                // per-warp epilogue staging: 32 rows x 128 bytes
 constexpr int kPrefetchAhead = 6;                 // K blocks of A pulled into L2 ahead of the TMA loads
@@ -980,7 +980,7 @@ template <int MT>
 static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const CUtensorMap& m2,
                                 int grid, cudaStream_t s) {
     const int tiles1 = (int)gemm_tiles(plan.g[0], MT);
-    // split stage 1 along K while it would leave SMs idle: up to 8 parts of at
+    // split stage 1 along K while it would leave SMs idle: up to kSplitMax parts of at
     // least 8 K blocks each, at most kSplitMaxParts parts in all
     int split = 1;
     if (plan.partial != nullptr) {
