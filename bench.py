@@ -59,7 +59,7 @@ L2_BYTES = 126 * 1024 * 1024
 # captured, or 0 for a single linear).
 MEASURED_TRAFFIC = {
     "stack70b-1.0": ("b8f7d12833ad983c", 215009024 + 5149184, 2),
-    "prefill-gate7b-1.0-M4096": ("33f9624454cfb4d2", 53061120 + 143990784, 0),
+    "prefill-gate7b-1.0-M4096": ("2b8315c018d03de4", 53410304 + 144020992, 0),
 }
 KERNEL_SOURCES = {
     "stack_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),
