@@ -303,8 +303,12 @@ class Stack:
             raise LbError(LB_ERR_INVALID_ARG, "lb_stack_workspace_size")
         dev = device if device is not None else torch.device("cuda")
         self.workspace = torch.empty(size, dtype=torch.uint8, device=dev)
-        _check(lib().lb_stack_prepare(ctypes.byref(self.desc), _ptr(self.workspace), size,
-                                      _stream(stream)), "lb_stack_prepare")
+        self.prepare(stream)
+
+    def prepare(self, stream=None) -> None:
+        """(Re)write the plan into the workspace: lb_stack_prepare (also clears a timeout)."""
+        _check(lib().lb_stack_prepare(ctypes.byref(self.desc), _ptr(self.workspace),
+                                      self.workspace.numel(), _stream(stream)), "lb_stack_prepare")
 
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:

@@ -232,9 +232,12 @@ lb_status lb_stack_prepare(const lb_stack_desc *d, void *workspace, size_t ws_by
 /*
  * lb_stack_forward — one token through a prepared stack.
  *   x : device bf16 [hidden];  y : device fp32 [hidden], overwritten.
- * One memset and one cooperative persistent kernel on `stream`.  Grid-wide
- * waits inside the kernel are bounded; if one gives up the kernel returns
- * early and lb_workspace_status reports LB_ERR_TIMEOUT.
+ * One cooperative persistent kernel on `stream` (it zeroes each phase's
+ * accumulators itself, one phase ahead).  Grid-wide waits inside the kernel
+ * are bounded (about 2 s); if one gives up, the kernel returns early, y is
+ * undefined and lb_workspace_status reports LB_ERR_TIMEOUT.  The error is
+ * sticky: later calls on the workspace return at once, until lb_stack_prepare
+ * runs on it again.
  */
 lb_status lb_stack_forward(const lb_stack_desc *d, void *workspace, size_t ws_bytes,
                            const void *x, float *y, void *stream);

@@ -3,6 +3,8 @@
 The oracle runs the whole stack itself from the same seeded inputs; no GPU
 intermediate ever enters it.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -70,6 +72,34 @@ def test_forward_host_matches_device():
     yh = torch.empty(SMALL.hidden, dtype=torch.float32).pin_memory()
     st.forward_host(xh, yh)
     torch.testing.assert_close(yh, y, rtol=1e-4, atol=1e-4 * y.abs().max().item())
+
+
+def test_bounded_wait_gives_up_and_workspace_recovers():
+    """A grid-wide wait that is never met ends in an error status, not a hang.  The
+    arrival counter in the workspace header is preset so that phase 0's arrivals wrap it
+    to zero, short of the first wait's target; each CTA gives up after its ~2 s bound, the
+    call ends and the workspace reports LB_ERR_TIMEOUT.  The error is sticky (the next
+    call returns at once) until the plan is prepared again, after which the stack gives
+    the same result as before."""
+    ranks = [64, 32, 32, 64, 96, 96, 96]
+    st = build_stack(SMALL, 1.0, base=4, n_layers=2, ranks=ranks)
+    x = synth.activation(SMALL.hidden, 11, torch.bfloat16, "cuda")
+    y_ok = st.forward(x).clone()
+    assert st.status() == lb.LB_OK
+    grid = torch.cuda.get_device_properties(0).multi_processor_count
+    st.workspace[:4].view(torch.int32)[0] = -grid          # 2^32 - G arrivals so far
+    t0 = time.perf_counter()
+    st.forward(x)
+    assert st.status() == lb.LB_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 30.0
+    t0 = time.perf_counter()
+    st.forward(x)                                           # sticky: returns at once
+    assert st.status() == lb.LB_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 1.0
+    st.prepare()
+    y = st.forward(x)
+    assert st.status() == lb.LB_OK
+    torch.testing.assert_close(y, y_ok, rtol=1e-5, atol=1e-5 * y_ok.abs().max().item())
 
 
 @pytest.mark.parametrize("bpw", [0.55, 0.1])
