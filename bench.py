@@ -58,7 +58,7 @@ L2_BYTES = 126 * 1024 * 1024
 # proportion.  workload: (sources hash, bytes per captured launch, layers
 # captured, or 0 for a single linear).
 MEASURED_TRAFFIC = {
-    "stack70b-1.0": ("b8f7d12833ad983c", 215009024 + 5149184, 2),
+    "stack70b-1.0": ("0e3097b271ec3bde", 214949888 + 3339008, 2),
     "prefill-gate7b-1.0-M4096": ("2b8315c018d03de4", 53410304 + 144020992, 0),
 }
 KERNEL_SOURCES = {

@@ -619,10 +619,22 @@ __device__ __forceinline__ void phase_begin(const Smem& sm, const CallArgs& args
     if (c.u < c.u_end) batch_begin(sm, args, c);
 }
 
-// The rest of the phase, after the grid-wide wait.
+// Request this warp's first rowblock of the current batch into R.
+__device__ __forceinline__ void first_load(const Cursor& c, RB& R) {
+    const int n = (int)(threadIdx.x >> 5);
+    if (n < c.n_rb) {
+        int rb;
+        const TileRt T = batch_tile(c, n, rb);
+        load_rb(T, rb, R);
+    }
+}
+
+// The rest of the phase, after the grid-wide wait.  loaded: this warp's first
+// rowblock of the first batch is already requested (during the wait).
 __device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, Cursor& c,
                                           RB (&buf)[kDepth],
-                          const uint32_t (&Bc)[2][4], const uint32_t (&S)[4]) {
+                                          const uint32_t (&Bc)[2][4], const uint32_t (&S)[4],
+                                          bool loaded) {
     const int G = gridDim.x, cta = blockIdx.x;
     float* zp = resolve(sm.phase->zero_ptr, args);
     const int zn = sm.phase->zero_n;
@@ -630,12 +642,15 @@ __device__ __forceinline__ void run_phase(const Smem& sm, const CallArgs& args, 
         for (int i = cta * kDecodeThreads + threadIdx.x; i < zn; i += G * kDecodeThreads)
             zp[i] = 0.0f;
     }
+    bool skip = loaded;
     while (c.u < c.u_end) {
         // each warp's first rowblock is requested before the vector is staged
         // (32 KB per CTA), its second after the tables are built
         {
             const int n = (int)(threadIdx.x >> 5);
-            if (n < c.n_rb) {
+            const bool sk = skip;
+            skip = false;
+            if (!sk && n < c.n_rb) {
                 int rb;
                 const TileRt T = batch_tile(c, n, rb);
                 load_rb(T, rb, buf[0]);
@@ -685,14 +700,14 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
     Cursor cur;
     RB buf[kDepth];
     phase_begin(sm, args, cur);
+    bool loaded = false;
     for (int p = 0; p < n_phases; ++p) {
-        run_phase(sm, args, cur, buf, Bc, S);
+        run_phase(sm, args, cur, buf, Bc, S, loaded);
         if (p + 1 < n_phases) {
             // Announce completion, then use the wait: switch to the next
-            // phase's plan, load the scales of its first batch and fetch the
-            // plan of the phase after it into the buffer this phase used.
-            // Nothing bulky is in flight while the CTA waits: the wait and
-            // the staging loads after it are the latency-critical requests.
+            // phase's plan, load the scales of its first batch, fetch the
+            // plan of the phase after it into the buffer this phase used and
+            // request the first rowblocks.
             grid_arrive(hdr);
             if (wp == kDecodeWarps - 1) plan_wait();
             __syncthreads();
@@ -706,6 +721,12 @@ __device__ __forceinline__ void run_program(const LbPhase* phases, int n_phases,
                 __syncthreads();
                 cache_plan(phases, p + 2, jobs, splits, starts, nb ^ 1);
             }
+            // The sign words do not depend on earlier phases, so every warp but
+            // the poller's requests its first rowblock now and the HBM latency
+            // overlaps the wait; the poller's warp keeps no loads in flight
+            // ahead of its polls (measured: loads there delay the acquire).
+            loaded = wp != 0;
+            if (loaded && cur.u < cur.u_end) first_load(cur, buf[0]);
             if (!grid_wait(hdr, (unsigned)(p + 1) * G, sm.flag)) {
                 if (wp == kDecodeWarps - 1) plan_wait();
                 return;

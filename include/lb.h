@@ -51,7 +51,7 @@ typedef enum {
     LB_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned                */
     LB_ERR_UNSUPPORTED = 3,   /* valid but not supported (e.g. no sm_100 device) */
     LB_ERR_CUDA = 4,          /* a CUDA runtime call failed                      */
-    LB_ERR_TIMEOUT = 5,       /* a device-side wait gave up (see lb_stack_status)*/
+    LB_ERR_TIMEOUT = 5,       /* a device-side wait gave up (lb_workspace_status) */
     LB_ERR_WORKSPACE = 6      /* workspace missing or smaller than required      */
 } lb_status;
 
