@@ -151,6 +151,12 @@ typedef struct {
  * LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED (no sm_100 device), LB_ERR_CUDA.
  * (The tensor-core path also reads g in 16-byte vectors; a g that is not
  * 16-byte aligned keeps the call on the lookup-table kernels.)
+ * The tensor-core path splits either GEMM along K when its tiles would leave
+ * SMs idle (small M or low rank); two environment variables, read on every
+ * call, fix its choices for testing, with results equal up to rounding:
+ * LB_PREFILL_SUBTILES=1|2 (128-row M sub-tiles per expanded sign tile) and
+ * LB_PREFILL_SPLIT2=1..4 (K parts of a second-GEMM tile, at most one per 64
+ * columns of K).
  */
 lb_status lb_linear_forward(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
                             int64_t out, int64_t r, const lb_branch *br, int n_branches,
