@@ -60,7 +60,8 @@ EXPORTS = ("lb_status_string", "lb_version", "lb_pack_signs", "lb_linear_forward
            "lb_linear_workspace_size", "lb_linear_path", "lb_stack_workspace_size",
            "lb_stack_prepare", "lb_stack_forward", "lb_stack_forward_host",
            "lb_workspace_status", "lb_stack_output", "lb_linear_forward_noalloc",
-           "lb_noalloc_scratch_bytes", "lb_pack_signs_sliced", "lb_packed_words")
+           "lb_noalloc_scratch_bytes", "lb_pack_signs_sliced", "lb_packed_words",
+           "lb_stack_plan_host")
 
 _lib = None
 
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.lb_stack_workspace_size.restype = sz
         L.lb_stack_prepare.argtypes = [vp, vp, sz, vp]
         L.lb_stack_prepare.restype = st
+        L.lb_stack_plan_host.argtypes = [vp, ctypes.c_int, vp, sz, vp, vp]
+        L.lb_stack_plan_host.restype = st
         L.lb_stack_forward.argtypes = [vp, vp, sz, vp, vp, vp]
         L.lb_stack_forward.restype = st
         L.lb_stack_forward_host.argtypes = [vp, vp, sz, vp, vp, vp]

@@ -511,8 +511,11 @@ size_t lb_stack_workspace_size(const lb_stack_desc* d) {
     return stack_layout(d).total;
 }
 
-lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_bytes,
-                           void* stream) {
+namespace {
+// Validation shared by the plan builders: descriptor, workspace pointer and
+// size, branch alignment.
+lb_status stack_plan_args(const lb_stack_desc* d, const void* workspace, size_t ws_bytes,
+                          StackLayout& L) {
     if (!stack_desc_ok(d) || !workspace) return LB_ERR_INVALID_ARG;
     if (!aligned(workspace, 256)) return LB_ERR_ALIGNMENT;
     const int nb = d->n_branches;
@@ -523,35 +526,83 @@ lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_by
                 if (!branch_aligned(d->lin[((size_t)l * LB_N_PROJ + p) * nb + b]))
                     return LB_ERR_ALIGNMENT;
         }
-    const StackLayout L = stack_layout(d);
+    L = stack_layout(d);
     if (ws_bytes < L.total) return LB_ERR_WORKSPACE;
-    lb_status st = ensure_device();
-    if (st != LB_OK) return st;
+    return LB_OK;
+}
+
+// The stack's execution plan for a grid of G CTAs, its pointers into the
+// workspace at address ws (host copies; nothing is dereferenced).
+struct StackPlan {
     std::vector<LbPhase> phases;
     std::vector<LbJob> jobs;
-    build_stack_plan(d, L, static_cast<char*>(workspace), phases, jobs);
-    if ((int)phases.size() != L.n_phases || (int)jobs.size() != L.n_jobs) return LB_ERR_CUDA;
-    std::vector<int> split((size_t)(kMaxGrid + 1) * L.n_phases, 0);
-    const int G = decode_grid();
-    plan_splits(phases.data(), L.n_phases, jobs.data(), G, split.data());
-    std::vector<LbStart> starts((size_t)kMaxGrid * L.n_phases, LbStart{});
-    plan_starts(phases.data(), L.n_phases, jobs.data(), split.data(), G, starts.data());
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<int> split;
+    std::vector<LbStart> starts;
+};
+bool make_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws, int G,
+                     StackPlan& P) {
+    build_stack_plan(d, L, ws, P.phases, P.jobs);
+    if ((int)P.phases.size() != L.n_phases || (int)P.jobs.size() != L.n_jobs) return false;
+    P.split.assign((size_t)(kMaxGrid + 1) * L.n_phases, 0);
+    plan_splits(P.phases.data(), L.n_phases, P.jobs.data(), G, P.split.data());
+    P.starts.assign((size_t)kMaxGrid * L.n_phases, LbStart{});
+    plan_starts(P.phases.data(), L.n_phases, P.jobs.data(), P.split.data(), G, P.starts.data());
+    return true;
+}
+}  // namespace
+
+lb_status lb_stack_prepare(const lb_stack_desc* d, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    StackLayout L;
+    lb_status st = stack_plan_args(d, workspace, ws_bytes, L);
+    if (st != LB_OK) return st;
+    if ((st = ensure_device()) != LB_OK) return st;
     char* ws = static_cast<char*>(workspace);
+    StackPlan P;
+    if (!make_stack_plan(d, L, ws, decode_grid(), P)) return LB_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, L.acc_end, s) != cudaSuccess) return LB_ERR_CUDA;
-    if (cudaMemcpyAsync(ws + L.phases, phases.data(), sizeof(LbPhase) * phases.size(),
+    if (cudaMemcpyAsync(ws + L.phases, P.phases.data(), sizeof(LbPhase) * P.phases.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
-    if (cudaMemcpyAsync(ws + L.jobs, jobs.data(), sizeof(LbJob) * jobs.size(),
+    if (cudaMemcpyAsync(ws + L.jobs, P.jobs.data(), sizeof(LbJob) * P.jobs.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
-    if (cudaMemcpyAsync(ws + L.splits, split.data(), sizeof(int) * split.size(),
+    if (cudaMemcpyAsync(ws + L.splits, P.split.data(), sizeof(int) * P.split.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
-    if (cudaMemcpyAsync(ws + L.starts, starts.data(), sizeof(LbStart) * starts.size(),
+    if (cudaMemcpyAsync(ws + L.starts, P.starts.data(), sizeof(LbStart) * P.starts.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess)
         return LB_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return LB_ERR_CUDA;
+    return LB_OK;
+}
+
+lb_status lb_stack_plan_host(const lb_stack_desc* d, int grid, void* image, size_t image_bytes,
+                             size_t* offsets, int* counts) {
+    StackLayout L;
+    const lb_status st = stack_plan_args(d, image, image_bytes, L);
+    if (st != LB_OK) return st;
+    if (grid < 1 || !offsets || !counts) return LB_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(image);
+    StackPlan P;
+    if (!make_stack_plan(d, L, ws, grid, P)) return LB_ERR_INVALID_ARG;
+    std::memset(ws, 0, L.total);
+    std::memcpy(ws + L.phases, P.phases.data(), sizeof(LbPhase) * P.phases.size());
+    std::memcpy(ws + L.jobs, P.jobs.data(), sizeof(LbJob) * P.jobs.size());
+    std::memcpy(ws + L.splits, P.split.data(), sizeof(int) * P.split.size());
+    std::memcpy(ws + L.starts, P.starts.data(), sizeof(LbStart) * P.starts.size());
+    offsets[0] = L.phases;
+    offsets[1] = L.jobs;
+    offsets[2] = L.splits;
+    offsets[3] = L.starts;
+    offsets[4] = L.acc_end;
+    counts[0] = L.n_phases;
+    counts[1] = L.n_jobs;
+    counts[2] = kMaxGrid;
+    counts[3] = (int)sizeof(LbPhase);
+    counts[4] = (int)sizeof(LbJob);
+    counts[5] = (int)sizeof(LbStart);
     return LB_OK;
 }
 

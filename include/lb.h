@@ -236,6 +236,22 @@ lb_status lb_stack_prepare(const lb_stack_desc *d, void *workspace, size_t ws_by
                            void *stream);
 
 /*
+ * lb_stack_plan_host — for inspection and tests, on the host only (no CUDA
+ * call): the plan lb_stack_prepare would write for a grid of `grid` CTAs,
+ * written into the host buffer `image` (256-byte aligned, >= the stack's
+ * workspace size) at its workspace offsets, its workspace pointers taken
+ * relative to `image` itself; the rest of the image is zero.  The packed
+ * factors and scales are not read.
+ *   offsets[5] : byte offsets of the phase headers, jobs, split table, start
+ *                table, and the end of the accumulator region
+ *   counts[6]  : phases, jobs, the split/start table stride in CTAs, and the
+ *                sizes in bytes of a phase header, a job and a start record
+ * Same argument errors as lb_stack_prepare (grid < 1: LB_ERR_INVALID_ARG).
+ */
+lb_status lb_stack_plan_host(const lb_stack_desc *d, int grid, void *image, size_t image_bytes,
+                             size_t *offsets, int *counts);
+
+/*
  * lb_stack_forward — one token through a prepared stack.
  *   x : device bf16 [hidden];  y : device fp32 [hidden], overwritten.
  * One cooperative persistent kernel on `stream` (it zeroes each phase's
