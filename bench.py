@@ -255,72 +255,67 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def cpu_oracle_rate(name: str, budget_s: float = 12.0):
-    """Oracle tokens/s on a bounded sample: a few whole layers of one token, scaled."""
+def oracle_sampler(name: str):
+    """One bounded sample of a workload for the oracle on the host cores.
+
+    Returns (step, tokens per step, what one step is): a stack step is one decoder
+    layer of one token (1/n_layers of a token), an MLP-block step one whole token, a
+    single-linear step one row of x.  The packed words and scales are drawn once
+    (uniform bits, |N(1, 0.1)| scales), outside the steps."""
     import numpy as np
     import oracle
     from oracle import stack as ostack
-    from binary_rank_linear_lb_b200.configs import MODELS
+    from binary_rank_linear_lb_b200.configs import MODELS, rank_for
     model_name, bpw, kind = WORKLOADS[name][:3]
     rng = np.random.default_rng(0)
-    if kind == "linear":
-        from binary_rank_linear_lb_b200.configs import rank_for
-        (i, o), M = model_name, WORKLOADS[name][3]
-        r = rank_for(bpw, i, o)
+
+    def branches(i, o, r):
         brs = []
         for _ in range(2):
             Vp = rng.integers(0, 2 ** 32, size=(r, (i + 31) // 32), dtype=np.uint64).astype(np.uint32)
             Up = rng.integers(0, 2 ** 32, size=(o, (r + 31) // 32), dtype=np.uint64).astype(np.uint32)
             sc = lambda n: np.abs(1 + 0.1 * rng.standard_normal(n))
             brs.append(oracle.Branch(Vp, Up, sc(o), sc(i), sc(r)))
+        return brs
+
+    if kind == "linear":
+        (i, o), M = model_name, WORKLOADS[name][3]
+        r = rank_for(bpw, i, o)
+        brs = branches(i, o, r)
         xs = rng.standard_normal((1, i))
-        t0 = time.perf_counter()
-        reps = 0
-        while reps < 1000:
-            oracle.forward(xs, brs, i, o, r)
-            reps += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
-        dt = (time.perf_counter() - t0) / reps
-        return 1.0 / dt, oracle.threads(), f"{reps} rows of x through the full layer (rows/s)"
+        return (lambda: oracle.forward(xs, brs, i, o, r)), 1.0, (
+            f"one row of x through the {i}->{o} layer (r={r}, 2 branches)")
     model = MODELS[model_name]
     rk = model.ranks(bpw)
 
     def lin(p):
         i, o = model.shapes()[p]
-        r = rk[p]
-        brs = []
-        for _ in range(2):
-            Vp = rng.integers(0, 2 ** 32, size=(r, (i + 31) // 32), dtype=np.uint64).astype(np.uint32)
-            Up = rng.integers(0, 2 ** 32, size=(o, (r + 31) // 32), dtype=np.uint64).astype(np.uint32)
-            sc = lambda n: np.abs(1 + 0.1 * rng.standard_normal(n))
-            brs.append(oracle.Branch(Vp, Up, sc(o), sc(i), sc(r)))
-        return ostack.Linear(brs, i, o, r)
+        return ostack.Linear(branches(i, o, rk[p]), i, o, rk[p])
 
     x = rng.standard_normal(model.hidden)
-    t0 = time.perf_counter()
-    layers_done = 0
     if kind == "mlp":
         g, u, d = lin(4), lin(5), lin(6)
-        t0 = time.perf_counter()
-        reps = 0
-        while True:
-            ostack.mlp_block(x, g, u, d)
-            reps += 1
-            if time.perf_counter() - t0 > budget_s or reps >= 50:
-                break
-        dt = (time.perf_counter() - t0) / reps
-        return 1.0 / dt, oracle.threads(), f"{reps} full MLP-block tokens"
-    elapsed = 0.0
-    while elapsed < budget_s and layers_done < model.n_layers:
-        L = {n: lin(p) for p, n in enumerate(("q", "k", "v", "o", "gate", "up", "down"))}
-        t0 = time.perf_counter()
-        ostack.decoder_stack(x, [L], model.n_heads, model.n_kv_heads, model.head_dim)
-        elapsed += time.perf_counter() - t0
-        layers_done += 1
-    per_token = elapsed / layers_done * model.n_layers
-    return 1.0 / per_token, oracle.threads(), (
-        f"{layers_done} of {model.n_layers} decoder layers of one token, time scaled to all layers")
+        return (lambda: ostack.mlp_block(x, g, u, d)), 1.0, "one token through the MLP block"
+    L = {n: lin(p) for p, n in enumerate(("q", "k", "v", "o", "gate", "up", "down"))}
+    return ((lambda: ostack.decoder_stack(x, [L], model.n_heads, model.n_kv_heads,
+                                          model.head_dim)),
+            1.0 / model.n_layers,
+            f"one decoder layer of one token (1/{model.n_layers} of a token)")
+
+
+def cpu_oracle_rate(name: str, budget_s: float = 12.0):
+    """Oracle tokens/s from repeated bounded samples, about budget_s seconds in all."""
+    import oracle
+    step, tokens, what = oracle_sampler(name)
+    step()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        step()
+        n += 1
+        if time.perf_counter() - t0 > budget_s or n >= 1000:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return tokens / dt, oracle.threads(), f"{n} timed samples, each {what}"
 
 
 # ---------------------------------------------------------------- sweeps
@@ -340,7 +335,7 @@ def _time_events(fn, iters, flush=None):
     return statistics.median(ts)
 
 
-def sweep_prefill(device, flush, tflops_peak):
+def sweep_prefill(device, flush, tflops_peak, fp8_peak=None):
     """The 7B gate projection (4096 -> 11008) over the token batch M, both paths."""
     import torch
     import binary_rank_linear_lb_b200 as lb
@@ -367,8 +362,106 @@ def sweep_prefill(device, flush, tflops_peak):
                         "path": "tcgen05" if lb.linear_path(M, in_f, out_f, r) else "lut-decode",
                         "ms": ms, "tflops": fl / ms / 1e9, "gbs": by / ms / 1e6,
                         "tensor_frac_fp16": fl / ms / 1e9 / tflops_peak,
-                        "tensor_frac_fp8": fl / ms / 1e9 / (2 * tflops_peak)})
+                        "tensor_frac_fp8": fl / ms / 1e9 / fp8_peak if fp8_peak else None})
             del x, y, ws
+    return out
+
+
+def measure_fp8_peak(device):
+    """Dense FP8 (e4m3) matmul rate of the library GEMM, 8192^3, best of 10 (TFLOP/s).
+
+    Plain library timing (torch._scaled_mm), the denominator of the FP8 tensor-core
+    fraction; None with the reason if the call is not available."""
+    import torch
+    n = 8192
+    try:
+        a = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=device).to(torch.float8_e4m3fn).t()
+        one = torch.tensor(1.0, device=device)
+        f = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        best = min(_time_events(f, 1) for _ in range(10))
+        del a, b
+        return {"fp8_tflops": 2 * n ** 3 / best / 1e9, "how": "torch._scaled_mm e4m3 8192^3, "
+                "bf16 out, best of 10 (CUDA events)"}
+    except Exception as e:   # pragma: no cover - depends on the library build
+        return {"fp8_tflops": None, "how": f"torch._scaled_mm failed: {type(e).__name__}: {e}"}
+
+
+def sweep_layer70b_vs_dense(device, flush, hbm_peak):
+    """One 8192 -> 28672 factorised linear at batch 1 for each bits/weight, and a dense
+    bf16 matrix-vector product of the same shape (torch.matmul over 470 MB of weights;
+    a library call, context only).  L2 flushed before every timed call."""
+    import torch
+    import binary_rank_linear_lb_b200 as lb
+    from binary_rank_linear_lb_b200 import synth
+    from binary_rank_linear_lb_b200.configs import linear_bytes, rank_for
+    from binary_rank_linear_lb_b200.model import build_linear
+    in_f, out_f = 8192, 28672
+    W = torch.randn(out_f, in_f, device=device, dtype=torch.bfloat16)
+    xd = torch.randn(in_f, 1, device=device, dtype=torch.bfloat16)
+    for _ in range(3):
+        torch.matmul(W, xd)
+    dense_ms = _time_events(lambda: torch.matmul(W, xd), 20, flush)
+    dense_bytes = W.numel() * 2
+    del W
+    torch.cuda.empty_cache()
+    rows = []
+    for bpw in (1.0, 0.55, 0.3, 0.1):
+        r = rank_for(bpw, in_f, out_f)
+        brs = build_linear(in_f, out_f, r, base=31, device=device, signs="bits")
+        x = synth.activation((1, in_f), 5, torch.bfloat16, device)
+        y = torch.empty((1, out_f), dtype=torch.float32, device=device)
+        ws = torch.empty(lb.linear_workspace_size(1, in_f, out_f, r, 2), dtype=torch.uint8,
+                         device=device)
+        fn = lambda: lb.linear_forward(x, brs, in_f, out_f, r, y=y, workspace=ws)
+        for _ in range(3):
+            fn()
+        ms = _time_events(fn, 20, flush)
+        by = linear_bytes(in_f, out_f, r)
+        rows.append({"bits_per_weight": bpw, "r": r, "ms": ms, "bytes": by,
+                     "gbs": by / ms / 1e6, "hbm_frac": by / ms / 1e6 / hbm_peak,
+                     "speedup_vs_dense_bf16": dense_ms / ms})
+        del brs, x, y, ws
+    return {"dense_bf16_ms": dense_ms, "dense_bf16_gbs": dense_bytes / dense_ms / 1e6,
+            "layers": rows,
+            "pages": "A100, same layer shape: speed-up grows as bits/weight fall, up to 11.6x"}
+
+
+def sweep_small_m(device, flush):
+    """The 7B gate projection at M = 1..16, 24, 32, 48, 64 rows on both kernel paths
+    (LB_LINEAR_PATH forces one), and the path lb_linear_forward picks by itself."""
+    import torch
+    import binary_rank_linear_lb_b200 as lb
+    from binary_rank_linear_lb_b200 import synth
+    from binary_rank_linear_lb_b200.configs import rank_for
+    from binary_rank_linear_lb_b200.model import build_linear
+    in_f, out_f = 4096, 11008
+    out = []
+    for bpw in (1.0, 0.1):
+        r = rank_for(bpw, in_f, out_f)
+        brs = build_linear(in_f, out_f, r, base=78, device=device, signs="bits")
+        for M in list(range(1, 17)) + [24, 32, 48, 64]:
+            x = synth.activation((M, in_f), 6, torch.bfloat16, device)
+            y = torch.empty((M, out_f), dtype=torch.float32, device=device)
+            rec = {"bits_per_weight": bpw, "r": r, "M": M}
+            for path, key in ((None, "default_ms"), ("0", "lut_ms"), ("1", "tensor_ms")):
+                if path is None:
+                    os.environ.pop("LB_LINEAR_PATH", None)
+                    rec["default_path"] = "tcgen05" if lb.linear_path(M, in_f, out_f, r) else "lut"
+                else:
+                    os.environ["LB_LINEAR_PATH"] = path
+                ws = torch.empty(lb.linear_workspace_size(M, in_f, out_f, r, 2),
+                                 dtype=torch.uint8, device=device)
+                fn = lambda: lb.linear_forward(x, brs, in_f, out_f, r, y=y, workspace=ws)
+                for _ in range(3):
+                    fn()
+                rec[key] = _time_events(fn, 10, flush)
+                del ws
+            os.environ.pop("LB_LINEAR_PATH", None)
+            rec["default_over_best"] = rec["default_ms"] / min(rec["lut_ms"], rec["tensor_ms"])
+            out.append(rec)
     return out
 
 
@@ -418,17 +511,27 @@ def main():
 
     if args.impl == "reference":
         # The reference arm is the oracle itself (no installable reference exists),
-        # run on the host cores by rank 0 only.
+        # run on the host cores by rank 0 only.  Each step is one bounded sample of
+        # the workload (see oracle_sampler); value is tokens/s from the timed steps.
         if rank != 0:
             return 0
-        rate, cores, sample = cpu_oracle_rate(args.workload,
-                                              budget_s=max(5.0, 20.0 / max(1, args.steps)))
+        import oracle
+        step, tokens, what = oracle_sampler(args.workload)
+        for _ in range(args.warmup):
+            step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        ms_per_step = (time.perf_counter() - t0) * 1e3 / args.steps
+        rate = tokens / (ms_per_step / 1e3)
+        sample = f"each step is {what}; value = tokens per step / time per step"
         line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1e3 / rate, "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": ms_per_step, "tokens_per_step": tokens,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": describe(args.workload)},
-                "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores,
+                "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": oracle.threads(),
                                  "kind": "oracle", "sample": sample},
                 "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -505,15 +608,22 @@ def main():
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_kind,
             "kernel": "stack_program_kernel"}
-    launches = args.steps
+    launches = args.steps                    # stacks: one cooperative launch per token
     if kind == "linear":
+        # the tensor-core path launches lmax, pre-pass and GEMM kernels; the lookup-table
+        # path one kernel per chunk of up to 8 rows
+        launches = args.steps * (3 if lb.linear_path(st.M, st.in_f, st.out_f, st.r)
+                                 else (st.M + 7) // 8)
         if lb.linear_path(st.M, st.in_f, st.out_f, st.r):
             tf = st.flops / (ms_per_step / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": tf, "peak": tflops_peak, "unit": "TFLOP/s",
                     "frac": tf / tflops_peak, "traffic": None,
                     "peak_source": peak_kind + " (bf16 dense; fp16 runs at the same rate)",
-                    "kernel": "prefill_gemm_kernel", "fp8_frac": tf / (2 * tflops_peak)}
-            launches = 4 * args.steps
+                    "kernel": "prefill_gemm_kernel"}
+            fp8 = measure_fp8_peak(device)
+            if fp8["fp8_tflops"]:
+                roof["fp8_frac"] = tf / fp8["fp8_tflops"]
+                roof["fp8_peak"] = fp8
         else:
             roof["kernel"] = "linear_program_kernel"
     roof["traffic"] = measured_traffic(args.workload, roof["kernel"],
@@ -543,11 +653,14 @@ def main():
         del st
         torch.cuda.empty_cache()
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+        fp8 = measure_fp8_peak(device)
         line["sweeps"] = {
-            "prefill_gate7b": sweep_prefill(device, flush, tflops_peak),
+            "peaks": {"hbm_gbs": hbm_peak, "fp16_tflops": tflops_peak, "source": peak_kind,
+                      "fp8_tflops_measured": fp8["fp8_tflops"], "fp8_how": fp8["how"]},
+            "prefill_gate7b": sweep_prefill(device, flush, tflops_peak, fp8["fp8_tflops"]),
+            "small_m_gate7b": sweep_small_m(device, flush),
+            "layer70b_vs_dense": sweep_layer70b_vs_dense(device, flush, hbm_peak),
             "stacks": sweep_stacks(device, args.workload, hbm_peak),
-            "peaks": {"hbm_gbs": hbm_peak, "fp16_tflops": tflops_peak,
-                      "fp8_tflops_nominal_ratio": 2 * tflops_peak, "source": peak_kind},
         }
     if rank == 0:
         print(json.dumps(line), flush=True)

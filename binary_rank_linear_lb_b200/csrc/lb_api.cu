@@ -1,6 +1,7 @@
 // Host side of liblb.so: argument validation, workspace layout, plan building
 // and launches for every entry point declared in include/lb.h.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -406,26 +407,55 @@ lb_status lb_pack_signs_sliced(const float* latent, int64_t rows, int64_t cols, 
                : LB_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// LB_LINEAR_PATH=0|1 in the environment (read on every call) forces the
+// lookup-table (0) or the tensor-core (1) kernels wherever the shapes allow
+// them, for measuring the two paths against each other.
+static int forced_path() {
+    const char* env = std::getenv("LB_LINEAR_PATH");
+    if (env == nullptr || env[1] != 0) return -1;
+    return env[0] == '0' ? 0 : env[0] == '1' ? 1 : -1;
+}
+
 // The tensor-core path runs for at least kPrefillMinM rows when the shapes
 // allow its 64-wide K blocks.
 static bool use_prefill(int64_t M, int64_t in, int64_t out, int64_t r) {
+    const int f = forced_path();
+    if (f >= 0) return f == 1 && prefill_shape_ok(M, in, out, r);
     return M >= kPrefillMinM && prefill_shape_ok(M, in, out, r);
 }
 
-size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r, int n_branches) {
-    if (M <= 0 || in <= 0 || out <= 0 || r <= 0 || n_branches < 1 || n_branches > 2) return 0;
-    if (use_prefill(M, in, out, r)) return prefill_workspace_bytes(M, in, r);
+namespace lb {
+
+size_t decode_workspace_bytes(int64_t M, int64_t r, int n_branches) {
     const int64_t mc = std::min<int64_t>(M, kMaxDecodeM);
     return sizeof(WsHeader) + round_up(sizeof(float) * (size_t)(mc * n_branches * r), 256);
 }
 
-int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r) {
-    return use_prefill(M, in, out, r) ? 1 : 0;
+LinearRoute default_route(int64_t M, int64_t in, int64_t out, int64_t r, const lb_branch* br,
+                          int n_branches) {
+    if (!br || n_branches < 1 || n_branches > 2 || !use_prefill(M, in, out, r))
+        return kRouteDecode;
+    // the tensor-core path reads g in 16-byte vectors and sign words in pairs
+    for (int b = 0; b < n_branches; ++b)
+        if (!(aligned(br[b].g, 16) &&
+              (br[b].layout == LB_LAYOUT_SLICES ||
+               (((br[b].ld_v ? br[b].ld_v : cdiv(in, 32)) & 1) == 0 &&
+                ((br[b].ld_u ? br[b].ld_u : cdiv(r, 32)) & 1) == 0))))
+            return kRouteDecode;
+    return kRoutePrefill;
 }
 
-lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t in, int64_t out,
-                            int64_t r, const lb_branch* br, int n_branches, float* y,
-                            void* workspace, size_t ws_bytes, void* stream) {
+size_t route_workspace_bytes(LinearRoute route, int64_t M, int64_t in, int64_t r, int nb) {
+    if (route == kRouteDecode) return decode_workspace_bytes(M, r, nb);
+    return prefill_workspace_bytes(M, in, r, route == kRoutePrefill);
+}
+
+lb_status linear_forward_route(const void* x, lb_dtype x_dtype, int64_t M, int64_t in,
+                               int64_t out, int64_t r, const lb_branch* br, int n_branches,
+                               float* y, void* workspace, size_t ws_bytes, size_t ws_need,
+                               cudaStream_t s, LinearRoute route) {
     if (!x || !y || !br || !workspace) return LB_ERR_INVALID_ARG;
     if (M <= 0 || in <= 0 || out <= 0 || r <= 0) return LB_ERR_INVALID_ARG;
     if (in > (1 << 28) || out > (1 << 28) || r > (1 << 24)) return LB_ERR_INVALID_ARG;
@@ -437,28 +467,27 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(workspace, 16)) return LB_ERR_ALIGNMENT;
     for (int b = 0; b < n_branches; ++b)
         if (!branch_aligned(br[b])) return LB_ERR_ALIGNMENT;
-    if (ws_bytes < lb_linear_workspace_size(M, in, out, r, n_branches)) return LB_ERR_WORKSPACE;
+    if (route != kRouteDecode && default_route(M, in, out, r, br, n_branches) == kRouteDecode)
+        return LB_ERR_INVALID_ARG;   // the tensor-core path cannot take these shapes or pointers
+    if (ws_bytes < ws_need || ws_bytes < route_workspace_bytes(route, M, in, r, n_branches))
+        return LB_ERR_WORKSPACE;
     lb_status st = ensure_device();
     if (st != LB_OK) return st;
 
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (use_prefill(M, in, out, r)) {
-        // the tensor-core path reads g in 16-byte vectors and sign words in pairs
-        bool ok = true;
-        for (int b = 0; b < n_branches; ++b)
-            ok = ok && aligned(br[b].g, 16) &&
-                 (br[b].layout == LB_LAYOUT_SLICES ||
-                  (((br[b].ld_v ? br[b].ld_v : cdiv(in, 32)) & 1) == 0 &&
-                   ((br[b].ld_u ? br[b].ld_u : cdiv(r, 32)) & 1) == 0));
-        if (ok)
-            return launch_prefill(x, vec_kind_for(x_dtype), M, in, out, r, br, n_branches, y,
-                                  workspace, s) == cudaSuccess
-                       ? LB_OK
-                       : LB_ERR_CUDA;
-    }
+    if (route != kRouteDecode)
+        return launch_prefill(x, vec_kind_for(x_dtype), M, in, out, r, br, n_branches, y,
+                              workspace, s, route == kRoutePrefill) == cudaSuccess
+                   ? LB_OK
+                   : LB_ERR_CUDA;
+    if ((int64_t)std::min<int64_t>(M, kMaxDecodeM) * out > 0x7fffffff) return LB_ERR_INVALID_ARG;
     const size_t xsz = x_dtype == LB_F32 ? 4 : 2;
     WsHeader* hdr = static_cast<WsHeader*>(workspace);
     float* t = reinterpret_cast<float*>(static_cast<char*>(workspace) + sizeof(WsHeader));
+    // The header (barrier counter, error) is cleared once per call, so a
+    // device-side time-out in one chunk of rows stays visible after the later
+    // chunks (which then return at once); the kernel leaves the barrier counter
+    // at zero when it finishes.  Each chunk clears its t accumulators.
+    if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return LB_ERR_CUDA;
     for (int64_t m0 = 0; m0 < M; m0 += kMaxDecodeM) {
         const int mc = (int)std::min<int64_t>(kMaxDecodeM, M - m0);
         LinearPlan plan;
@@ -494,16 +523,38 @@ lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t 
                 J.out = y + (size_t)(m0 + m) * (size_t)out;
                 add_job(p1, jobs, J);
             }
-        if ((int64_t)mc * out > 0x7fffffff) return LB_ERR_INVALID_ARG;
         plan.phases[0] = p0;
         plan.phases[1] = p1;
         std::copy(jobs.begin(), jobs.end(), plan.jobs);
         plan_splits(plan.phases, 2, plan.jobs, decode_grid(), plan.split);
-        const size_t zero_bytes = sizeof(WsHeader) + sizeof(float) * (size_t)mc * n_branches * r;
-        if (cudaMemsetAsync(workspace, 0, zero_bytes, s) != cudaSuccess) return LB_ERR_CUDA;
+        if (cudaMemsetAsync(t, 0, sizeof(float) * (size_t)mc * n_branches * r, s) != cudaSuccess)
+            return LB_ERR_CUDA;
         if (launch_linear_plan(plan, hdr, 2, s) != cudaSuccess) return LB_ERR_CUDA;
     }
     return LB_OK;
+}
+
+}  // namespace lb
+
+extern "C" {
+
+size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r, int n_branches) {
+    if (M <= 0 || in <= 0 || out <= 0 || r <= 0 || n_branches < 1 || n_branches > 2) return 0;
+    if (use_prefill(M, in, out, r)) return prefill_workspace_bytes(M, in, r);
+    return decode_workspace_bytes(M, r, n_branches);
+}
+
+int lb_linear_path(int64_t M, int64_t in, int64_t out, int64_t r) {
+    return use_prefill(M, in, out, r) ? 1 : 0;
+}
+
+lb_status lb_linear_forward(const void* x, lb_dtype x_dtype, int64_t M, int64_t in, int64_t out,
+                            int64_t r, const lb_branch* br, int n_branches, float* y,
+                            void* workspace, size_t ws_bytes, void* stream) {
+    return linear_forward_route(x, x_dtype, M, in, out, r, br, n_branches, y, workspace, ws_bytes,
+                                lb_linear_workspace_size(M, in, out, r, n_branches),
+                                static_cast<cudaStream_t>(stream),
+                                default_route(M, in, out, r, br, n_branches));
 }
 
 size_t lb_stack_workspace_size(const lb_stack_desc* d) {

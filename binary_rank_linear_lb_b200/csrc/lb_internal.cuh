@@ -264,11 +264,29 @@ void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* sp
 // Tensor-core prefill path (lb_prefill.cu).
 constexpr int kPrefillMinM = 16;             // lb_linear_forward uses it from this many rows
 cudaError_t prefill_configure();
-size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r);
+// with_split: room for the stage-1 K split's partial sums (tens of MB when the
+// split is possible); without it the launch never splits stage 1.
+size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r, bool with_split = true);
 bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r);
 cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int64_t out,
                            int64_t r, const lb_branch* br, int nb, float* y, void* workspace,
-                           cudaStream_t s);
+                           cudaStream_t s, bool allow_split = true);
+
+// Which kernels a linear call runs (lb_api.cu).
+enum LinearRoute { kRouteDecode = 0, kRoutePrefill = 1, kRoutePrefillNoSplit = 2 };
+// The tensor-core path when lb_linear_forward would take it (shape and pointer
+// alignment), else the decode path.
+LinearRoute default_route(int64_t M, int64_t in, int64_t out, int64_t r, const lb_branch* br,
+                          int n_branches);
+// Workspace bytes of the decode path, and of any route.
+size_t decode_workspace_bytes(int64_t M, int64_t r, int n_branches);
+size_t route_workspace_bytes(LinearRoute route, int64_t M, int64_t in, int64_t r, int nb);
+// lb_linear_forward on a given route, with its argument checks; the call is
+// refused (LB_ERR_WORKSPACE) unless ws_bytes >= ws_need and >= what the route needs.
+lb_status linear_forward_route(const void* x, lb_dtype x_dtype, int64_t M, int64_t in,
+                               int64_t out, int64_t r, const lb_branch* br, int n_branches,
+                               float* y, void* workspace, size_t ws_bytes, size_t ws_need,
+                               cudaStream_t s, LinearRoute route);
 
 // Packer (lb_pack.cu).  sliced: write the sliced layout (ld_words unused).
 cudaError_t launch_pack(const float* latent, int64_t rows, int64_t cols, int64_t ld, int axis,

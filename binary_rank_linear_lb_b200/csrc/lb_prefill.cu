@@ -931,11 +931,11 @@ static size_t split_bytes(int64_t M, int64_t r) {
            (size_t)kSplitMaxParts * kEpiWarps * sizeof(int);
 }
 
-size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r) {
+size_t prefill_workspace_bytes(int64_t M, int64_t in, int64_t r, bool with_split) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     return up(sizeof(WsHeader)) + up(2 * (size_t)M * in) + up(2 * (size_t)M * 2 * r) +
            up(8 * (size_t)M) + 256 + up(4 * (size_t)((M + kTileM - 1) / kTileM)) +
-           up(split_bytes(M, r));
+           (with_split ? up(split_bytes(M, r)) : 0);
 }
 
 bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
@@ -1029,7 +1029,7 @@ static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const 
 
 cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int64_t out,
                            int64_t r, const lb_branch* br, int nb, float* y, void* workspace,
-                           cudaStream_t s) {
+                           cudaStream_t s, bool allow_split) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     char* ws = static_cast<char*>(workspace);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -1047,7 +1047,7 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     off += up(4 * (size_t)((M + kTileM - 1) / kTileM));
     float* partial = nullptr;                       // stage-1 K split: partial sums, tickets
     int* tickets = nullptr;
-    if (split_possible(M, r)) {
+    if (allow_split && split_possible(M, r)) {
         partial = reinterpret_cast<float*>(ws + off);
         tickets = reinterpret_cast<int*>(ws + off + (size_t)kSplitMaxParts * kEpiWarps * kPartFloats * sizeof(float));
     }

@@ -33,7 +33,9 @@
  *     anything is launched.  Launch failures return LB_ERR_CUDA.  Faults that
  *     happen later on the device surface at the caller's next synchronisation.
  *   - Matrices are row-major.  x is M x in, y is M x out.
- *   - The library keeps no state between calls and is thread-safe.
+ *   - The library is thread-safe.  On the host it caches per-device properties;
+ *     on the device it keeps no state between calls, except the fixed scratch
+ *     array of lb_linear_forward_noalloc (see there).
  */
 #ifndef LB_H
 #define LB_H
@@ -156,7 +158,10 @@ typedef struct {
  * call, fix its choices for testing, with results equal up to rounding:
  * LB_PREFILL_SUBTILES=1|2 (128-row M sub-tiles per expanded sign tile) and
  * LB_PREFILL_SPLIT2=1..4 (K parts of a second-GEMM tile, at most one per 64
- * columns of K).
+ * columns of K).  LB_LINEAR_PATH=0|1, also read on every call (and by
+ * lb_linear_workspace_size and lb_linear_path), forces the lookup-table (0) or
+ * the tensor-core (1) kernels wherever the shapes allow them, so that the two
+ * can be timed against each other; both give the layer within the same bound.
  */
 lb_status lb_linear_forward(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
                             int64_t out, int64_t r, const lb_branch *br, int n_branches,
@@ -175,14 +180,25 @@ size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
  * Same arguments and results as lb_linear_forward, without `workspace`: the
  * scratch lives in a fixed __device__ array of lb_noalloc_scratch_bytes()
  * bytes (256 KiB) inside liblb.so, which every GPU that loads the library holds
- * until the process exits.  Calls whose lb_linear_workspace_size(M, in, out, r,
- * n_branches) exceeds it return LB_ERR_WORKSPACE (with two branches: r up to 32736 for
- * M = 1, up to 4092 for M >= 8).  The first call on a device looks up the
- * array's device address; make that first call before any stream capture.
+ * until the process exits.  Limits, with S = lb_noalloc_scratch_bytes():
+ *   - where lb_linear_forward takes the tensor-core path, this call takes it
+ *     too if 256 + pad(2*M*in) + pad(4*M*r) + pad(8*M) + 256 + pad(4*ceil(M/128))
+ *     <= S (pad = round up to 256 bytes), running stage 1 without its K split
+ *     (e.g. M = 16, in = 4096, r = 1472 fits; M = 64, in = 4096 does not);
+ *   - otherwise it takes the lookup-table path, which needs
+ *     256 + pad(4 * min(M, 8) * n_branches * r) <= S (two branches: r up to
+ *     32736 for M = 1, up to 4092 for M >= 8);
+ *   - beyond both it returns LB_ERR_WORKSPACE.
+ * Both paths give the layer's result within the same fp32 accuracy.
+ * A call on a device looks up the array's device address until one lookup
+ * succeeds; make the first call on each device before any stream capture.
  * All calls share the array and it keeps the last call's contents; each call
  * clears what must start at zero, and calls that overlap on the GPU (streams
  * not ordered with each other) race on it.  It never calls cudaMalloc,
- * cudaFree or any allocating routine.
+ * cudaFree or any allocating routine.  A device-side wait that gives up
+ * (about 2 s) leaves y undefined; the array's status word is not exposed, so
+ * callers that must detect that case should use lb_linear_forward and
+ * lb_workspace_status.
  */
 lb_status lb_linear_forward_noalloc(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
                                     int64_t out, int64_t r, const lb_branch *br,

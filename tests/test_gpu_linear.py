@@ -174,3 +174,43 @@ def test_prefill_large_activations_do_not_overflow():
     ref = oracle.forward(to_f64(x), ob, in_f, out_f, r)
     for m in range(32):
         assert_close(y[m].cpu().numpy(), ref[m], what=f"row {m}")
+
+
+@pytest.mark.parametrize("bpw", [1.0, 0.1])
+@pytest.mark.parametrize("M", [64, 4096])
+def test_prefill_timed_7b_gate_every_m_block(M, bpw):
+    """The 7B gate projection (4096 -> 11008) exactly as bench.py times it: seed 0, sign
+    words drawn directly, the sliced layout, bf16 x from seed 1, one lb_linear_forward call
+    (at M = 4096: 32 M blocks of 128 rows, no K split, stage-2 tiles waiting per block on
+    their stage-1 rows).  The oracle evaluates every output feature of the first, a middle
+    and the last row of every 128-row M block."""
+    from helpers import oracle_branch_bits
+    in_f, out_f = 4096, 11008
+    r = rank_for(bpw, in_f, out_f)
+    assert lb.linear_path(M, in_f, out_f, r) == 1
+    brs = build_linear(in_f, out_f, r, base=0, signs="bits")
+    x = synth.activation((M, in_f), 1, torch.bfloat16, "cuda")
+    y = lb.linear_forward(x, brs, in_f, out_f, r)
+    torch.cuda.synchronize()
+    toks = sorted({t for b0 in range(0, M, 128)
+                   for t in (b0, b0 + min(64, M - b0 - 1), min(b0 + 127, M - 1))})
+    ob = [oracle_branch_bits(in_f, out_f, r, 0, 0, 0, b) for b in range(2)]
+    ref = oracle.forward(to_f64(x[toks]), ob, in_f, out_f, r)
+    got = y[toks].cpu().numpy().astype(np.float64)
+    for i, t in enumerate(toks):
+        assert_close(got[i], ref[i], what=f"7B gate M={M} @ {bpw}, token {t}")
+    assert_close(got, ref, what=f"7B gate M={M} @ {bpw}")
+
+
+@pytest.mark.parametrize("path", ["0", "1"])
+@pytest.mark.parametrize("M", [1, 5, 8, 15, 16, 24, 64])
+def test_forced_paths_small_m(M, path, monkeypatch):
+    """Both kernel paths at the token counts where lb_linear_forward switches between them
+    (LB_LINEAR_PATH forces one: the tensor-core kernels also below 16 rows, the lookup-table
+    kernels also above), on a 64-aligned shape with a ragged output width."""
+    monkeypatch.setenv("LB_LINEAR_PATH", path)
+    in_f, out_f, r = 1024, 1001, 192
+    assert lb.linear_path(M, in_f, out_f, r) == int(path)
+    got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=12)
+    for m in range(M):
+        assert_close(got[m], ref[m], what=f"M={M} path={path} row {m}")

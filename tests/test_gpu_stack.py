@@ -53,6 +53,39 @@ def run_stack(model, bpw, n_layers, base, ranks=None, layout=lb.LB_LAYOUT_SLICES
 SMALL = Model("small", hidden=256, inter=512, n_layers=3, n_heads=4, n_kv_heads=2, head_dim=64)
 
 
+def prefix_output(st, model, n_layers, x):
+    """The residual stream after the first n_layers layers of GPU stack st: the same
+    device-resident weights run as a stack of n_layers layers (x itself for 0)."""
+    if n_layers == 0:
+        return to_f64(x)
+    rk = [[int(st._ranks[li * 7 + p]) for p in range(7)] for li in range(n_layers)]
+    pre = lb.Stack(st._keep[:n_layers], rk, model.hidden, model.inter, model.n_heads,
+                   model.n_kv_heads, model.head_dim)
+    h = to_f64(pre.forward(x))
+    torch.cuda.synchronize()
+    assert pre.status() == lb.LB_OK
+    return h
+
+
+def check_layer_teacher_forced(st, model, li, h_in, h_out, L, what):
+    """Every linear of layer li of a GPU stack run, each against the oracle fed with the
+    GPU's own input to that linear (teacher-forced): q, k, v from rmsnorm(h_in); o from the
+    GPU's v; gate, up from rmsnorm(h_in + o); down from the GPU's gate and up.  o and down
+    add into the residual stream, so their sum is checked as h_out - h_in."""
+    a = ostack.rmsnorm(h_in)
+    got = {p: to_f64(st.output(li, i)) for i, p in ((0, "q"), (1, "k"), (2, "v"), (4, "gate"),
+                                                      (5, "up"))}
+    for name in ("q", "k", "v"):
+        assert_close(got[name], L[name](a), what=f"{what} layer {li} {name}")
+    o_ref = L["o"](ostack.gqa_broadcast(got["v"], model.n_heads, model.n_kv_heads,
+                                        model.head_dim))
+    a2 = ostack.rmsnorm(h_in + o_ref)
+    for name in ("gate", "up"):
+        assert_close(got[name], L[name](a2), what=f"{what} layer {li} {name}")
+    down_ref = L["down"](ostack.silu(got["gate"]) * got["up"])
+    assert_close(h_out - h_in, o_ref + down_ref, what=f"{what} layer {li} o + down")
+
+
 @pytest.mark.parametrize("layout", [lb.LB_LAYOUT_SLICES, lb.LB_LAYOUT_ROWS])
 def test_small_decoder_stack_and_intermediates(layout):
     st, x, y, h_ref, outs = run_stack(SMALL, 1.0, 3, base=3, ranks=[64, 32, 32, 64, 96, 96, 96],
@@ -102,10 +135,19 @@ def test_bounded_wait_gives_up_and_workspace_recovers():
     torch.testing.assert_close(y, y_ok, rtol=1e-5, atol=1e-5 * y_ok.abs().max().item())
 
 
+def check_two_layer_stack(model, bpw, base, what):
+    st, x, y, h_ref, _ = run_stack(model, bpw, 2, base=base)
+    assert_close(y.cpu().numpy(), h_ref, what=what)
+    layers = oracle_layers(model, model.ranks(bpw), 2, base)
+    h1 = prefix_output(st, model, 1, x)
+    check_layer_teacher_forced(st, model, 0, to_f64(x), h1, layers[0], what)
+    check_layer_teacher_forced(st, model, 1, h1, to_f64(y), layers[1], what)
+
+
 @pytest.mark.parametrize("bpw", [0.55, 0.1])
 def test_13b_stack_two_layers_full_width(bpw):
-    _, _, y, h_ref, _ = run_stack(LLAMA2_13B, bpw, 2, base=5)
-    assert_close(y.cpu().numpy(), h_ref, what=f"13B x2 @ {bpw}")
+    """The final hidden state, and every linear of both layers teacher-forced."""
+    check_two_layer_stack(LLAMA2_13B, bpw, 5, f"13B x2 @ {bpw}")
 
 
 @pytest.mark.slow
@@ -116,8 +158,8 @@ def test_13b_stack_full_depth_0p1():
 
 @pytest.mark.slow
 def test_70b_stack_two_layers_full_width():
-    _, _, y, h_ref, _ = run_stack(LLAMA2_70B, 0.55, 2, base=7)
-    assert_close(y.cpu().numpy(), h_ref, what="70B x2 @ 0.55")
+    """The final hidden state, and every linear of both layers teacher-forced."""
+    check_two_layer_stack(LLAMA2_70B, 0.55, 7, "70B x2 @ 0.55")
 
 
 @pytest.mark.slow
@@ -131,18 +173,30 @@ def test_70b_stack_full_depth_bench_workload():
     y = st.forward(x).cpu().numpy()
     torch.cuda.synchronize()
     assert st.status() == lb.LB_OK
-    del st
-    torch.cuda.empty_cache()
     rk = model.ranks(1.0)
-    h = to_f64(x)
-    for li in range(model.n_layers):
+
+    def layer(li):
         L = {}
         for p, name in enumerate(ostack_names()):
             i, o = model.shapes()[p]
             L[name] = ostack.Linear([oracle_branch_bits(i, o, rk[p], base, li, p, b)
                                      for b in range(2)], i, o, rk[p])
-        h = ostack.decoder_stack(h, [L], model.n_heads, model.n_kv_heads, model.head_dim)
-    assert_close(y, h, what="70B x80 @ 1.0, bench workload")
+        return L
+
+    # every linear of the first and the last layer, teacher-forced
+    last = model.n_layers - 1
+    h_first = prefix_output(st, model, 1, x)
+    h_last = prefix_output(st, model, last, x)
+    what = "70B x80 @ 1.0, bench workload"
+    check_layer_teacher_forced(st, model, 0, to_f64(x), h_first, layer(0), what)
+    check_layer_teacher_forced(st, model, last, h_last, y.astype(np.float64), layer(last), what)
+    del st
+    torch.cuda.empty_cache()
+    # and the final hidden state against the oracle run free from x
+    h = to_f64(x)
+    for li in range(model.n_layers):
+        h = ostack.decoder_stack(h, [layer(li)], model.n_heads, model.n_kv_heads, model.head_dim)
+    assert_close(y, h, what=what)
 
 
 @pytest.mark.parametrize("bpw", [1.0, 0.55, 0.3, 0.1])
