@@ -30,11 +30,12 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the C oracle with gcc (OpenMP, -O2, no fast-math)."""
+    """Compile the C oracle with gcc (OpenMP, -O2, no fast-math, no fused multiply-add)."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-Wextra",
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off",
+             "-Wall", "-Wextra",
              "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -51,6 +52,11 @@ def _load():
         lib.lbo_forward.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int,
                                     vp, i64, vp, i64, vp, vp, vp, vp, i64, vp]
         lib.lbo_forward.restype = ctypes.c_int
+        lib.lbo_forward_xor.argtypes = [vp, i64, i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                        vp, i64, vp, i64, vp, vp, vp, vp]
+        lib.lbo_forward_xor.restype = ctypes.c_int
+        lib.lbo_xor_quantise.argtypes = [vp, i64, ctypes.c_int, vp]
+        lib.lbo_xor_quantise.restype = ctypes.c_float
         lib.lbo_threads.restype = ctypes.c_int
         lib.lbo_set_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -146,3 +152,43 @@ def forward(x: np.ndarray, branches: Sequence[Branch], in_f: int, out_f: int, r:
     if rc != 0:
         raise ValueError("lbo_forward rejected its arguments")
     return y
+
+
+def _check_branches(branches, in_f, out_f, r):
+    for b in branches:
+        if b.Vp.shape[0] != r or b.Up.shape[0] != out_f:
+            raise ValueError("packed factor shapes do not match (in, out, r)")
+        if b.h.shape[0] != out_f or b.g.shape[0] != in_f or b.l.shape[0] != r:
+            raise ValueError("scale lengths do not match (in, out, r)")
+
+
+def forward_xor(x: np.ndarray, branches: Sequence[Branch], in_f: int, out_f: int, r: int,
+                bits: int = 16) -> np.ndarray:
+    """The bit-serial (XOR / popcount) variant of the layer, per its definition in
+    lb_oracle.c: each vector quantised to ``bits``-bit odd-integer codes (fp32
+    decisions), exact integer contractions, y in fp64.  x is (M, in) or (in,)."""
+    lib = _load()
+    xx = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    M = xx.shape[0]
+    if xx.shape[1] != in_f:
+        raise ValueError("x has the wrong width")
+    _check_branches(branches, in_f, out_f, r)
+    nb = len(branches)
+    arr = lambda vals: ctypes.cast((ctypes.c_void_p * nb)(*vals), ctypes.c_void_p)
+    y = np.empty((M, out_f), dtype=np.float64)
+    rc = lib.lbo_forward_xor(_ptr(xx), M, in_f, out_f, r, nb, int(bits),
+                             arr([_ptr(b.Vp) for b in branches]), branches[0].Vp.shape[1],
+                             arr([_ptr(b.Up) for b in branches]), branches[0].Up.shape[1],
+                             arr([_ptr(b.h) for b in branches]), arr([_ptr(b.g) for b in branches]),
+                             arr([_ptr(b.l) for b in branches]), _ptr(y))
+    if rc != 0:
+        raise ValueError("lbo_forward_xor rejected its arguments")
+    return y
+
+
+def xor_quantise(v: np.ndarray, bits: int = 16):
+    """(D, codes) of the bit-serial variant's quantiser for the fp32 vector v."""
+    vv = np.ascontiguousarray(v, dtype=np.float32).reshape(-1)
+    codes = np.empty(vv.shape[0], dtype=np.int64)
+    D = _load().lbo_xor_quantise(_ptr(vv), vv.shape[0], int(bits), _ptr(codes))
+    return float(D), codes

@@ -29,6 +29,7 @@
  *   V (in x r) is packed along `in` for every latent column k: Vp[k][in/32].
  *   U (out x r) is packed along r for every output row i:     Up[i][r/32].
  */
+#include <math.h>
 #include <stdint.h>
 #include <stddef.h>
 #include <stdlib.h>
@@ -161,4 +162,107 @@ int lbo_forward(const double *x, int64_t M, int64_t in, int64_t out, int64_t r,
     free(u);
     free(tp);
     return 0;
+}
+
+/*
+ * Bit-serial variant of the forward ("The XOR claim" on the same page: when
+ * both operands are signs, a multiply becomes an XOR plus a popcount).  The
+ * activations are not signs, so this variant first quantises each vector to
+ * B-bit fixed point in a code whose B bit-planes are themselves signs:
+ *
+ *   Q_B(v[0..n)): A = max|v_j| (fp32), D = 2^e with e the smallest integer
+ *   (e >= -100) such that A <= (2^B - 1) * D; q_j = 2*floor(v_j / (2D)) + 1,
+ *   an odd integer in [-(2^B - 1), 2^B - 1], so that |D*q_j - v_j| <= D.
+ *   Every odd q in that range is sum_p 2^p sigma_p with sigma_p in {-1, +1}
+ *   (sigma_p = 2*bit_p((q + 2^B - 1)/2) - 1).
+ *
+ * so that sum_j s_j q_j = sum_p 2^p sum_j s_j sigma_jp, a sum of sign-times-
+ * sign products.  This oracle takes the definition as written: the integer
+ * dot products sum_j s_j q_j directly (the popcount identity is what the GPU
+ * side uses and what the tests check it against).  Decisions that choose an
+ * integer code are taken in fp32, as the kernel takes them:
+ *
+ *   u_j  = fp32(g_j * x_j)                         (exact)
+ *   (D1, q) = Q_B(u);     T_k = sum_j s(V_jk) q_j  (exact integer)
+ *   t'_k = fp32(l_k * fp32(D1 * T_k))
+ *   (D2, q') = Q_B(t');   Z_i = sum_k s(U_ik) q'_k (exact integer)
+ *   y_i += h_i * D2 * Z_i                          (fp64, summed over branches)
+ */
+static float xor_scale(const float *v, int64_t n, int B)
+{
+    float A = 0.0f;
+    for (int64_t j = 0; j < n; ++j) {
+        float a = fabsf(v[j]);
+        if (a > A) A = a;
+    }
+    const float top = (float)((1L << B) - 1);
+    int e = -100;
+    /* the smallest e with A <= top * 2^e (exact products of powers of two) */
+    if (A > top * ldexpf(1.0f, e)) {
+        int ea;
+        frexpf(A, &ea);            /* A < 2^ea */
+        e = ea - B - 1;
+        if (e < -100) e = -100;
+        while (A > top * ldexpf(1.0f, e)) ++e;
+        while (e > -100 && A <= top * ldexpf(1.0f, e - 1)) --e;
+    }
+    return ldexpf(1.0f, e);
+}
+
+static int64_t xor_code(float v, float D)
+{
+    return 2 * (int64_t)floorf(v / (2.0f * D)) + 1;
+}
+
+int lbo_forward_xor(const double *x, int64_t M, int64_t in, int64_t out, int64_t r,
+                    int nb, int B, const uint32_t *const *Vp, int64_t ldv,
+                    const uint32_t *const *Up, int64_t ldu,
+                    const double *const *h, const double *const *g,
+                    const double *const *l, double *y)
+{
+    if (!x || !y || M < 0 || in <= 0 || out <= 0 || r <= 0 || nb < 1) return -1;
+    if (B < 1 || B > 24 || ldv * 32 < in || ldu * 32 < r) return -1;
+    float *u = (float *)malloc(sizeof(float) * (size_t)in);
+    float *tp = (float *)malloc(sizeof(float) * (size_t)r);
+    int64_t *q = (int64_t *)malloc(sizeof(int64_t) * (size_t)in);
+    int64_t *q2 = (int64_t *)malloc(sizeof(int64_t) * (size_t)r);
+    if (!u || !tp || !q || !q2) { free(u); free(tp); free(q); free(q2); return -1; }
+    for (int64_t m = 0; m < M; ++m) {
+        double *ym = y + m * out;
+        for (int64_t i = 0; i < out; ++i) ym[i] = 0.0;
+        for (int b = 0; b < nb; ++b) {
+            for (int64_t j = 0; j < in; ++j) u[j] = (float)g[b][j] * (float)x[m * in + j];
+            const float D1 = xor_scale(u, in, B);
+            for (int64_t j = 0; j < in; ++j) q[j] = xor_code(u[j], D1);
+#pragma omp parallel for schedule(static)
+            for (int64_t k = 0; k < r; ++k) {
+                const uint32_t *vrow = Vp[b] + k * ldv;
+                int64_t T = 0;
+                for (int64_t j = 0; j < in; ++j)
+                    T += (((vrow[j >> 5] >> (uint32_t)(j & 31)) & 1u) ? -q[j] : q[j]);
+                const float DT = D1 * (float)T;
+                tp[k] = (float)l[b][k] * DT;
+            }
+            const float D2 = xor_scale(tp, r, B);
+            for (int64_t k = 0; k < r; ++k) q2[k] = xor_code(tp[k], D2);
+#pragma omp parallel for schedule(static)
+            for (int64_t i = 0; i < out; ++i) {
+                const uint32_t *urow = Up[b] + i * ldu;
+                int64_t Z = 0;
+                for (int64_t k = 0; k < r; ++k)
+                    Z += (((urow[k >> 5] >> (uint32_t)(k & 31)) & 1u) ? -q2[k] : q2[k]);
+                ym[i] += h[b][i] * (double)D2 * (double)Z;
+            }
+        }
+    }
+    free(u); free(tp); free(q); free(q2);
+    return 0;
+}
+
+/* The quantiser alone (for the tests): D and the codes of v[0..n). */
+float lbo_xor_quantise(const float *v, int64_t n, int B, int64_t *codes)
+{
+    const float D = xor_scale(v, n, B);
+    for (int64_t j = 0; j < n; ++j) codes[j] = xor_code(v[j], D);
+    return D;
 }
