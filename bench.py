@@ -419,11 +419,18 @@ def sweep_layer70b_vs_dense(device, flush, hbm_peak):
         for _ in range(3):
             fn()
         ms = _time_events(fn, 20, flush)
+        # the bit-serial (XOR / popcount) variant of the same layer, 16 bit-planes
+        xws = torch.empty(lb.lib().lb_linear_xor_workspace_size(1, in_f, out_f, r, 2, 16),
+                          dtype=torch.uint8, device=device)
+        fx = lambda: lb.linear_forward_xor(x, brs, in_f, out_f, r, bits=16, y=y, workspace=xws)
+        for _ in range(3):
+            fx()
+        xor_ms = _time_events(fx, 20, flush)
         by = linear_bytes(in_f, out_f, r)
         rows.append({"bits_per_weight": bpw, "r": r, "ms": ms, "bytes": by,
                      "gbs": by / ms / 1e6, "hbm_frac": by / ms / 1e6 / hbm_peak,
-                     "speedup_vs_dense_bf16": dense_ms / ms})
-        del brs, x, y, ws
+                     "speedup_vs_dense_bf16": dense_ms / ms, "xor_popcount_ms": xor_ms})
+        del brs, x, y, ws, xws
     return {"dense_bf16_ms": dense_ms, "dense_bf16_gbs": dense_bytes / dense_ms / 1e6,
             "layers": rows,
             "pages": "A100, same layer shape: speed-up grows as bits/weight fall, up to 11.6x"}

@@ -61,7 +61,7 @@ EXPORTS = ("lb_status_string", "lb_version", "lb_pack_signs", "lb_linear_forward
            "lb_stack_prepare", "lb_stack_forward", "lb_stack_forward_host",
            "lb_workspace_status", "lb_stack_output", "lb_linear_forward_noalloc",
            "lb_noalloc_scratch_bytes", "lb_pack_signs_sliced", "lb_packed_words",
-           "lb_stack_plan_host")
+           "lb_stack_plan_host", "lb_linear_forward_xor", "lb_linear_xor_workspace_size")
 
 _lib = None
 
@@ -109,6 +109,11 @@ def lib() -> ctypes.CDLL:
                                                 vp]
         L.lb_linear_forward_noalloc.restype = st
         L.lb_noalloc_scratch_bytes.restype = sz
+        L.lb_linear_forward_xor.argtypes = [vp, st, i64, i64, i64, i64, vp, ctypes.c_int,
+                                            ctypes.c_int, vp, vp, sz, vp]
+        L.lb_linear_forward_xor.restype = st
+        L.lb_linear_xor_workspace_size.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.c_int]
+        L.lb_linear_xor_workspace_size.restype = sz
         _lib = L
     return _lib
 
@@ -265,6 +270,31 @@ def linear_forward_noalloc(x: torch.Tensor, branches: Sequence[Branch], in_f: in
     _check(lib().lb_linear_forward_noalloc(_ptr(x2), dt, x2.shape[0], in_f, out_f, r,
                                            ctypes.addressof(arr), nb, _ptr(y), _stream(stream)),
            "lb_linear_forward_noalloc")
+    return y
+
+
+def linear_forward_xor(x: torch.Tensor, branches: Sequence[Branch], in_f: int, out_f: int,
+                       r: int, bits: int = 16, y: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lb_linear_forward_xor: the bit-serial (XOR / popcount) variant, activations
+    quantised to ``bits``-bit sign-plane codes; y (M x out, fp32)."""
+    x2 = x if x.dim() == 2 else x.reshape(1, -1)
+    M = x2.shape[0]
+    if y is None:
+        y = torch.empty((M, out_f), dtype=torch.float32, device=x.device)
+    nb = len(branches)
+    if workspace is None:
+        n = int(lib().lb_linear_xor_workspace_size(M, in_f, out_f, r, nb, bits))
+        if n == 0:
+            raise LbError(LB_ERR_INVALID_ARG, "lb_linear_xor_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    arr = (lb_branch * nb)(*[b.c_struct() for b in branches])
+    dt = _DTYPES.get(x2.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported x dtype {x2.dtype}")
+    _check(lib().lb_linear_forward_xor(_ptr(x2), dt, M, in_f, out_f, r, ctypes.addressof(arr), nb,
+                                       int(bits), _ptr(y), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "lb_linear_forward_xor")
     return y
 
 

@@ -563,10 +563,13 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     float v[32];
                     __syncwarp();
                     tmem_ld32(tacc + (uint32_t)c0, v);
+                    // rows past M are never stored, so their partial sums are not kept
+                    if (mok) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        __stcg(reinterpret_cast<float4*>(pw + ci * 1024 + (i * 32 + lane) * 4),
-                               make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+                        for (int i = 0; i < 8; ++i)
+                            __stcg(reinterpret_cast<float4*>(pw + ci * 1024 + (i * 32 + lane) * 4),
+                                   make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+                    }
                 }
                 __syncwarp();
                 int ticket = 0;
@@ -584,7 +587,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         float v[16];
                         __syncwarp();
                         tmem_ld16(tacc + (uint32_t)(c_begin + 16 * h), v);
-                        for (int p = 0; p < plan.split; ++p) {
+                        for (int p = 0; p < plan.split && mok; ++p) {
                             if (p == r.part) continue;
                             const float* pc = p0 + (size_t)p * kEpiWarps * kPartFloats + h * 512;
 #pragma unroll
@@ -786,24 +789,71 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
 }
 
 // Pre-pass: per row m, 2^a_m (brings max|x| into [2^14, 2^15)), the fp16 copy
-// of x * 2^a_m, and 2^c_m (keeps |T| <= 65504; see the header comment).
+// of x * 2^a_m, and 2^c_m (keeps |T| <= 65504; see the header comment).  One
+// block per row; every thread takes 8 consecutive elements at a time with
+// 16-byte loads (in is a multiple of 64 and x, g are 16-byte aligned), two
+// steps unrolled so that their loads are in flight together.
+__device__ __forceinline__ void load8_x(const void* x, int x_kind, size_t at, float (&v)[8]) {
+    if (x_kind == VK_X_F32) {
+        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at);
+        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        return;
+    }
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + at);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (x_kind == VK_X_F16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+            v[2 * i] = f.x; v[2 * i + 1] = f.y;
+        } else {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            v[2 * i] = f.x; v[2 * i + 1] = f.y;
+        }
+    }
+}
+__device__ __forceinline__ void load8_h(const __half* p, size_t at, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p + at));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        v[2 * i] = f.x; v[2 * i + 1] = f.y;
+    }
+}
+
 __global__ void __launch_bounds__(256) prefill_prepass_kernel(
     const void* __restrict__ x, int x_kind, int M, int in, int nb,
     const __half* __restrict__ g0, const __half* __restrict__ g1,
     const float* __restrict__ lmax, __half* __restrict__ X16, float* __restrict__ row_sa,
     float* __restrict__ row_sc) {
     const int m = blockIdx.x;
+    const size_t row = (size_t)m * in;
     __shared__ float red[3][8];
     float mx = 0.0f, s0 = 0.0f, s1 = 0.0f;
-    for (int j = threadIdx.x; j < in; j += 256) {
-        float v;
-        if (x_kind == VK_X_F16) v = __half2float(reinterpret_cast<const __half*>(x)[(size_t)m * in + j]);
-        else if (x_kind == VK_X_BF16)
-            v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[(size_t)m * in + j]);
-        else v = reinterpret_cast<const float*>(x)[(size_t)m * in + j];
-        mx = fmaxf(mx, fabsf(v));
-        s0 += fabsf(v * __half2float(g0[j]));
-        if (nb > 1) s1 += fabsf(v * __half2float(g1[j]));
+    constexpr int kStep = 256 * 8;
+    for (int j0 = threadIdx.x * 8; j0 < in; j0 += 2 * kStep) {
+        float xv[2][8], gv[2][8], hv[2][8];
+        const bool two = j0 + kStep < in;
+        load8_x(x, x_kind, row + j0, xv[0]);
+        load8_h(g0, j0, gv[0]);
+        if (nb > 1) load8_h(g1, j0, hv[0]);
+        if (two) {
+            load8_x(x, x_kind, row + j0 + kStep, xv[1]);
+            load8_h(g0, j0 + kStep, gv[1]);
+            if (nb > 1) load8_h(g1, j0 + kStep, hv[1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (u == 1 && !two) break;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                mx = fmaxf(mx, fabsf(xv[u][i]));
+                s0 += fabsf(xv[u][i] * gv[u][i]);
+                if (nb > 1) s1 += fabsf(xv[u][i] * hv[u][i]);
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -836,13 +886,16 @@ __global__ void __launch_bounds__(256) prefill_prepass_kernel(
         row_sa[m] = sa;
         row_sc[m] = sc;
     }
-    for (int j = threadIdx.x; j < in; j += 256) {
-        float v;
-        if (x_kind == VK_X_F16) v = __half2float(reinterpret_cast<const __half*>(x)[(size_t)m * in + j]);
-        else if (x_kind == VK_X_BF16)
-            v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[(size_t)m * in + j]);
-        else v = reinterpret_cast<const float*>(x)[(size_t)m * in + j];
-        X16[(size_t)m * in + j] = __float2half_rn(v * sa);
+    for (int j0 = threadIdx.x * 8; j0 < in; j0 += kStep) {
+        float xv[8];
+        load8_x(x, x_kind, row + j0, xv);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h2 = __floats2half2_rn(xv[2 * i] * sa, xv[2 * i + 1] * sa);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(X16 + row + j0) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -852,7 +905,15 @@ __global__ void __launch_bounds__(256) lmax_kernel(const __half* __restrict__ l0
                                                    float* __restrict__ out) {
     const __half* l = blockIdx.x == 0 ? l0 : l1;
     float mx = 0.0f;
-    for (int k = threadIdx.x; k < r; k += 256) mx = fmaxf(mx, fabsf(__half2float(l[k])));
+    for (int k0 = threadIdx.x; k0 < r; k0 += 4 * 256) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u * 256;
+            v[u] = k < r ? fabsf(__half2float(__ldg(l + k))) : 0.0f;
+        }
+        mx = fmaxf(mx, fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     __shared__ float red[8];

@@ -204,6 +204,35 @@ lb_status lb_linear_forward_noalloc(const void *x, lb_dtype x_dtype, int64_t M, 
                                     int64_t out, int64_t r, const lb_branch *br,
                                     int n_branches, float *y, void *stream);
 
+/*
+ * lb_linear_forward_xor — the bit-serial variant of the layer ("The XOR
+ * claim" on the same page: with both operands signs, a multiply becomes an
+ * XOR plus a popcount).  Each activation vector v (g_b o x, then l_b o t) is
+ * quantised to `bits`-bit fixed point in a code whose bit-planes are signs:
+ *   D = 2^e, the smallest (e >= -100) with max|v| <= (2^bits - 1) D;
+ *   q_j = 2 floor(v_j / 2D) + 1  (odd, |D q_j - v_j| <= D);
+ *   q_j = sum_p 2^p sigma_jp with sigma_jp in {-1, +1},
+ * and every contraction sum_j s_j q_j = sum_p 2^p (n - 2 popc(s XOR plane_p))
+ * is computed exactly in integers on 32-bit words.  The result:
+ *   t'_k = fp32(l_k * fp32(D1 * T_k)),  y_i = sum_b h_bi * D2_b * Z_bi  (fp32).
+ * With bits = 16 the quantisation error is about 1e-4 of max|y|.
+ *   x, br, M, in, out, r, n_branches, y : as lb_linear_forward (any layout,
+ *                     packed pointers 4-byte aligned, scales 2-byte aligned)
+ *   bits      : 1 .. 24 bit-planes per activation
+ *   workspace : device, >= lb_linear_xor_workspace_size(...) bytes, 16-byte
+ *               aligned, clobbered.
+ * Four kernel launches on `stream`.  Errors: LB_ERR_INVALID_ARG,
+ * LB_ERR_ALIGNMENT, LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED, LB_ERR_CUDA.
+ * It is the reference form of the claim, not the fast path: on this GPU the
+ * lookup-table kernels of lb_linear_forward need fewer instructions per sign.
+ */
+lb_status lb_linear_forward_xor(const void *x, lb_dtype x_dtype, int64_t M, int64_t in,
+                                int64_t out, int64_t r, const lb_branch *br, int n_branches,
+                                int bits, float *y, void *workspace, size_t ws_bytes,
+                                void *stream);
+size_t lb_linear_xor_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
+                                    int n_branches, int bits);
+
 /* Size in bytes of the fixed scratch array used by lb_linear_forward_noalloc. */
 size_t lb_noalloc_scratch_bytes(void);
 
