@@ -75,7 +75,8 @@ bool ld_ok(int64_t ld, int64_t k) { return ld == 0 || (ld >= cdiv(k, 32) && ld <
 // Give each phase a cost-balanced split of its units over G CTAs, written to
 // `split` (kMaxGrid+1 ints per phase); phases keep the even split if G does
 // not fit the table.
-void plan_splits(LbPhase* phases, int n_phases, LbJob* jobs, int G, int* split) {
+void plan_splits(LbPhase* phases, int n_phases, LbJob* jobs, int G, int* split,
+                 bool search = false) {
     for (int p = 0; p < n_phases; ++p) {
         phases[p].next_job_begin = p + 1 < n_phases ? phases[p + 1].job_begin : 0;
         phases[p].next_n_jobs = p + 1 < n_phases ? phases[p + 1].n_jobs : 0;
@@ -83,7 +84,7 @@ void plan_splits(LbPhase* phases, int n_phases, LbJob* jobs, int G, int* split) 
         phases[p].split_g = -1;
         phases[p].starts_g = -1;   // no start table unless plan_starts makes one
         plan_row_groups(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units,
-                        std::max(G, 1));
+                        std::max(G, 1), search);
         if (G < 1 || G > kMaxGrid) continue;
         balanced_split(jobs + phases[p].job_begin, phases[p].n_jobs, phases[p].n_units, G,
                        split + phases[p].split_off);
@@ -595,7 +596,7 @@ bool make_stack_plan(const lb_stack_desc* d, const StackLayout& L, char* ws, int
     build_stack_plan(d, L, ws, P.phases, P.jobs);
     if ((int)P.phases.size() != L.n_phases || (int)P.jobs.size() != L.n_jobs) return false;
     P.split.assign((size_t)(kMaxGrid + 1) * L.n_phases, 0);
-    plan_splits(P.phases.data(), L.n_phases, P.jobs.data(), G, P.split.data());
+    plan_splits(P.phases.data(), L.n_phases, P.jobs.data(), G, P.split.data(), true);
     P.starts.assign((size_t)kMaxGrid * L.n_phases, LbStart{});
     plan_starts(P.phases.data(), L.n_phases, P.jobs.data(), P.split.data(), G, P.starts.data());
     return true;

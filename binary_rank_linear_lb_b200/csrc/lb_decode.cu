@@ -47,6 +47,8 @@
 // it will stage.  It keeps bulk loads out of the memory queues until the wait
 // and the staging loads after it, which are on the critical path, have been
 // issued.
+#include <vector>
+
 #include "lb_internal.cuh"
 
 namespace lb {
@@ -779,8 +781,9 @@ cudaError_t launch_coop(const void* fn, void** args, cudaStream_t s) {
 int decode_grid() { return device_sm_count() * kCtasPerSm; }
 
 // Contiguous unit ranges for G CTAs with the smallest largest cost.  A CTA
-// takes its tiles in batches of up to kTables; a batch costs kTileCost per
-// tile (vector stage + table build, in rowblock times) plus one per rowblock.
+// takes its tiles in batches of up to kTables; a batch costs kBatchCost
+// (staging its vectors) plus kTileCost per tile (a table build) plus its
+// rowblocks (see rb_cost), all in 1/16 of a round of 16 rowblocks.
 // Units run job by job, slice-major inside a job, so a phase is a list of
 // tiles of n_rowblocks units each; a greedy fill is optimal for a given bound,
 // which a bisection minimises.
@@ -813,16 +816,17 @@ struct Fill {
     long long rb;       // rowblocks in its open batch
 };
 // The CTA's state and cost once `take` rowblocks of a new tile join it.
+long long open_cost(const Fill& g) { return kBatchCost + g.tiles * kTileCost; }
 long long join(const Fill& f, long long take, Fill& g) {
     g = f;
     if (g.tiles == kTables) {
-        g.closed += g.tiles * kTileCost + rb_cost(g.rb);
+        g.closed += open_cost(g) + rb_cost(g.rb);
         g.tiles = 0;
         g.rb = 0;
     }
     g.tiles += 1;
     g.rb += take;
-    return g.closed + g.tiles * kTileCost + rb_cost(g.rb);
+    return g.closed + open_cost(g) + rb_cost(g.rb);
 }
 // CTAs a greedy fill under cost bound T needs; boundaries go to `out` if set.
 int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
@@ -837,7 +841,7 @@ int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
                 f = Fill{0, 0, 0};
             }
             join(f, 0, g);
-            const long long room = rb_room(T - g.closed - g.tiles * kTileCost) - g.rb;
+            const long long room = rb_room(T - g.closed - open_cost(g)) - g.rb;
             const int take = (int)std::max<long long>(1, std::min<long long>(n, room));
             join(f, take, f);
             n -= take;
@@ -846,22 +850,47 @@ int greedy_fill(const LbJob* jobs, int n_jobs, long long T, int* out) {
     });
     return used;
 }
-}  // namespace
 
-// A job gets about as many row groups as the CTAs its share of the phase's
-// units would occupy, divided by its slices, so that a CTA's range is
-// usually one tile and the n_slices CTAs of a group read the same rows.
-void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G) {
+// A job gets about alpha times as many row groups as the CTAs its share of
+// the phase's units would occupy, divided by its slices, so that a CTA's range
+// is usually one tile and the n_slices CTAs of a group read the same rows.
+void row_groups(LbJob* jobs, int n_jobs, int n_units, int G, double alpha) {
     for (int j = 0; j < n_jobs; ++j) {
         LbJob& J = jobs[j];
         const double ctas = (double)G * (double)(J.n_slices * J.n_rowblocks) / (double)n_units;
-        const int groups = std::max(1, (int)(ctas / J.n_slices + 0.5));
+        const int groups = std::max(1, (int)(alpha * ctas / J.n_slices + 0.5));
         J.rg = (J.n_rowblocks + groups - 1) / groups;
     }
 }
+}  // namespace
 
-void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out) {
-    long long lo = kTileCost + kDecodeWarps, hi = lo;
+long long balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
+
+// Row groups of a phase: with `search`, the scaling of the CTA-proportional
+// count whose cost-balanced split has the smallest largest cost (rounding the
+// count to the nearest integer can leave most CTAs with a range across two
+// tiles, and so two table builds, where one tile per CTA fits in the same
+// time); stack plans, made once, search; single-linear calls plan on every
+// call and take the unscaled count.
+void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G, bool search) {
+    if (!search) {
+        row_groups(jobs, n_jobs, n_units, G, 1.0);
+        return;
+    }
+    static const double kAlphas[] = {1.0, 0.9, 0.8, 0.7, 0.6, 0.5, 1.15, 1.3};
+    std::vector<int> split(G + 1);
+    double best_alpha = 1.0;
+    long long best = -1;
+    for (double a : kAlphas) {
+        row_groups(jobs, n_jobs, n_units, G, a);
+        const long long c = balanced_split(jobs, n_jobs, n_units, G, split.data());
+        if (best < 0 || c < best) { best = c; best_alpha = a; }
+    }
+    row_groups(jobs, n_jobs, n_units, G, best_alpha);
+}
+
+long long balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out) {
+    long long lo = kBatchCost + kTileCost + kDecodeWarps, hi = lo;
     {
         Fill f = {0, 0, 0};
         for_each_tile(jobs, n_jobs, [&](int n) { hi = join(f, n, f); });
@@ -875,6 +904,7 @@ void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out)
     const int used = greedy_fill(jobs, n_jobs, lo, out);
     out[0] = 0;
     for (int c = used; c <= G; ++c) out[c] = n_units;
+    return lo;
 }
 
 void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* split, int G,

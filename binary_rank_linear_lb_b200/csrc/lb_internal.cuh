@@ -141,7 +141,9 @@ static_assert(kMiscBytes + 1024 <= (int)kTableAddr0, "decode plan cache overlaps
 
 // Plan of a single linear call, passed by value as a kernel parameter.
 constexpr int kMaxGrid = 256;                // CTAs a split table has room for
-constexpr int kTileCost = 12;                // vector stage + table build, in 1/16 warp iterations
+// Costs of the host's work split, in 1/16 of a round of 16 rowblocks (one per rowblock).
+constexpr int kBatchCost = 0;                // staging a batch's vectors
+constexpr int kTileCost = 12;                // building a tile's table (and, with kBatchCost 0, its staging)
 
 struct LinearPlan {
     LbJob jobs[2 * kMaxLinearJobs];
@@ -252,17 +254,21 @@ cudaError_t launch_stack_plan(const LbPhase* phases, const LbJob* jobs, const in
                               const LbStart* starts, int n_phases, WsHeader* hdr, const void* x,
                               float* y, cudaStream_t s);
 int decode_grid();                   // CTAs of a decode launch on the current device
-// Row-group sizes of a phase's jobs for a grid of G CTAs.
-void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G);
-// Cost-balanced contiguous unit ranges for the G CTAs of a phase (out: G+1 boundaries).
-void balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
+// Row-group sizes of a phase's jobs for a grid of G CTAs (search: try scalings).
+void plan_row_groups(LbJob* jobs, int n_jobs, int n_units, int G, bool search);
+// Cost-balanced contiguous unit ranges for the G CTAs of a phase (out: G+1
+// boundaries); returns the largest CTA cost of the split.
+long long balanced_split(const LbJob* jobs, int n_jobs, int n_units, int G, int* out);
 // The first batch of each CTA of each phase from the split table (G <= kMaxGrid);
 // out holds n_phases * kMaxGrid records, phase q's at q * kMaxGrid.  Sets starts_g.
 void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* split, int G,
                  LbStart* out);
 
 // Tensor-core prefill path (lb_prefill.cu).
-constexpr int kPrefillMinM = 16;             // lb_linear_forward uses it from this many rows
+// lb_linear_forward uses the tensor cores from this many rows: measured on the
+// 7B gate shape (4096 -> 11008) at 1.0 and 0.1 bits/weight, the lookup-table
+// kernels are faster up to 16 rows (two launches of 8), the tensor cores from 17.
+constexpr int kPrefillMinM = 17;
 cudaError_t prefill_configure();
 // with_split: room for the stage-1 K split's partial sums (tens of MB when the
 // split is possible); without it the launch never splits stage 1.

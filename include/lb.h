@@ -184,7 +184,7 @@ size_t lb_linear_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
  *   - where lb_linear_forward takes the tensor-core path, this call takes it
  *     too if 256 + pad(2*M*in) + pad(4*M*r) + pad(8*M) + 256 + pad(4*ceil(M/128))
  *     <= S (pad = round up to 256 bytes), running stage 1 without its K split
- *     (e.g. M = 16, in = 4096, r = 1472 fits; M = 64, in = 4096 does not);
+ *     (e.g. M = 17, in = 4096, r = 1472 fits; M = 64, in = 4096 does not);
  *   - otherwise it takes the lookup-table path, which needs
  *     256 + pad(4 * min(M, 8) * n_branches * r) <= S (two branches: r up to
  *     32736 for M = 1, up to 4092 for M >= 8);
