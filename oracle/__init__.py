@@ -9,6 +9,9 @@ The arithmetic lives in ``lb_oracle.c`` (plain C, fp64) and in ``stack.py``
 library and converts arrays.  Parity of every function here is pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``.
 
+``dual_svid.py`` holds the Dual-SVID initialisation (numpy fp64, library SVD),
+pinned by ``tests/test_oracle_svid_pins.py``.
+
 Sources (web pages on LittleBit; cited by page title and section):
   * "Samsung LittleBit: A 13B LLM Under 1 GB, and What the Paper Really Shows",
     section "How it works": 1 (binary factors U, V), 2 (FP16 scales along rows,
