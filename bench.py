@@ -472,6 +472,35 @@ def sweep_small_m(device, flush):
     return out
 
 
+def sweep_dual_svid(device):
+    """Dual-SVID initialisation (lb_dual_svid) of the 7B gate shape (11008 x 4096) from a
+    seeded N(0, 0.02^2) dense weight, at 1.0 and 0.1 bits/weight: seconds, and the
+    initialised layer's output error against the dense layer on 64 N(0, 1) rows,
+    ||y - W x|| / ||W x||."""
+    import torch
+    import binary_rank_linear_lb_b200 as lb
+    from binary_rank_linear_lb_b200.configs import rank_for
+    out_f, in_f = 11008, 4096
+    g = torch.Generator(device=device)
+    g.manual_seed(2024)
+    W = 0.02 * torch.randn((out_f, in_f), generator=g, device=device)
+    x = torch.randn((64, in_f), generator=g, device=device)
+    y_ref = x @ W.T
+    rows = []
+    for bpw in (1.0, 0.1):
+        r = rank_for(bpw, in_f, out_f)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        brs = lb.dual_svid(W, r, 2)
+        torch.cuda.synchronize()
+        dt = time.perf_counter() - t0
+        y = lb.linear_forward(x, brs, in_f, out_f, r)
+        err = (torch.linalg.norm(y - y_ref) / torch.linalg.norm(y_ref)).item()
+        rows.append({"bits_per_weight": bpw, "r": r, "seconds": dt, "layer_output_rel_err": err})
+        del brs
+    return {"shape": [out_f, in_f], "weight": "N(0, 0.02^2), seed 2024", "runs": rows}
+
+
 def sweep_stacks(device, skip: str, hbm_peak):
     """tokens/s of the other stack workloads (fewer steps; same timing rules)."""
     import torch
@@ -667,6 +696,7 @@ def main():
             "prefill_gate7b": sweep_prefill(device, flush, tflops_peak, fp8["fp8_tflops"]),
             "small_m_gate7b": sweep_small_m(device, flush),
             "layer70b_vs_dense": sweep_layer70b_vs_dense(device, flush, hbm_peak),
+            "dual_svid_gate7b": sweep_dual_svid(device),
             "stacks": sweep_stacks(device, args.workload, hbm_peak),
         }
     if rank == 0:

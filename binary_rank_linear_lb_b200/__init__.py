@@ -61,7 +61,8 @@ EXPORTS = ("lb_status_string", "lb_version", "lb_pack_signs", "lb_linear_forward
            "lb_stack_prepare", "lb_stack_forward", "lb_stack_forward_host",
            "lb_workspace_status", "lb_stack_output", "lb_linear_forward_noalloc",
            "lb_noalloc_scratch_bytes", "lb_pack_signs_sliced", "lb_packed_words",
-           "lb_stack_plan_host", "lb_linear_forward_xor", "lb_linear_xor_workspace_size")
+           "lb_stack_plan_host", "lb_linear_forward_xor", "lb_linear_xor_workspace_size",
+           "lb_dual_svid", "lb_dual_svid_workspace_size")
 
 _lib = None
 
@@ -114,6 +115,11 @@ def lib() -> ctypes.CDLL:
         L.lb_linear_forward_xor.restype = st
         L.lb_linear_xor_workspace_size.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.c_int]
         L.lb_linear_xor_workspace_size.restype = sz
+        L.lb_dual_svid.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp,
+                                   vp, vp, sz, vp]
+        L.lb_dual_svid.restype = st
+        L.lb_dual_svid_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int]
+        L.lb_dual_svid_workspace_size.restype = sz
         _lib = L
     return _lib
 
@@ -296,6 +302,38 @@ def linear_forward_xor(x: torch.Tensor, branches: Sequence[Branch], in_f: int, o
                                        int(bits), _ptr(y), _ptr(workspace), workspace.numel(),
                                        _stream(stream)), "lb_linear_forward_xor")
     return y
+
+
+def dual_svid(W: torch.Tensor, r: int, n_branches: int = 2, layout: int = LB_LAYOUT_SLICES,
+              stream=None) -> List[Branch]:
+    """lb_dual_svid: the branches of a factorised layer initialised from the dense
+    fp32 weight W (out x in) by Dual-SVID, packed in ``layout``."""
+    out_f, in_f = W.shape
+    W = W.contiguous()
+    dev = W.device
+    brs = []
+    for _ in range(n_branches):
+        if layout == LB_LAYOUT_SLICES:
+            Vp = torch.empty(packed_words(r, in_f, layout), dtype=torch.int32, device=dev)
+            Up = torch.empty(packed_words(out_f, r, layout), dtype=torch.int32, device=dev)
+        else:
+            Vp = torch.empty((r, (in_f + 31) // 32), dtype=torch.int32, device=dev)
+            Up = torch.empty((out_f, (r + 31) // 32), dtype=torch.int32, device=dev)
+        brs.append(Branch(Vp, Up, torch.empty(out_f, dtype=torch.float16, device=dev),
+                          torch.empty(in_f, dtype=torch.float16, device=dev),
+                          torch.empty(r, dtype=torch.float16, device=dev), layout))
+    n = int(lib().lb_dual_svid_workspace_size(out_f, in_f, r, n_branches))
+    if n == 0:
+        raise LbError(LB_ERR_INVALID_ARG, "lb_dual_svid_workspace_size")
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    off = (-ws.data_ptr()) % 256
+    arr = lambda ts: (ctypes.c_void_p * n_branches)(*[t.data_ptr() for t in ts])
+    _check(lib().lb_dual_svid(_ptr(W), out_f, in_f, r, n_branches, int(layout),
+                              arr([b.Vp for b in brs]), arr([b.Up for b in brs]),
+                              arr([b.h for b in brs]), arr([b.g for b in brs]),
+                              arr([b.l for b in brs]), ws.data_ptr() + off, n, _stream(stream)),
+           "lb_dual_svid")
+    return brs
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:

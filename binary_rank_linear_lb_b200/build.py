@@ -60,7 +60,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         subprocess.check_call(cmd)
         objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"])
+    subprocess.check_call([nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda", "-lcublas",
+                           "-lcusolver"])
     os.replace(tmp, LIB)
     return LIB
 

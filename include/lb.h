@@ -233,6 +233,37 @@ lb_status lb_linear_forward_xor(const void *x, lb_dtype x_dtype, int64_t M, int6
 size_t lb_linear_xor_workspace_size(int64_t M, int64_t in, int64_t out, int64_t r,
                                     int n_branches, int bits);
 
+/*
+ * lb_dual_svid — initialise the branches of a factorised layer from a dense
+ * weight ("How it works", item 3: Dual-SVID starts from a truncated SVD of the
+ * real weights, maps signs and magnitudes onto the binary factors and the
+ * scales, and fits a residual branch to what the first one missed).  Per
+ * branch, on the residual R (W for the first):
+ *   R ~ U S V^T (rank r; cuSOLVER's randomized truncated SVD),
+ *   U' = U S^(1/2), V' = V S^(1/2);  Up, Vp = packed signs of U', V';
+ *   |U'| ~ h l_u^T, |V'| ~ g l_v^T (rank-1 fits), h and g scaled to mean 1,
+ *   l = l_u o l_v, all rounded to fp16;
+ *   R <- R - diag(h) sign(U') diag(l) sign(V')^T diag(g) (from the stored values).
+ *   W        : device, out x in fp32 row-major, 16-byte aligned, not modified
+ *   r        : 1 .. min(out, in);  n_branches: 1 or 2;  layout: lb_layout of the outputs
+ *   Vp[b], Up[b] : device, lb_packed_words(r, in, layout, 0) and
+ *              lb_packed_words(out, r, layout, 0) words, 16-byte aligned, written
+ *   h[b], g[b], l[b] : device fp16 [out], [in], [r], written
+ *   workspace : device, >= lb_dual_svid_workspace_size(...) bytes, 256-byte aligned
+ * Synchronous (returns when the branches are written).  It is an offline step:
+ * it creates its own cuSOLVER and cuBLAS handles for the call (their internal
+ * state is allocated by those libraries).  The SVD is defined up to the signs of
+ * its singular-vector pairs, which flip a column of sign(U') and of sign(V')
+ * together and leave the branch unchanged.  Errors: LB_ERR_INVALID_ARG,
+ * LB_ERR_ALIGNMENT, LB_ERR_WORKSPACE, LB_ERR_UNSUPPORTED, LB_ERR_CUDA (also when
+ * the SVD reports a failure).
+ */
+lb_status lb_dual_svid(const float *W, int64_t out, int64_t in, int64_t r, int n_branches,
+                       int layout, uint32_t *const *Vp, uint32_t *const *Up, uint16_t *const *h,
+                       uint16_t *const *g, uint16_t *const *l, void *workspace, size_t ws_bytes,
+                       void *stream);
+size_t lb_dual_svid_workspace_size(int64_t out, int64_t in, int64_t r, int n_branches);
+
 /* Size in bytes of the fixed scratch array used by lb_linear_forward_noalloc. */
 size_t lb_noalloc_scratch_bytes(void);
 
