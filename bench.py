@@ -58,8 +58,8 @@ L2_BYTES = 126 * 1024 * 1024
 # proportion.  workload: (sources hash, bytes per captured launch, layers
 # captured, or 0 for a single linear).
 MEASURED_TRAFFIC = {
-    "stack70b-1.0": ("0e3097b271ec3bde", 214949888 + 3339008, 2),
-    "prefill-gate7b-1.0-M4096": ("2b8315c018d03de4", 53410304 + 144020992, 0),
+    "stack70b-1.0": ("fa65e09bcb813709", 214949888 + 3215872, 2),
+    "prefill-gate7b-0.1-M4096": ("9b8eea8d6cdeb78b", 35183872 + 140968704, 0),
 }
 KERNEL_SOURCES = {
     "stack_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),

@@ -484,11 +484,11 @@ lb_status linear_forward_route(const void* x, lb_dtype x_dtype, int64_t M, int64
     const size_t xsz = x_dtype == LB_F32 ? 4 : 2;
     WsHeader* hdr = static_cast<WsHeader*>(workspace);
     float* t = reinterpret_cast<float*>(static_cast<char*>(workspace) + sizeof(WsHeader));
-    // The header (barrier counter, error) is cleared once per call, so a
-    // device-side time-out in one chunk of rows stays visible after the later
-    // chunks (which then return at once); the kernel leaves the barrier counter
-    // at zero when it finishes.  Each chunk clears its t accumulators.
-    if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return LB_ERR_CUDA;
+    // The header (barrier counter, error) is cleared once per call, together
+    // with the first chunk's t accumulators (they follow it), so a device-side
+    // time-out in one chunk of rows stays visible after the later chunks (which
+    // then return at once); the kernel leaves the barrier counter at zero when
+    // it finishes.  Later chunks clear only their t accumulators.
     for (int64_t m0 = 0; m0 < M; m0 += kMaxDecodeM) {
         const int mc = (int)std::min<int64_t>(kMaxDecodeM, M - m0);
         LinearPlan plan;
@@ -528,7 +528,9 @@ lb_status linear_forward_route(const void* x, lb_dtype x_dtype, int64_t M, int64
         plan.phases[1] = p1;
         std::copy(jobs.begin(), jobs.end(), plan.jobs);
         plan_splits(plan.phases, 2, plan.jobs, decode_grid(), plan.split);
-        if (cudaMemsetAsync(t, 0, sizeof(float) * (size_t)mc * n_branches * r, s) != cudaSuccess)
+        const size_t t_bytes = sizeof(float) * (size_t)mc * n_branches * r;
+        if ((m0 == 0 ? cudaMemsetAsync(hdr, 0, sizeof(WsHeader) + t_bytes, s)
+                     : cudaMemsetAsync(t, 0, t_bytes, s)) != cudaSuccess)
             return LB_ERR_CUDA;
         if (launch_linear_plan(plan, hdr, 2, s) != cudaSuccess) return LB_ERR_CUDA;
     }

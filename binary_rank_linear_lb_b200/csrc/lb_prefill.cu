@@ -789,18 +789,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
 }
 
 // Pre-pass: per row m, 2^a_m (brings max|x| into [2^14, 2^15)), the fp16 copy
-// of x * 2^a_m, and 2^c_m (keeps |T| <= 65504; see the header comment).  One
-// block per row; every thread takes 8 consecutive elements at a time with
-// 16-byte loads (in is a multiple of 64 and x, g are 16-byte aligned), two
-// steps unrolled so that their loads are in flight together.
-__device__ __forceinline__ void load8_x(const void* x, int x_kind, size_t at, float (&v)[8]) {
-    if (x_kind == VK_X_F32) {
-        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at);
-        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-        return;
-    }
-    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + at);
+// of x * 2^a_m, and 2^c_m (keeps |T| <= 65504; see the header comment).  Every
+// thread takes 8 consecutive elements at a time with 16-byte loads (in is a
+// multiple of 64 and x, g are 16-byte aligned).
+__device__ __forceinline__ void cvt8_x(uint4 u, int x_kind, float (&v)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -813,6 +805,20 @@ __device__ __forceinline__ void load8_x(const void* x, int x_kind, size_t at, fl
         }
     }
 }
+// The 16 bytes of a 16-bit x at element `at` (raw), unused for fp32 x.
+__device__ __forceinline__ uint4 raw8_x(const void* x, int x_kind, size_t at) {
+    if (x_kind == VK_X_F32) return make_uint4(0u, 0u, 0u, 0u);
+    return *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + at);
+}
+__device__ __forceinline__ void load8_x(const void* x, int x_kind, size_t at, float (&v)[8]) {
+    if (x_kind == VK_X_F32) {
+        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at);
+        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + at + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        return;
+    }
+    cvt8_x(raw8_x(x, x_kind, at), x_kind, v);
+}
 __device__ __forceinline__ void load8_h(const __half* p, size_t at, float (&v)[8]) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(p + at));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -823,106 +829,119 @@ __device__ __forceinline__ void load8_h(const __half* p, size_t at, float (&v)[8
     }
 }
 
-__global__ void __launch_bounds__(256) prefill_prepass_kernel(
+constexpr int kPrepassThreads = 512;
+constexpr int kPrepassRows = 4;                               // rows of x per block
+constexpr int kRowThreads = kPrepassThreads / kPrepassRows;   // threads per row
+constexpr int kRowStep = 8 * kRowThreads;                     // elements of a row per step
+constexpr int kCachedSteps = 4;                               // steps kept in registers
+
+// One block takes kPrepassRows rows (kRowThreads threads each), so that an SM
+// has several rows' loads in flight; a thread's first kCachedSteps steps of a
+// 16-bit x stay in registers for the second pass (rows up to 4096 elements are
+// read once).  The block also takes max_k |l_b[k]| of each branch itself.
+__global__ void __launch_bounds__(kPrepassThreads, 2) prefill_prepass_kernel(
     const void* __restrict__ x, int x_kind, int M, int in, int nb,
     const __half* __restrict__ g0, const __half* __restrict__ g1,
-    const float* __restrict__ lmax, __half* __restrict__ X16, float* __restrict__ row_sa,
-    float* __restrict__ row_sc) {
-    const int m = blockIdx.x;
-    const size_t row = (size_t)m * in;
-    __shared__ float red[3][8];
-    float mx = 0.0f, s0 = 0.0f, s1 = 0.0f;
-    constexpr int kStep = 256 * 8;
-    for (int j0 = threadIdx.x * 8; j0 < in; j0 += 2 * kStep) {
-        float xv[2][8], gv[2][8], hv[2][8];
-        const bool two = j0 + kStep < in;
-        load8_x(x, x_kind, row + j0, xv[0]);
-        load8_h(g0, j0, gv[0]);
-        if (nb > 1) load8_h(g1, j0, hv[0]);
-        if (two) {
-            load8_x(x, x_kind, row + j0 + kStep, xv[1]);
-            load8_h(g0, j0 + kStep, gv[1]);
-            if (nb > 1) load8_h(g1, j0 + kStep, hv[1]);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (u == 1 && !two) break;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                mx = fmaxf(mx, fabsf(xv[u][i]));
-                s0 += fabsf(xv[u][i] * gv[u][i]);
-                if (nb > 1) s1 += fabsf(xv[u][i] * hv[u][i]);
-            }
-        }
+    const __half* __restrict__ l0, const __half* __restrict__ l1, int r,
+    __half* __restrict__ X16, float* __restrict__ row_sa, float* __restrict__ row_sc) {
+    constexpr int kWarps = kPrepassThreads / 32, kGroupWarps = kRowThreads / 32;
+    __shared__ float red[kWarps][3];
+    __shared__ float lred[kWarps][2];
+    const int grp = threadIdx.x / kRowThreads, t = threadIdx.x % kRowThreads;
+    const int m = blockIdx.x * kPrepassRows + grp;
+    const bool row_ok = m < M;
+    const size_t row = (size_t)(row_ok ? m : 0) * in;
+    // max |l| of each branch, over the block (its loads go out with x's)
+    float lm0 = 0.0f, lm1 = 0.0f;
+    for (int k = threadIdx.x; k < r; k += kPrepassThreads) {
+        lm0 = fmaxf(lm0, fabsf(__half2float(__ldg(l0 + k))));
+        if (nb > 1) lm1 = fmaxf(lm1, fabsf(__half2float(__ldg(l1 + k))));
     }
+    float mx = 0.0f, s0 = 0.0f, s1 = 0.0f;
+    uint4 xc[kCachedSteps];
+    auto step = [&](int j0, uint4& raw) {
+        float xv[8], gv[8], hv[8];
+        raw = raw8_x(x, x_kind, row + j0);
+        if (x_kind == VK_X_F32) load8_x(x, x_kind, row + j0, xv);
+        else cvt8_x(raw, x_kind, xv);
+        load8_h(g0, j0, gv);
+        if (nb > 1) load8_h(g1, j0, hv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            mx = fmaxf(mx, fabsf(xv[i]));
+            s0 += fabsf(xv[i] * gv[i]);
+            if (nb > 1) s1 += fabsf(xv[i] * hv[i]);
+        }
+    };
+#pragma unroll
+    for (int c = 0; c < kCachedSteps; ++c) {
+        const int j0 = c * kRowStep + 8 * t;
+        if (row_ok && j0 < in) step(j0, xc[c]);
+    }
+    for (int j0 = kCachedSteps * kRowStep + 8 * t; row_ok && j0 < in; j0 += kRowStep) {
+        uint4 raw;
+        step(j0, raw);
+    }
+    const int w = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         s0 += __shfl_xor_sync(0xffffffffu, s0, o);
         s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        lm0 = fmaxf(lm0, __shfl_xor_sync(0xffffffffu, lm0, o));
+        lm1 = fmaxf(lm1, __shfl_xor_sync(0xffffffffu, lm1, o));
     }
     if ((threadIdx.x & 31) == 0) {
-        red[0][threadIdx.x >> 5] = mx;
-        red[1][threadIdx.x >> 5] = s0;
-        red[2][threadIdx.x >> 5] = s1;
+        red[w][0] = mx; red[w][1] = s0; red[w][2] = s1;
+        lred[w][0] = lm0; lred[w][1] = lm1;
     }
     __syncthreads();
-    float M0 = 0.0f, L0 = 0.0f, L1 = 0.0f;
-    for (int w = 0; w < 8; ++w) {
-        M0 = fmaxf(M0, red[0][w]);
-        L0 += red[1][w];
-        L1 += red[2][w];
+    float M0 = 0.0f, L0 = 0.0f, L1 = 0.0f, lmax0 = 0.0f, lmax1 = 0.0f;
+    for (int v = 0; v < kWarps; ++v) {
+        lmax0 = fmaxf(lmax0, lred[v][0]);
+        lmax1 = fmaxf(lmax1, lred[v][1]);
     }
+    for (int v = grp * kGroupWarps; v < (grp + 1) * kGroupWarps; ++v) {
+        M0 = fmaxf(M0, red[v][0]);
+        L0 += red[v][1];
+        L1 += red[v][2];
+    }
+    if (!row_ok) return;
     // 2^a: the largest power of two with max|x| * 2^a < 2^15
     float sa = 1.0f;
     if (M0 > 0.0f && isfinite(M0)) sa = exp2f(fminf(fmaxf(14.0f - floorf(log2f(M0)), -126.0f), 126.0f));
     // 2^c: the largest power of two with bound * 2^c <= 2^15 (< 65504); the
     // bound is padded by 1/64 for fp32 rounding in the sums.
-    const float bound = fmaxf(L0 * lmax[0], nb > 1 ? L1 * lmax[1] : 0.0f) * (1.0f + 1.0f / 64);
+    const float bound = fmaxf(L0 * lmax0, nb > 1 ? L1 * lmax1 : 0.0f) * (1.0f + 1.0f / 64);
     float sc = 1.0f;
     if (bound > 0.0f && isfinite(bound))
         sc = exp2f(fminf(fmaxf(15.0f - ceilf(log2f(bound)), -126.0f), 126.0f));
-    if (threadIdx.x == 0) {
+    if (t == 0) {
         row_sa[m] = sa;
         row_sc[m] = sc;
     }
-    for (int j0 = threadIdx.x * 8; j0 < in; j0 += kStep) {
-        float xv[8];
-        load8_x(x, x_kind, row + j0, xv);
-        uint32_t w[4];
+    auto put = [&](int j0, const float (&xv)[8]) {
+        uint32_t q[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const __half2 h2 = __floats2half2_rn(xv[2 * i] * sa, xv[2 * i + 1] * sa);
-            w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            q[i] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        *reinterpret_cast<uint4*>(X16 + row + j0) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-// max_k |l_b[k]| for each branch (one block per branch).
-__global__ void __launch_bounds__(256) lmax_kernel(const __half* __restrict__ l0,
-                                                   const __half* __restrict__ l1, int r,
-                                                   float* __restrict__ out) {
-    const __half* l = blockIdx.x == 0 ? l0 : l1;
-    float mx = 0.0f;
-    for (int k0 = threadIdx.x; k0 < r; k0 += 4 * 256) {
-        float v[4];
+        *reinterpret_cast<uint4*>(X16 + row + j0) = make_uint4(q[0], q[1], q[2], q[3]);
+    };
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u * 256;
-            v[u] = k < r ? fabsf(__half2float(__ldg(l + k))) : 0.0f;
-        }
-        mx = fmaxf(mx, fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+    for (int c = 0; c < kCachedSteps; ++c) {
+        const int j0 = c * kRowStep + 8 * t;
+        if (j0 >= in) continue;
+        float xv[8];
+        if (x_kind == VK_X_F32) load8_x(x, x_kind, row + j0, xv);
+        else cvt8_x(xc[c], x_kind, xv);
+        put(j0, xv);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    __shared__ float red[8];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float m = 0.0f;
-        for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
-        out[blockIdx.x] = m;
+    for (int j0 = kCachedSteps * kRowStep + 8 * t; j0 < in; j0 += kRowStep) {
+        float xv[8];
+        load8_x(x, x_kind, row + j0, xv);
+        put(j0, xv);
     }
 }
 
@@ -1102,8 +1121,7 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     float* sa = reinterpret_cast<float*>(ws + off);
     float* sc = sa + M;
     off += up(8 * (size_t)M);
-    float* lmax = reinterpret_cast<float*>(ws + off);
-    off += 256;
+    off += 256;                                     // (reserved)
     int* done = reinterpret_cast<int*>(ws + off);   // per M block, stage-1 tiles finished
     off += up(4 * (size_t)((M + kTileM - 1) / kTileM));
     float* partial = nullptr;                       // stage-1 K split: partial sums, tickets
@@ -1116,11 +1134,11 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
     if (e != cudaSuccess) return e;
     const __half* l1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].l);
-    lmax_kernel<<<nb, 256, 0, s>>>(reinterpret_cast<const __half*>(br[0].l), l1, (int)r, lmax);
     const __half* g1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].g);
-    prefill_prepass_kernel<<<(unsigned)M, 256, 0, s>>>(
-        x, x_kind, (int)M, (int)in, nb, reinterpret_cast<const __half*>(br[0].g), g1, lmax, X16,
-        sa, sc);
+    prefill_prepass_kernel<<<(unsigned)((M + kPrepassRows - 1) / kPrepassRows), kPrepassThreads, 0,
+                             s>>>(x, x_kind, (int)M, (int)in, nb,
+                                  reinterpret_cast<const __half*>(br[0].g), g1,
+                                  reinterpret_cast<const __half*>(br[0].l), l1, (int)r, X16, sa, sc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     PrefillPlan plan = {};
