@@ -28,6 +28,7 @@
 // LB_ERR_TIMEOUT, lets every role finish, frees its TMEM and returns.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstdlib>
 
 #include "lb_internal.cuh"
@@ -269,8 +270,11 @@ __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb
 
 // Expand row n of one 256 x 64 B tile (K-major, 128-byte swizzle) from its 64
 // packed sign bits.  Element k is the scale with its sign bit flipped when the
-// bit is set: stage 1 scales per k (g slice staged in shared memory), stage 2
-// per row (hh = h[row] in both halves).  Per 16-byte piece (8 elements): one
+// bit is set: stage 1 scales per k (the K block's 64 values of g: read from
+// global memory, every thread the same 128 bytes, with one M sub-tile per
+// tile, so the expansion need not wait for the A tile; copied in with the A
+// tile and read from shared memory with two, where the expansion's loads
+// measured slower), stage 2 per row (hh = h[row] in both halves).  Per 16-byte piece (8 elements): one
 // multiply spreads four sign bits to the top bits of the four bytes of a word
 // (bit i to bit 8i + 7; the partial products never overlap, so nothing
 // carries); PRMT in sign-replicating mode copies the top bit of byte 2p and
@@ -278,8 +282,9 @@ __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb
 // and 31 of that and flips them into the scales.  Rows past the matrix are
 // expanded from whatever bits they get: only output columns that are never
 // stored read them.
-__device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int n, uint2 bits,
-                                           bool per_k, uint32_t hh) {
+template <bool kGlobalG>
+__device__ __forceinline__ void expand_row(uint32_t b_smem, const __half* gk, uint32_t g_smem, int n,
+                                           uint2 bits, bool per_k, uint32_t hh) {
     // 16-byte piece c of row n sits at slot c ^ (n & 7) of the row's 128 bytes
     const uint32_t rowx = (uint32_t)(n >> 3) * 1024u + (uint32_t)(n & 7) * 144u;
 #pragma unroll
@@ -288,13 +293,15 @@ __device__ __forceinline__ void expand_row(uint32_t b_smem, uint32_t g_smem, int
         const uint32_t byte = c & 3 ? (word >> (8 * (c & 3))) & 0xFFu : word & 0xFFu;
         const uint32_t slo = (byte & 0xFu) * 0x10204080u;
         const uint32_t shi = (byte >> 4) * 0x10204080u;
-        uint4 base;
+        uint4 base = make_uint4(hh, hh, hh, hh);
         if (per_k) {
-            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(base.x), "=r"(base.y), "=r"(base.z), "=r"(base.w)
-                         : "r"(g_smem + 16u * (uint32_t)c));
-        } else {
-            base = make_uint4(hh, hh, hh, hh);
+            if (kGlobalG) {
+                base = __ldg(reinterpret_cast<const uint4*>(gk) + c);
+            } else {
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(base.x), "=r"(base.y), "=r"(base.z), "=r"(base.w)
+                             : "r"(g_smem + 16u * (uint32_t)c));
+            }
         }
         const uint32_t o0 = base.x ^ (prmt(slo, 0u, 0x9988u) & 0x80008000u);
         const uint32_t o1 = base.y ^ (prmt(slo, 0u, 0xBBAAu) & 0x80008000u);
@@ -467,7 +474,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const uint32_t fb = smem_u32(&ctl->full_a[s]);
                     const int kcol = acol(r, kb);
                     const uint32_t sa = base + s * kStageBytes;
-                    if (!r.stage2) {
+                    if (MT == 2 && !r.stage2) {   // the g slice, for the expansion (see expand_row)
                         const int kloc = kcol - (kb / r.kb_per_seg) * g.k_seg_len;
                         mbar_expect_tx(fb, MT * kABytes + kGBytes);
                         bulk_load(base + S::kOffG + s * kGBytes, g.bscale[r.nseg] + kloc, kGBytes, fb);
@@ -757,12 +764,16 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     if (kb >= n_kb) break;
                     const uint2 cur = nx[j];
                     if (kb + kBitsAhead < n_kb) nx[j] = fetch();
+                    // with one sub-tile the expansion reads g from memory and does not
+                    // wait for the A tile; with two it reads the copy that came with it
+                    constexpr bool kGlobalG = MT == 1;
                     bool w = wait_bar(ctl, &ctl->empty[s], ph ^ 1, err);
-                    if (w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, err);
+                    if (!kGlobalG && w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, err);
                     if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
                     const uint32_t sb = base + s * kStageBytes + MT * kABytes;
-                    expand_row(sb, base + S::kOffG + s * kGBytes, e, cur, g.stage == 1,
-                               (seg & 1) ? hh1 : hh0);
+                    const __half* gk = g.stage == 1 ? g.bscale[nseg] + (size_t)kin * kBlockK : nullptr;
+                    expand_row<kGlobalG>(sb, gk, base + S::kOffG + s * kGBytes, e, cur, g.stage == 1,
+                                         (seg & 1) ? hh1 : hh0);
                     fence_async_smem();              // make the stores visible to the tensor core
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&ctl->full_b[s]));
@@ -839,12 +850,33 @@ constexpr int kCachedSteps = 4;                               // steps kept in r
 // has several rows' loads in flight; a thread's first kCachedSteps steps of a
 // 16-bit x stay in registers for the second pass (rows up to 4096 elements are
 // read once).  The block also takes max_k |l_b[k]| of each branch itself.
+// The launch also clears what the GEMM kernel counts or adds into (the
+// workspace header, the per-M-block completion counts, the split tickets and,
+// when the second GEMM is split along K, y), so a call is two launches.
+struct PrepassZero {
+    int* i[3];
+    int ni[3];
+    float* f;          // 16-byte aligned
+    long long nf;
+};
+
 __global__ void __launch_bounds__(kPrepassThreads, 2) prefill_prepass_kernel(
     const void* __restrict__ x, int x_kind, int M, int in, int nb,
     const __half* __restrict__ g0, const __half* __restrict__ g1,
     const __half* __restrict__ l0, const __half* __restrict__ l1, int r,
-    __half* __restrict__ X16, float* __restrict__ row_sa, float* __restrict__ row_sc) {
+    __half* __restrict__ X16, float* __restrict__ row_sa, float* __restrict__ row_sc,
+    const PrepassZero z) {
     constexpr int kWarps = kPrepassThreads / 32, kGroupWarps = kRowThreads / 32;
+    {
+        const long long tid = (long long)blockIdx.x * kPrepassThreads + threadIdx.x;
+        const long long nth = (long long)gridDim.x * kPrepassThreads;
+        for (int k = 0; k < 3; ++k)
+            for (long long i = tid; i < z.ni[k]; i += nth) z.i[k][i] = 0;
+        const long long n4 = z.nf / 4;
+        for (long long i = tid; i < n4; i += nth)
+            reinterpret_cast<float4*>(z.f)[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (long long i = 4 * n4 + tid; i < z.nf; i += nth) z.f[i] = 0.0f;
+    }
     __shared__ float red[kWarps][3];
     __shared__ float lred[kWarps][2];
     const int grp = threadIdx.x / kRowThreads, t = threadIdx.x % kRowThreads;
@@ -1056,9 +1088,9 @@ static int pick_subtiles(const PrefillGemm* p, int grid) {
     return c[2] < c[1] ? 2 : 1;
 }
 
+// The K splits of both GEMMs for tiles of MT sub-tiles on `grid` CTAs (host only).
 template <int MT>
-static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const CUtensorMap& m2,
-                                int grid, cudaStream_t s) {
+static void plan_gemms(PrefillPlan& plan, int grid) {
     const int tiles1 = (int)gemm_tiles(plan.g[0], MT);
     // split stage 1 along K while it would leave SMs idle: up to kSplitMax parts of at
     // least 8 K blocks each, at most kSplitMaxParts parts in all
@@ -1071,7 +1103,7 @@ static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const 
     }
     plan.split = split;
     plan.n_tiles[0] = tiles1 * split;
-    // and stage 2 the same way (its parts reduce into y, zeroed below)
+    // and stage 2 the same way (its parts reduce into y, zeroed first)
     const int tiles2 = (int)gemm_tiles(plan.g[1], MT);
     const int n_kb2 = plan.g[1].n_kseg * (plan.g[1].k_seg_len / kBlockK);
     int split2 = 1;
@@ -1086,21 +1118,15 @@ static cudaError_t launch_gemms(PrefillPlan& plan, const CUtensorMap& m1, const 
     plan.split2 = split2;
     plan.n_tiles[1] = tiles2 * split2;
     plan.done_target = kEpiWarps * plan.g[0].n_nseg * ((plan.g[0].n_seg_rows + kTileN - 1) / kTileN);
-    const int blocks = (plan.g[0].M + MT * kTileM - 1) / (MT * kTileM);
-    cudaError_t e = cudaMemsetAsync(plan.done, 0, sizeof(int) * (size_t)blocks, s);
-    if (e != cudaSuccess) return e;
-    if (split > 1 &&
-        (e = cudaMemsetAsync(plan.tickets, 0, sizeof(int) * (size_t)tiles1 * kEpiWarps, s)) != cudaSuccess)
-        return e;
-    if (split2 > 1 &&
-        (e = cudaMemsetAsync(plan.g[1].y, 0,
-                             sizeof(float) * (size_t)plan.g[1].M * (size_t)plan.g[1].n_seg_rows, s)) !=
-            cudaSuccess)
-        return e;
+}
+
+template <int MT>
+static cudaError_t launch_gemms(const PrefillPlan& plan, const CUtensorMap& m1,
+                                const CUtensorMap& m2, int grid, cudaStream_t s) {
     // the split instantiations cost registers, so shapes that split nothing run without them
-    if (split2 > 1)
+    if (plan.split2 > 1)
         prefill_gemm_kernel<MT, true, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
-    else if (split > 1)
+    else if (plan.split > 1)
         prefill_gemm_kernel<MT, true, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
     else
         prefill_gemm_kernel<MT, false, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
@@ -1130,16 +1156,6 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         partial = reinterpret_cast<float*>(ws + off);
         tickets = reinterpret_cast<int*>(ws + off + (size_t)kSplitMaxParts * kEpiWarps * kPartFloats * sizeof(float));
     }
-
-    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s);
-    if (e != cudaSuccess) return e;
-    const __half* l1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].l);
-    const __half* g1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].g);
-    prefill_prepass_kernel<<<(unsigned)((M + kPrepassRows - 1) / kPrepassRows), kPrepassThreads, 0,
-                             s>>>(x, x_kind, (int)M, (int)in, nb,
-                                  reinterpret_cast<const __half*>(br[0].g), g1,
-                                  reinterpret_cast<const __half*>(br[0].l), l1, (int)r, X16, sa, sc);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     PrefillPlan plan = {};
     plan.done = done;
@@ -1181,8 +1197,31 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         p.row_sa = sa; p.row_sc = sc; p.T = nullptr; p.y = y; p.err = &hdr->error;
     }
     const int grid = device_sm_count();
-    return pick_subtiles(plan.g, grid) == 2 ? launch_gemms<2>(plan, amap1, amap2, grid, s)
-                                            : launch_gemms<1>(plan, amap1, amap2, grid, s);
+    const int mt = pick_subtiles(plan.g, grid);
+    if (mt == 2) plan_gemms<2>(plan, grid);
+    else plan_gemms<1>(plan, grid);
+
+    // pre-pass (and the clearing the GEMM kernel relies on), then both GEMMs
+    PrepassZero z = {};
+    z.i[0] = reinterpret_cast<int*>(hdr);
+    z.ni[0] = (int)(sizeof(WsHeader) / sizeof(int));
+    z.i[1] = done;
+    z.ni[1] = (int)((M + mt * kTileM - 1) / (mt * kTileM));
+    z.i[2] = tickets;
+    z.ni[2] = plan.split > 1 ? (int)(plan.n_tiles[0] / plan.split) * kEpiWarps : 0;
+    z.f = plan.split2 > 1 ? y : nullptr;
+    z.nf = plan.split2 > 1 ? (long long)M * out : 0;
+    const long long row_blocks = (M + kPrepassRows - 1) / kPrepassRows;
+    const long long zero_blocks = std::min<long long>(4LL * grid, (z.nf / 4 + kPrepassThreads - 1) / kPrepassThreads);
+    const __half* l1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].l);
+    const __half* g1 = reinterpret_cast<const __half*>(br[nb > 1 ? 1 : 0].g);
+    prefill_prepass_kernel<<<(unsigned)std::max(row_blocks, zero_blocks), kPrepassThreads, 0, s>>>(
+        x, x_kind, (int)M, (int)in, nb, reinterpret_cast<const __half*>(br[0].g), g1,
+        reinterpret_cast<const __half*>(br[0].l), l1, (int)r, X16, sa, sc, z);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return mt == 2 ? launch_gemms<2>(plan, amap1, amap2, grid, s)
+                   : launch_gemms<1>(plan, amap1, amap2, grid, s);
 }
 
 }  // namespace lb
