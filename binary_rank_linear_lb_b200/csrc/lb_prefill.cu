@@ -58,7 +58,6 @@ constexpr int kSplitMaxParts = 160;               // stage-1 tile parts the spli
 constexpr int kSplitMax = 4;                      // K parts of one stage-1 tile (the last one folds the others)
 
 constexpr int kEpiBytes = 32 * 128;                // per-warp epilogue staging: 32 rows x 128 bytes
-constexpr int kPrefetchAhead = 6;                 // K blocks of A pulled into L2 ahead of the TMA loads
 constexpr int kBitsAhead = 4;                     // K blocks of sign bits held in registers ahead
 
 // Shared memory of one CTA, from the 1024-aligned base: the pipeline stages
@@ -114,12 +113,6 @@ __device__ __forceinline__ bool wait_bar(Ctl* c, uint64_t* bar, uint32_t parity,
             return false;
         }
     }
-}
-
-// Pull one A box into L2 (no shared-memory destination, no barrier).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 :: "l"(map), "r"(x), "r"(y) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -412,40 +405,15 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp == kTmaWarp) {
-        // ---------------- TMA producer for A (and the g slice of stage 1).  A
-        // boxes kPrefetchAhead K blocks ahead (into the next tile at the end of
-        // one) are pulled into L2 first, so the loads find them there; a
-        // stage-2 tile's boxes only once its rows of T are complete.
+        // ---------------- TMA producer for A (and, with two sub-tiles, the g slice
+        // of stage 1); a stage-2 tile's boxes only once its rows of T are complete.
+        // (A is not pulled into L2 ahead of the loads: the pre-pass has just
+        // written it, and the prefetches only held up the TMA unit.)
         if (lane == 0) {
             auto acol = [](const TileRef& r, int kb) {
                 const int ks = kb / r.kb_per_seg;
                 return ks * r.g->k_seg_len + (kb - ks * r.kb_per_seg) * kBlockK;
             };
-            auto ready = [&](const TileRef& r) {
-                return !r.stage2 ||
-                       *reinterpret_cast<volatile const int*>(plan.done + r.mb) >= plan.done_target;
-            };
-            auto prefetch = [&](const TileRef& cur, int t, int kb) {
-                int pb = kb + kPrefetchAhead;
-                TileRef r = cur;
-                if (pb >= cur.kb1) {
-                    t += gridDim.x;
-                    if (t >= n_tiles) return;
-                    r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
-                    pb = r.kb0 + (pb - cur.kb1);
-                    if (pb >= r.kb1 || !ready(r)) return;
-                }
-#pragma unroll
-                for (int j = 0; j < MT; ++j)
-                    if ((r.mb * MT + j) * kTileM < r.g->M)
-                        tma_prefetch_2d(r.map, acol(r, pb), (r.mb * MT + j) * kTileM);
-            };
-            if (blockIdx.x < n_tiles) {
-                const TileRef r0 = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, blockIdx.x);
-                if (ready(r0))
-                    for (int kb = r0.kb0; kb < r0.kb0 + kPrefetchAhead && kb < r0.kb1; ++kb)
-                        prefetch(r0, blockIdx.x, kb - kPrefetchAhead);
-            }
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !ctl->abort; t += gridDim.x) {
                 const TileRef r = tile_ref<SPLIT, SPLIT2>(plan, &amap1, &amap2, t);
@@ -467,7 +435,6 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                 }
                 for (int kb = r.kb0; kb < r.kb1; ++kb, ++it) {
-                    prefetch(r, t, kb);
                     const int s = it % kStages;
                     const uint32_t par = ((it / kStages) & 1) ^ 1;
                     if (!wait_bar(ctl, &ctl->empty[s], par, err)) break;
