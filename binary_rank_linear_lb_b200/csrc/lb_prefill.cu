@@ -219,6 +219,11 @@ struct PrefillGemm {
     const float* row_sa;                             // [M] 2^a_m (stage 1 divides it out)
     const float* row_sc;                             // [M] 2^c_m
     __half* T;                                       // stage 1 output [M][n_nseg * n_seg_rows]
+    int n_cat;                                       // stage 1 with one sub-tile: the N tiles run
+                                                     // over the segments back to back (row R of
+                                                     // segment R / n_seg_rows), so two branches of
+                                                     // low rank share a tile instead of half-filling
+                                                     // one each
     float* y;                                        // stage 2 output [M][n_seg_rows]
     int* err;
 };
@@ -247,14 +252,34 @@ struct PrefillPlan {
     int* tickets;        // [tile][epilogue warp], zeroed per call
     int split2;          // K parts of a stage-2 tile (1: no split; else y, zeroed first,
                          // takes each part's sums by reduction)
+    int y_tma;           // stage 2 writes y with tensor stores (ymap); needs split2 == 1,
+                         // a 16-byte aligned y and out % 4 == 0
 };
 
 namespace {
 
+// Rows one N tile list runs over, and how many such lists (segments) a GEMM has.
+__host__ __device__ __forceinline__ int tile_span(const PrefillGemm& g) {
+    return g.n_cat ? g.n_nseg * g.n_seg_rows : g.n_seg_rows;
+}
+__host__ __device__ __forceinline__ int tile_segs(const PrefillGemm& g) {
+    return g.n_cat ? 1 : g.n_nseg;
+}
+
+// Segment and row within it of row n of tile list nseg (n_cat: the segment
+// holding row n of the concatenation; past its end, segment 0 and row
+// n_seg_rows, which reads as zeros).
+__device__ __forceinline__ void seg_row(const PrefillGemm& g, int nseg, int n, int& s, int& rin) {
+    if (!g.n_cat) { s = nseg; rin = n; return; }
+    s = n / g.n_seg_rows;
+    rin = n - s * g.n_seg_rows;
+    if (s >= g.n_nseg) { s = 0; rin = g.n_seg_rows; }
+}
+
 __device__ __forceinline__ void tile_coords(const PrefillGemm& g, int t, int& mb, int& nseg,
                                             int& nt) {
-    const int nt_per_seg = (g.n_seg_rows + kTileN - 1) / kTileN;
-    const int n_tiles = g.n_nseg * nt_per_seg;
+    const int nt_per_seg = (tile_span(g) + kTileN - 1) / kTileN;
+    const int n_tiles = tile_segs(g) * nt_per_seg;
     mb = t / n_tiles;
     const int r = t - mb * n_tiles;
     nseg = r / nt_per_seg;
@@ -368,6 +393,7 @@ template <int MT, bool SPLIT, bool SPLIT2>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const __grid_constant__ CUtensorMap amap2,
+                    const __grid_constant__ CUtensorMap ymap,
                     const __grid_constant__ PrefillPlan plan) {
     using S = Shape<MT>;
     constexpr int kStages = S::kStages, kStageBytes = S::kStageBytes;
@@ -494,6 +520,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
         // the warp's staging buffer (16-byte piece c of row r at slot c ^ (r & 7),
         // conflict-free both ways) and read back so that every store
         // instruction writes whole row segments (128 bytes of y, 64 of T).
+        // The staging layout is the tensor map's 128-byte swizzle, so with
+        // plan.y_tma a chunk of y leaves as one tensor store issued by lane 0
+        // (rows and columns past y clipped by the map), and the warp goes on
+        // to the next chunk while the TMA unit writes it.
         const int q = warp & 3, hw = warp >> 2;
         const int sub = MT == 2 ? hw : 0;
         const int c_begin = MT == 2 ? 0 : hw * (kTileN / 2);
@@ -516,8 +546,12 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             const float sc = mok ? __ldg(g.row_sc + m) : 1.0f;
             // (stage 1) lane p < 4 holds piece p of the next chunk's l
             uint4 lnext = make_uint4(0u, 0u, 0u, 0u);
-            if (g.stage == 1 && lane < 4 && nt * kTileN + c_begin < g.n_seg_rows)
-                lnext = load_l8(g, nseg, nt * kTileN + c_begin, lane);
+            const int span = tile_span(g);
+            if (g.stage == 1 && lane < 4 && nt * kTileN + c_begin < span) {
+                int ls, ln;
+                seg_row(g, nseg, nt * kTileN + c_begin, ls, ln);
+                lnext = load_l8(g, ls, ln, lane);
+            }
             // every lane waits; the warp stops together so the .sync.aligned loads stay converged
             if (!__all_sync(0xffffffffu, wait_bar(ctl, &ctl->acc_full[buf],
                                                   (uint32_t)(tl / S::kBufs) & 1, err)))
@@ -558,19 +592,30 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     const float* p0 = plan.partial + (size_t)r.t * plan.split * kEpiWarps * kPartFloats +
                                       (size_t)warp * kPartFloats;
                     for (int h = 0; h < (c_end - c_begin) / 16; ++h) {
+                        // every other part's piece is requested before any is added, so
+                        // a half chunk costs one round trip to L2, not one per part
+                        float4 o[kSplitMax - 1][4];
+#pragma unroll
+                        for (int q = 0; q < kSplitMax - 1; ++q) {
+                            const int p = q < r.part ? q : q + 1;   // the parts other than this one
+                            const bool use = p < plan.split && mok;
+                            const float* pc = p0 + (size_t)p * kEpiWarps * kPartFloats + h * 512;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                o[q][i] = use ? __ldcg(reinterpret_cast<const float4*>(pc + (i * 32 + lane) * 4))
+                                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        }
                         float v[16];
                         __syncwarp();
                         tmem_ld16(tacc + (uint32_t)(c_begin + 16 * h), v);
-                        for (int p = 0; p < plan.split && mok; ++p) {
-                            if (p == r.part) continue;
-                            const float* pc = p0 + (size_t)p * kEpiWarps * kPartFloats + h * 512;
+#pragma unroll
+                        for (int q = 0; q < kSplitMax - 1; ++q) {
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                const float4 o = __ldcg(reinterpret_cast<const float4*>(pc + (i * 32 + lane) * 4));
-                                v[4 * i] += o.x;
-                                v[4 * i + 1] += o.y;
-                                v[4 * i + 2] += o.z;
-                                v[4 * i + 3] += o.w;
+                                v[4 * i] += o[q][i].x;
+                                v[4 * i + 1] += o[q][i].y;
+                                v[4 * i + 2] += o[q][i].z;
+                                v[4 * i + 3] += o[q][i].w;
                             }
                         }
                         tmem_st16(tacc + (uint32_t)(c_begin + 16 * h), v);
@@ -582,8 +627,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                 float v[32];
                 __syncwarp();
                 tmem_ld32(tacc + (uint32_t)c0, v);
-                const int n0 = nt * kTileN + c0;       // row within the N segment
-                if (n0 >= g.n_seg_rows) continue;      // warp-uniform
+                const int n0 = nt * kTileN + c0;       // row within the N tile list
+                if (n0 >= span) continue;              // warp-uniform
                 if (g.stage == 1) {
                     // T = l * t * 2^c with t = D / 2^a, fp16, 4 pieces of 16 bytes per row.
                     // This chunk's l goes to the half of row 0 of the staging buffer
@@ -594,8 +639,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                                      :: "r"(lbuf + 16u * (uint32_t)lane), "r"(lnext.x), "r"(lnext.y),
                                         "r"(lnext.z), "r"(lnext.w) : "memory");
-                        if (c0 + 32 < c_end && n0 + 32 < g.n_seg_rows)
-                            lnext = load_l8(g, nseg, n0 + 32, lane);
+                        if (c0 + 32 < c_end && n0 + 32 < span) {
+                            int ls, ln;      // (a chunk never straddles two segments: r % 32 == 0)
+                            seg_row(g, nseg, n0 + 32, ls, ln);
+                            lnext = load_l8(g, ls, ln, lane);
+                        }
                     }
                     __syncwarp();
 #pragma unroll
@@ -627,25 +675,39 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
                                      : "r"(stg + (uint32_t)rr * 128u + (uint32_t)((cc ^ (rr & 7)) * 16)));
-                        if (m0 + rr < g.M && col < g.n_seg_rows) {
-                            __half* dst = g.T + (size_t)(m0 + rr) * ldt + (size_t)nseg * g.n_seg_rows + col;
-                            if (col + 8 <= g.n_seg_rows) {
+                        if (m0 + rr < g.M && col < span) {
+                            __half* dst = g.T + (size_t)(m0 + rr) * ldt +
+                                          (size_t)(g.n_cat ? 0 : nseg) * g.n_seg_rows + col;
+                            if (col + 8 <= span) {
                                 *reinterpret_cast<uint4*>(dst) = o;
                             } else {
                                 const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-                                for (int e = 0; e < 8 && col + e < g.n_seg_rows; ++e)
+                                for (int e = 0; e < 8 && col + e < span; ++e)
                                     reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(ow[e >> 1] >> (16 * (e & 1)));
                             }
                         }
                     }
                 } else {
                     // y = D / 2^c, fp32, 8 pieces of 16 bytes per row
+                    if (plan.y_tma) {   // the previous chunk's store has read the buffer
+                        if (lane == 0) bulk_wait_read();
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
                                      :: "r"(my_row + (uint32_t)((c ^ (lane & 7)) * 16)),
                                         "f"(v[4 * c] * f), "f"(v[4 * c + 1] * f), "f"(v[4 * c + 2] * f),
                                         "f"(v[4 * c + 3] * f) : "memory");
+                    if (plan.y_tma) {
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0 && m0 < g.M) {   // (rows past M: nothing to store)
+                            tma_store_2d(&ymap, stg, n0, m0);
+                            bulk_commit();
+                        }
+                        continue;
+                    }
                     __syncwarp();
                     const int cc = lane & 7;
                     const int col = n0 + 4 * cc;
@@ -690,6 +752,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                                  :: "l"(plan.done + mb) : "memory");
             }
         }
+        if (plan.y_tma && lane == 0) bulk_wait_all();   // this warp's tensor stores are done
     } else if (warp >= kExpandWarp0) {
         // ---------------- B producers: packed signs -> fp16 tile, one row per thread
         const int e = threadIdx.x - kExpandWarp0 * 32;
@@ -702,6 +765,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             const int nseg = r.nseg, nt = r.nt, kb_per_seg = r.kb_per_seg;
             const int n_kb = r.kb1 - r.kb0;          // K blocks of this tile (its part of K)
             const int row = nt * kTileN + e;
+            int bseg = nseg, brow = row;             // stage 1: this row's branch and row in it
+            if (g.stage == 1) seg_row(g, nseg, row, bseg, brow);
             uint32_t hh0 = 0u, hh1 = 0u;             // h[row] of each branch in both fp16 halves
             if (g.stage == 2 && row < g.n_seg_rows) {
                 const uint32_t h0 = __half_as_ushort(__ldg(g.bscale[0] + row));
@@ -716,7 +781,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
             const int seg0 = r.kb0 / kb_per_seg, kin0 = r.kb0 - seg0 * kb_per_seg;
             int fs = seg0, fk = kin0;
             auto fetch = [&]() {
-                const uint2 v = load_bits(g, g.stage == 1 ? nseg : fs, row, fk);
+                const uint2 v = g.stage == 1 ? load_bits(g, bseg, brow, fk) : load_bits(g, fs, row, fk);
                 if (++fk == kb_per_seg) { fk = 0; ++fs; }
                 return v;
             };
@@ -738,7 +803,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap amap1,
                     if (!kGlobalG && w && g.stage == 1) w = wait_bar(ctl, &ctl->full_a[s], ph, err);
                     if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
                     const uint32_t sb = base + s * kStageBytes + MT * kABytes;
-                    const __half* gk = g.stage == 1 ? g.bscale[nseg] + (size_t)kin * kBlockK : nullptr;
+                    const __half* gk = g.stage == 1 ? g.bscale[bseg] + (size_t)kin * kBlockK : nullptr;
                     expand_row<kGlobalG>(sb, gk, base + S::kOffG + s * kGBytes, e, cur, g.stage == 1,
                                          (seg & 1) ? hh1 : hh0);
                     fence_async_smem();              // make the stores visible to the tensor core
@@ -963,6 +1028,20 @@ EncodeTiled get_encode() {
     return fn;
 }
 
+// Row-major fp32 [rows][cols] (cols % 4 == 0, 16-byte aligned) with a 32 x 32
+// box and the 128-byte swizzle: one epilogue chunk of y.
+bool make_ymap(CUtensorMap* map, float* ptr, int rows, int cols) {
+    EncodeTiled enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major fp16 [rows][cols] with a 64 x 128 box and the 128-byte swizzle.
 bool make_amap(CUtensorMap* map, const __half* ptr, int rows, int cols) {
     EncodeTiled enc = get_encode();
@@ -1028,7 +1107,7 @@ bool prefill_shape_ok(int64_t M, int64_t in, int64_t out, int64_t r) {
 // costing kTile2Cost one-sub-tile tiles.  LB_PREFILL_SUBTILES=1 or 2 in the
 // environment (read on every call) fixes the choice; both give the same result.
 static long long gemm_tiles(const PrefillGemm& p, int mt) {
-    return (long long)p.n_nseg * ((p.n_seg_rows + kTileN - 1) / kTileN) *
+    return (long long)tile_segs(p) * ((tile_span(p) + kTileN - 1) / kTileN) *
            ((p.M + mt * kTileM - 1) / (mt * kTileM));
 }
 
@@ -1084,19 +1163,20 @@ static void plan_gemms(PrefillPlan& plan, int grid) {
     }
     plan.split2 = split2;
     plan.n_tiles[1] = tiles2 * split2;
-    plan.done_target = kEpiWarps * plan.g[0].n_nseg * ((plan.g[0].n_seg_rows + kTileN - 1) / kTileN);
+    plan.done_target = kEpiWarps * tile_segs(plan.g[0]) * ((tile_span(plan.g[0]) + kTileN - 1) / kTileN);
 }
 
 template <int MT>
 static cudaError_t launch_gemms(const PrefillPlan& plan, const CUtensorMap& m1,
-                                const CUtensorMap& m2, int grid, cudaStream_t s) {
+                                const CUtensorMap& m2, const CUtensorMap& ym, int grid,
+                                cudaStream_t s) {
     // the split instantiations cost registers, so shapes that split nothing run without them
     if (plan.split2 > 1)
-        prefill_gemm_kernel<MT, true, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+        prefill_gemm_kernel<MT, true, true><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, ym, plan);
     else if (plan.split > 1)
-        prefill_gemm_kernel<MT, true, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+        prefill_gemm_kernel<MT, true, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, ym, plan);
     else
-        prefill_gemm_kernel<MT, false, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, plan);
+        prefill_gemm_kernel<MT, false, false><<<grid, kPrefillThreads, Shape<MT>::kSmem, s>>>(m1, m2, ym, plan);
     return cudaGetLastError();
 }
 
@@ -1165,6 +1245,13 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
     }
     const int grid = device_sm_count();
     const int mt = pick_subtiles(plan.g, grid);
+    // with one sub-tile (the expansion then reads g per row from memory) the
+    // branches of stage 1 share N tiles when that takes fewer of them
+    if (mt == 1 && nb > 1) {
+        PrefillGemm cat = plan.g[0];
+        cat.n_cat = 1;
+        if (gemm_tiles(cat, 1) < gemm_tiles(plan.g[0], 1)) plan.g[0].n_cat = 1;
+    }
     if (mt == 2) plan_gemms<2>(plan, grid);
     else plan_gemms<1>(plan, grid);
 
@@ -1187,8 +1274,12 @@ cudaError_t launch_prefill(const void* x, int x_kind, int64_t M, int64_t in, int
         reinterpret_cast<const __half*>(br[0].l), l1, (int)r, X16, sa, sc, z);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return mt == 2 ? launch_gemms<2>(plan, amap1, amap2, grid, s)
-                   : launch_gemms<1>(plan, amap1, amap2, grid, s);
+    // y by tensor stores when nothing reduces into it and the map can describe it
+    CUtensorMap ymap = {};
+    plan.y_tma = plan.split2 == 1 && out % 4 == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0 &&
+                 make_ymap(&ymap, y, (int)M, (int)out);
+    return mt == 2 ? launch_gemms<2>(plan, amap1, amap2, ymap, grid, s)
+                   : launch_gemms<1>(plan, amap1, amap2, ymap, grid, s);
 }
 
 }  // namespace lb
