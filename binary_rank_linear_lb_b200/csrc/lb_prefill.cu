@@ -881,7 +881,8 @@ constexpr int kCachedSteps = 4;                               // steps kept in r
 // One block takes kPrepassRows rows (kRowThreads threads each), so that an SM
 // has several rows' loads in flight; a thread's first kCachedSteps steps of a
 // 16-bit x stay in registers for the second pass (rows up to 4096 elements are
-// read once).  The block also takes max_k |l_b[k]| of each branch itself.
+// read once), and all of them are requested before the first is used.  The
+// block also takes max_k |l_b[k]| and max_k |g_b[k]| of each branch itself.
 // The launch also clears what the GEMM kernel counts or adds into (the
 // workspace header, the per-M-block completion counts, the split tickets and,
 // when the second GEMM is split along K, y), so a call is two launches.
@@ -909,74 +910,88 @@ __global__ void __launch_bounds__(kPrepassThreads, 2) prefill_prepass_kernel(
             reinterpret_cast<float4*>(z.f)[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         for (long long i = 4 * n4 + tid; i < z.nf; i += nth) z.f[i] = 0.0f;
     }
-    __shared__ float red[kWarps][3];
+    __shared__ float red[kWarps][2];
     __shared__ float lred[kWarps][2];
     const int grp = threadIdx.x / kRowThreads, t = threadIdx.x % kRowThreads;
     const int m = blockIdx.x * kPrepassRows + grp;
     const bool row_ok = m < M;
     const size_t row = (size_t)(row_ok ? m : 0) * in;
-    // max |l| of each branch, over the block (its loads go out with x's)
-    float lm0 = 0.0f, lm1 = 0.0f;
+    // the row's first steps of x, all requested before any is used
+    uint4 xc[kCachedSteps];
+#pragma unroll
+    for (int c = 0; c < kCachedSteps; ++c) {
+        const int j0 = c * kRowStep + 8 * t;
+        xc[c] = row_ok && j0 < in ? raw8_x(x, x_kind, row + j0) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // max |l| and max |g| of each branch, over the block (their loads go out with x's)
+    float lm0 = 0.0f, lm1 = 0.0f, gm0 = 0.0f, gm1 = 0.0f;
     for (int k = threadIdx.x; k < r; k += kPrepassThreads) {
         lm0 = fmaxf(lm0, fabsf(__half2float(__ldg(l0 + k))));
         if (nb > 1) lm1 = fmaxf(lm1, fabsf(__half2float(__ldg(l1 + k))));
     }
-    float mx = 0.0f, s0 = 0.0f, s1 = 0.0f;
-    uint4 xc[kCachedSteps];
-    auto step = [&](int j0, uint4& raw) {
-        float xv[8], gv[8], hv[8];
-        raw = raw8_x(x, x_kind, row + j0);
-        if (x_kind == VK_X_F32) load8_x(x, x_kind, row + j0, xv);
-        else cvt8_x(raw, x_kind, xv);
-        load8_h(g0, j0, gv);
-        if (nb > 1) load8_h(g1, j0, hv);
+    for (int k = 8 * threadIdx.x; k < in; k += 8 * kPrepassThreads) {
+        float gv[8];
+        load8_h(g0, k, gv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gm0 = fmaxf(gm0, fabsf(gv[i]));
+        if (nb > 1) {
+            load8_h(g1, k, gv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gm1 = fmaxf(gm1, fabsf(gv[i]));
+        }
+    }
+    // max |x| and sum |x| of the row
+    float mx = 0.0f, sx = 0.0f;
+    auto take = [&](const float (&xv)[8]) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             mx = fmaxf(mx, fabsf(xv[i]));
-            s0 += fabsf(xv[i] * gv[i]);
-            if (nb > 1) s1 += fabsf(xv[i] * hv[i]);
+            sx += fabsf(xv[i]);
         }
     };
 #pragma unroll
     for (int c = 0; c < kCachedSteps; ++c) {
         const int j0 = c * kRowStep + 8 * t;
-        if (row_ok && j0 < in) step(j0, xc[c]);
+        if (!row_ok || j0 >= in) continue;
+        float xv[8];
+        if (x_kind == VK_X_F32) load8_x(x, x_kind, row + j0, xv);
+        else cvt8_x(xc[c], x_kind, xv);
+        take(xv);
     }
     for (int j0 = kCachedSteps * kRowStep + 8 * t; row_ok && j0 < in; j0 += kRowStep) {
-        uint4 raw;
-        step(j0, raw);
+        float xv[8];
+        load8_x(x, x_kind, row + j0, xv);
+        take(xv);
     }
     const int w = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        sx += __shfl_xor_sync(0xffffffffu, sx, o);
         lm0 = fmaxf(lm0, __shfl_xor_sync(0xffffffffu, lm0, o));
         lm1 = fmaxf(lm1, __shfl_xor_sync(0xffffffffu, lm1, o));
+        gm0 = fmaxf(gm0, __shfl_xor_sync(0xffffffffu, gm0, o));
+        gm1 = fmaxf(gm1, __shfl_xor_sync(0xffffffffu, gm1, o));
     }
     if ((threadIdx.x & 31) == 0) {
-        red[w][0] = mx; red[w][1] = s0; red[w][2] = s1;
-        lred[w][0] = lm0; lred[w][1] = lm1;
+        red[w][0] = mx; red[w][1] = sx;
+        lred[w][0] = lm0 * gm0; lred[w][1] = lm1 * gm1;
     }
     __syncthreads();
-    float M0 = 0.0f, L0 = 0.0f, L1 = 0.0f, lmax0 = 0.0f, lmax1 = 0.0f;
-    for (int v = 0; v < kWarps; ++v) {
-        lmax0 = fmaxf(lmax0, lred[v][0]);
-        lmax1 = fmaxf(lmax1, lred[v][1]);
-    }
+    float M0 = 0.0f, L0 = 0.0f, lg = 0.0f;
+    for (int v = 0; v < kWarps; ++v) lg = fmaxf(lg, fmaxf(lred[v][0], nb > 1 ? lred[v][1] : 0.0f));
     for (int v = grp * kGroupWarps; v < (grp + 1) * kGroupWarps; ++v) {
         M0 = fmaxf(M0, red[v][0]);
         L0 += red[v][1];
-        L1 += red[v][2];
     }
     if (!row_ok) return;
     // 2^a: the largest power of two with max|x| * 2^a < 2^15
     float sa = 1.0f;
     if (M0 > 0.0f && isfinite(M0)) sa = exp2f(fminf(fmaxf(14.0f - floorf(log2f(M0)), -126.0f), 126.0f));
-    // 2^c: the largest power of two with bound * 2^c <= 2^15 (< 65504); the
-    // bound is padded by 1/64 for fp32 rounding in the sums.
-    const float bound = fmaxf(L0 * lmax0, nb > 1 ? L1 * lmax1 : 0.0f) * (1.0f + 1.0f / 64);
+    // 2^c: the largest power of two with bound * 2^c <= 2^15 (< 65504), where
+    // |T| <= max|l| max|g| sum|x|; the bound is padded by 1/64 for fp32 rounding
+    // in the sums.
+    const float bound = L0 * lg * (1.0f + 1.0f / 64);
     float sc = 1.0f;
     if (bound > 0.0f && isfinite(bound))
         sc = exp2f(fminf(fmaxf(15.0f - ceilf(log2f(bound)), -126.0f), 126.0f));
