@@ -242,23 +242,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         :: "r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y) : "memory");
 }
 
-// Tensor store of the box at (x, y) from shared memory (bulk async-group of the
-// issuing thread); the shared source must be made visible to the async proxy
-// first (fence.proxy.async) and stay untouched until wait_group.read.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 :: "l"(map), "r"(src), "r"(x), "r"(y) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read() {      // sources of earlier stores reusable
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {       // earlier stores complete
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // ------------------------------------------------------------ host helpers
 int device_sm_count();               // SMs of the current device (cached per device)
 bool device_is_sm100();
