@@ -59,8 +59,8 @@ L2_BYTES = 126 * 1024 * 1024
 # captured, or 0 for a single linear).
 MEASURED_TRAFFIC = {
     "stack70b-1.0": ("fa65e09bcb813709", 214949888 + 3215872, 2),
-    "prefill-gate7b-1.0-M4096": ("7aaa8dd0c2c8c3e3", 53419008 + 144395008, 0),
-    "prefill-gate7b-0.1-M4096": ("7aaa8dd0c2c8c3e3", 34847232 + 140641536, 0),
+    "prefill-gate7b-1.0-M4096": ("38ee1e7d648a507e", 53460736 + 144450560, 0),
+    "prefill-gate7b-0.1-M4096": ("38ee1e7d648a507e", 35022336 + 138610688, 0),
 }
 KERNEL_SOURCES = {
     "stack_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),
