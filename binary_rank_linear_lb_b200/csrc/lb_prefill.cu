@@ -895,8 +895,9 @@ constexpr int kRowThreads = kPrepassThreads / kPrepassRows;   // threads per row
 constexpr int kRowStep = 8 * kRowThreads;                     // elements of a row per step
 constexpr int kCachedSteps = 4;                               // steps kept in registers
 
-// One block takes kPrepassRows rows (kRowThreads threads each), so that an SM
-// has several rows' loads in flight; a thread's first kCachedSteps steps of a
+// One block takes kPrepassRows rows (kRowThreads threads each), three blocks
+// to an SM (40 registers a thread), so that an SM has several rows' loads in
+// flight; a thread's first kCachedSteps steps of a
 // 16-bit x stay in registers for the second pass (rows up to 4096 elements are
 // read once), and all of them are requested before the first is used.  The
 // block also takes max_k |l_b[k]| and max_k |g_b[k]| of each branch itself.
@@ -910,7 +911,7 @@ struct PrepassZero {
     long long nf;
 };
 
-__global__ void __launch_bounds__(kPrepassThreads, 2) prefill_prepass_kernel(
+__global__ void __launch_bounds__(kPrepassThreads, 3) prefill_prepass_kernel(
     const void* __restrict__ x, int x_kind, int M, int in, int nb,
     const __half* __restrict__ g0, const __half* __restrict__ g1,
     const __half* __restrict__ l0, const __half* __restrict__ l1, int r,
