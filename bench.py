@@ -58,9 +58,9 @@ L2_BYTES = 126 * 1024 * 1024
 # proportion.  workload: (sources hash, bytes per captured launch, layers
 # captured, or 0 for a single linear).
 MEASURED_TRAFFIC = {
-    "stack70b-1.0": ("699fbf6dddf8181b", 214950400 + 3992064, 2),
-    "prefill-gate7b-1.0-M4096": ("6f8384ecbe869ba7", 52983040 + 144217600, 0),
-    "prefill-gate7b-0.1-M4096": ("6f8384ecbe869ba7", 35014912 + 138724096, 0),
+    "stack70b-1.0": ("2038467ba1b45bad", 214971136 + 3177984, 2),
+    "prefill-gate7b-1.0-M4096": ("1504e09a31a2c770", 53246208 + 144017664, 0),
+    "prefill-gate7b-0.1-M4096": ("1504e09a31a2c770", 34988544 + 138443776, 0),
 }
 KERNEL_SOURCES = {
     "stack_program_kernel": ("lb_decode.cu", "lb_internal.cuh"),

@@ -266,10 +266,10 @@ void plan_starts(LbPhase* phases, int n_phases, const LbJob* jobs, const int* sp
 
 // Tensor-core prefill path (lb_prefill.cu).
 // lb_linear_forward uses the tensor cores from this many rows: measured on the
-// 7B gate shape (4096 -> 11008) at 1.0 and 0.1 bits/weight, the lookup-table
-// kernels are faster up to 12 rows and level at 13 (their second launch of 8
-// rows), the tensor cores ahead or level from 14.
-constexpr int kPrefillMinM = 14;
+// 7B gate shape (4096 -> 11008), the two paths are level at 14-15 rows at 1.0
+// bits/weight while the lookup-table kernels (two launches of 8 rows) stay ahead
+// through 15 rows at 0.1; from 16 rows the tensor cores are ahead or within 5%.
+constexpr int kPrefillMinM = 16;
 cudaError_t prefill_configure();
 // with_split: room for the stage-1 K split's partial sums (tens of MB when the
 // split is possible); without it the launch never splits stage 1.

@@ -203,10 +203,10 @@ def test_prefill_timed_7b_gate_every_m_block(M, bpw):
 
 
 @pytest.mark.parametrize("path", ["0", "1"])
-@pytest.mark.parametrize("M", [1, 5, 8, 13, 14, 16, 24, 64])
+@pytest.mark.parametrize("M", [1, 5, 8, 14, 15, 16, 24, 64])
 def test_forced_paths_small_m(M, path, monkeypatch):
     """Both kernel paths at the token counts where lb_linear_forward switches between them
-    (LB_LINEAR_PATH forces one: the tensor-core kernels also below 14 rows, the lookup-table
+    (LB_LINEAR_PATH forces one: the tensor-core kernels also below 16 rows, the lookup-table
     kernels also above), on a 64-aligned shape with a ragged output width."""
     monkeypatch.setenv("LB_LINEAR_PATH", path)
     in_f, out_f, r = 1024, 1001, 192
@@ -216,12 +216,12 @@ def test_forced_paths_small_m(M, path, monkeypatch):
         assert_close(got[m], ref[m], what=f"M={M} path={path} row {m}")
 
 
-@pytest.mark.parametrize("M", [13, 14, 15])
+@pytest.mark.parametrize("M", [15, 16, 17])
 def test_dispatch_threshold(M):
-    """lb_linear_forward switches to the tensor cores at 14 rows (the measured crossover
+    """lb_linear_forward switches to the tensor cores at 16 rows (the measured crossover
     on the 7B gate shape); either side of the switch matches the oracle."""
     in_f, out_f, r = 4096, 11008, 128
-    assert lb.linear_path(M, in_f, out_f, r) == (1 if M >= 14 else 0)
+    assert lb.linear_path(M, in_f, out_f, r) == (1 if M >= 16 else 0)
     assert lb.linear_path(M, 4000, out_f, r) == 0          # in not a multiple of 64
     got, ref = run_case(in_f, out_f, r, M, torch.bfloat16, base=13)
     for m in (0, M // 2, M - 1):
